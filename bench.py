@@ -1,0 +1,377 @@
+"""Benchmark of the mHC pre-map + post-map hot path (HC = 4) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload large] [--impl ours|reference]
+
+One step = one mhc_pre (norm, projection, gates, Sinkhorn, aggregate) plus one mhc_post over one
+batch of the workload (default: T=8192 tokens, H=7168, bf16; seeded synthetic inputs). The inputs
+(R = 470 MB) are larger than the 126 MB L2, so no flush is needed between steps. Each rank runs
+its own token shard (weak scaling, no data-path collective); rank 0 prints one JSON line with the
+whole-job tokens/s taken over the slowest rank.
+
+--impl reference times the fp64 CPU oracle (the only other implementation of this method here) on
+a bounded sample of the same workload, on this host's cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "mHC pre+post tokens/s and HBM GB/s (% of roofline), T=8192 H=7168 bf16"
+UNIT = "tokens/s"
+
+
+def pre_bytes(T, H):
+    """Algorithmic bytes of one pre-map call: R (8H) + y (2H) + pre/post/comb (96) per token, plus
+    hc_fn (4H x 24 fp32) and scale/base once."""
+    return T * (8 * H + 2 * H + 96) + 4 * H * 24 * 4 + 12 + 96
+
+
+def post_bytes(T, H):
+    """Algorithmic bytes of one post-map call: R (8H) + x (2H) + out (8H) + post/comb (80) per token."""
+    return T * (18 * H + 80)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling during the timed region (median SM clock, throttle reasons)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sms, maxs, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sms.append(float(parts[1]))
+                maxs = max(maxs, float(parts[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sms:
+            return None
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": maxs,
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+def oracle_sample(w, n_tokens):
+    """Time the fp64 oracle (pre + post) on the first n_tokens tokens of the workload."""
+    import oracle
+    R, x = w.R[:n_tokens], w.x[:n_tokens]
+    t0 = time.perf_counter()
+    r = oracle.pre(R, w.hc_fn, w.hc_scale, w.hc_base, rms_eps=w.rms_eps, pre_eps=w.pre_eps,
+                   post_mult=w.post_mult, iters=w.iters, eps=w.eps)
+    oracle.post(x, R, r["post"].astype(np.float32), r["comb"].astype(np.float32))
+    dt = time.perf_counter() - t0
+    return n_tokens / dt, dt, oracle.threads()
+
+
+def cpu_baseline(w, budget_s=12.0):
+    """Bounded sample: calibrate on a few tokens, then time about budget_s seconds of oracle work."""
+    rate, _, _ = oracle_sample(w, 16)
+    n = int(max(16, min(w.T, rate * budget_s)))
+    rate, dt, cores = oracle_sample(w, n)
+    return {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"first {n} of {w.T} tokens (pre+post), {dt:.1f} s"}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    from mhc_hyper_connection_02_b200 import inputs
+    w = inputs.WORKLOADS[args.workload]()
+    per_step = []
+    base = None
+    for i in range(args.warmup + args.steps):
+        rate, dt, cores = oracle_sample(w, args.reference_tokens)
+        if i >= args.warmup:
+            per_step.append(dt)
+        base = cores
+    tot = sum(per_step)
+    value = args.reference_tokens * len(per_step) / tot
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(per_step),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"{args.workload} T={w.T} H={w.H}", "tokens_per_step": args.reference_tokens},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": base, "kind": "oracle",
+                         "sample": f"first {args.reference_tokens} of {w.T} tokens per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def load_traffic():
+    """ncu DRAM bytes per launch recorded under profiles/, valid only for the kernel source they were
+    taken from (sha256 of the library sources)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            return json.load(f)
+    except Exception:
+        return {}
+
+
+def source_digest():
+    import hashlib
+    from mhc_hyper_connection_02_b200 import build
+    h = hashlib.sha256()
+    for s in build.sources():
+        with open(s, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="large", choices=["large", "post4k", "small", "tail", "decode"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--reference-tokens", type=int, default=256)
+    ap.add_argument("--pre-path", type=int, default=0)
+    ap.add_argument("--post-path", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    import mhc_hyper_connection_02_b200 as mhc
+    from mhc_hyper_connection_02_b200 import inputs
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if ws > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    w = inputs.WORKLOADS[args.workload]()
+    T, H = w.T, w.H
+    dev = torch.device("cuda", local)
+    R = torch.from_numpy(w.R.view(np.int16)).view(torch.bfloat16).to(dev)
+    x = torch.from_numpy(w.x.view(np.int16)).view(torch.bfloat16).to(dev)
+    hc_fn = torch.from_numpy(w.hc_fn).to(dev)
+    scale = torch.from_numpy(w.hc_scale).to(dev)
+    base = torch.from_numpy(w.hc_base).to(dev)
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    pre = torch.empty((T, 4), dtype=torch.float32, device=dev)
+    post = torch.empty((T, 4), dtype=torch.float32, device=dev)
+    comb = torch.empty((T, 4, 4), dtype=torch.float32, device=dev)
+    out = torch.empty_like(R)
+    ws_bytes = mhc.workspace_bytes(T, H)
+    workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    params = mhc.make_params(iters=w.iters, eps=w.eps, rms_eps=w.rms_eps, pre_eps=w.pre_eps,
+                             post_mult=w.post_mult)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        mhc.pre(R, hc_fn, scale, base, y=y, pre=pre, post=post, comb=comb, workspace=workspace,
+                params=params, path=args.pre_path, stream=stream)
+        mhc.post(x, R, post, comb, out=out, path=args.post_path, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert mhc.device_status() == 0
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = mhc.launch_count()
+    start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        mhc.pre(R, hc_fn, scale, base, y=y, pre=pre, post=post, comb=comb, workspace=workspace,
+                params=params, path=args.pre_path, stream=stream)
+        ev[i][1].record(stream)
+        mhc.post(x, R, post, comb, out=out, path=args.post_path, stream=stream)
+        ev[i][2].record(stream)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    launches = mhc.launch_count() - launches0
+    if ws > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    assert mhc.device_status() == 0
+
+    total_ms = start.elapsed_time(stop)
+    pre_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    post_ms = [b.elapsed_time(c) for _, b, c in ev]
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if ws > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+
+    # End to end through the public API with host buffers: pinned H2D of the step's inputs, the
+    # two calls, D2H of the step's results, all inside the timed region.
+    e2e = None
+    if not args.no_e2e:
+        hR = torch.from_numpy(w.R.view(np.int16)).view(torch.bfloat16).pin_memory()
+        hx = torch.from_numpy(w.x.view(np.int16)).view(torch.bfloat16).pin_memory()
+        hW = torch.from_numpy(w.hc_fn).pin_memory()
+        hs = torch.from_numpy(w.hc_scale).pin_memory()
+        hb = torch.from_numpy(w.hc_base).pin_memory()
+        o_out = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+        o_y = torch.empty(y.shape, dtype=torch.bfloat16).pin_memory()
+        o_c = torch.empty((T, 24), dtype=torch.float32).pin_memory()
+        h2d = sum(a.numel() * a.element_size() for a in (hR, hx, hW, hs, hb))
+        d2h = sum(a.numel() * a.element_size() for a in (o_out, o_y, o_c))
+        coef = torch.empty((T, 24), dtype=torch.float32, device=dev)
+
+        def e2e_step():
+            R.copy_(hR, non_blocking=True)
+            x.copy_(hx, non_blocking=True)
+            hc_fn.copy_(hW, non_blocking=True)
+            scale.copy_(hs, non_blocking=True)
+            base.copy_(hb, non_blocking=True)
+            mhc.pre(R, hc_fn, scale, base, y=y, pre=pre, post=post, comb=comb,
+                    workspace=workspace, params=params, stream=stream)
+            mhc.post(x, R, post, comb, out=out, stream=stream)
+            coef[:, 0:4].copy_(pre)
+            coef[:, 4:8].copy_(post)
+            coef[:, 8:24].copy_(comb.view(T, 16))
+            o_out.copy_(out, non_blocking=True)
+            o_y.copy_(y, non_blocking=True)
+            o_c.copy_(coef, non_blocking=True)
+
+        e2e_steps = max(3, min(args.steps, 10))
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
+        if ws > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": ws * T * e2e_steps / (float(te.item()) / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    if rank == 0:
+        hbm, tflops, peak_src = load_peaks()
+        post_avg_s = statistics.mean(post_ms) / 1e3
+        pre_avg_s = statistics.mean(pre_ms) / 1e3
+        pb, qb = post_bytes(T, H), pre_bytes(T, H)
+        post_gbs = pb / post_avg_s / 1e9
+        pre_gbs = qb / pre_avg_s / 1e9
+        dominant = "post" if post_avg_s >= pre_avg_s else "pre"
+        traffic_rec = load_traffic().get(f"{dominant}:{args.workload}")
+        traffic = None
+        if traffic_rec and traffic_rec.get("source") == source_digest():
+            traffic = traffic_rec.get("bytes_per_launch")
+        ach = post_gbs if dominant == "post" else pre_gbs
+        line = {
+            "metric": METRIC,
+            "value": ws * T * args.steps / (max_ms / 1e3),
+            "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{args.workload}: T={T} H={H} HC=4 bf16, seeded synthetic",
+                       "tokens_per_gpu": T, "hidden": H, "sinkhorn_iters": w.iters,
+                       "parallelism": f"token shards x{ws}, no collective",
+                       "l2": "inputs larger than L2 (R = %d MB)" % (T * 8 * H // 2 ** 20)},
+            "roofline": {"bound": "hbm", "kernel": f"mhc_{dominant}", "achieved": ach,
+                         "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "traffic": traffic,
+                         "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)"},
+            "kernels": {
+                "pre": {"us": pre_avg_s * 1e6, "algo_bytes": qb, "GBps": pre_gbs,
+                        "frac_measured": pre_gbs / hbm, "frac_8TBps": pre_gbs / 8000.0,
+                        "path": args.pre_path},
+                "post": {"us": post_avg_s * 1e6, "algo_bytes": pb, "GBps": post_gbs,
+                         "frac_measured": post_gbs / hbm, "frac_8TBps": post_gbs / 8000.0,
+                         "path": args.post_path},
+            },
+            "gpu_launches": int(launches),
+            "clocks": clocks,
+            "e2e": e2e,
+        }
+        if not args.no_cpu_baseline and ws == 1:
+            line["cpu_baseline"] = cpu_baseline(w)
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

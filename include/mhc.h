@@ -1,0 +1,193 @@
+/*
+ * mhc.h -- C ABI of libmhc.so: the mHC (manifold-constrained hyper-connection) residual mix with
+ * HC = 4 streams, on NVIDIA B200 (sm_100a).
+ *
+ * Two steps make up the path, and a third entry exposes the Sinkhorn step on its own:
+ *
+ *   mhc_pre       per token: RMS-normalise the flattened [4H] residual row, project it through
+ *                 hc_fn [4H,24] to 24 logits, apply hc_scale / hc_base, and emit
+ *                 pre = sigmoid(l[0:4]) + pre_eps, post = post_mult * sigmoid(l[4:8]),
+ *                 comb = Sinkhorn(exp(l[8:24]) as 4x4) and y = sum_i pre_i * R_i.
+ *   mhc_post      out[n][h] = x[h] * post[n] + sum_o R[o][h] * comb[o][n].
+ *   mhc_sinkhorn  the Sinkhorn normalisation of caller-given 4x4 logits.
+ *
+ * Sources (page title and section):
+ *   "FlashInfer mHC module deep dive" (www.pwwt.cn/news/5432433):
+ *       §1 fixed HC = 4 and the 24-wide mix layout pre(4) | post(4) | comb(16);
+ *       §2.1 post-map formula; §2.2 shapes ([T,4] or [T,4,1] post, comb [old][new]);
+ *       §2.3 empty input returns without a launch; §3.1-3.2 pre-map parameters and defaults
+ *       (rms_eps, sinkhorn eps, sinkhorn_repeat >= 1, eps > 0); §3.4 kernel phases (sum of
+ *       squares, rstd, sigmoid gates, softmax with row-max shift, row -> column Sinkhorn rounds,
+ *       vec8 aggregate); §4 RMS denominator 4*H; §5.2 test reference math.
+ *   rwkv-ops 0.6.1 "rwkv_ops/mhc_kernel/jax_kernel/mhu_jax.py": docstrings of sinkhorn_knopp
+ *       (eps guards the division), stream_aggregate (fp32 accumulate, cast back), mhc_pre_op
+ *       (H_pre = sigmoid, H_post = 2 * sigmoid).
+ *   "metrale_model_layers/layers/ops/hyper_connection_dispatch.rs": hc_pre_site / hc_post_site
+ *       argument lists (device pointers, token count, hidden size, stream; out may alias residual).
+ *   "metrale_model_arch/glm5next_mhc.rs": glm_hc_pre (refuse to launch past the scratch
+ *       allocation), glm_hc_post (out may alias residual: every stream of an element is read
+ *       before it is written), mix_hc.
+ *
+ * Conventions for every entry point:
+ *   - All array pointers are DEVICE pointers into the current CUDA context's memory, dense and
+ *     row-major; bf16 arrays are passed as their 16-bit patterns (uint16_t). The caller owns and
+ *     allocates every buffer, including the pre-map workspace; the library allocates no device
+ *     memory and keeps no state between calls.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy default stream) and the call
+ *     returns without synchronising. Results are ready when the stream reaches that point.
+ *   - Arguments are validated on the host BEFORE anything is launched; on an error nothing is
+ *     written and nothing is enqueued. T == 0 returns MHC_OK without a launch.
+ *   - The device must be sm_100 (B200); the kernels are built for sm_100a only.
+ *   - Return value: MHC_OK (0) or a negative MHC_ERR_* code; mhc_status_string() names it.
+ */
+#ifndef MHC_H
+#define MHC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MHC_API __attribute__((visibility("default")))
+#else
+#define MHC_API
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* mhc_stream_t;
+
+enum {
+    MHC_HC = 4,   /* streams (fixed) */
+    MHC_MIX = 24, /* logits per token: pre(4) | post(4) | comb(16) */
+};
+
+enum mhc_status {
+    MHC_OK = 0,
+    MHC_ERR_INVALID_ARG = -1,         /* null pointer, T < 0, H <= 0, iters < 1, eps <= 0 ... */
+    MHC_ERR_WORKSPACE_TOO_SMALL = -2, /* workspace_bytes < mhc_pre_workspace_bytes(T, H) */
+    MHC_ERR_ALIAS = -3,               /* an output partially overlaps an input (see each call) */
+    MHC_ERR_CUDA = -4,                /* a CUDA runtime call or a launch failed */
+    MHC_ERR_UNSUPPORTED = -5,         /* device is not sm_100, or a forced path cannot run */
+    MHC_ERR_TIMEOUT = -6,             /* a bounded device-side wait gave up (see mhc_device_status) */
+};
+
+/* Pre-map parameters. Defaults (mhc_default_params): sinkhorn_iters 20 and sinkhorn_eps 1e-6
+ * ("FlashInfer mHC module deep dive" §3.2, sinkhorn_repeat / mhc_sinkhorn_eps), rms_eps 1e-6
+ * (same table), pre_eps 0 and post_mult 2 (rwkv-ops mhc_pre_op: H_pre = sigmoid,
+ * H_post = 2 * sigmoid; FlashInfer's defaults 1e-6 and 1.0 are reachable by setting them). */
+typedef struct {
+    int sinkhorn_iters; /* >= 1: rounds of (row normalise, column normalise) */
+    float sinkhorn_eps; /* > 0: added to every row / column sum before dividing by it */
+    float rms_eps;      /* > 0: rstd = 1 / sqrt(sum(R^2) / (4H) + rms_eps) */
+    float pre_eps;      /* >= 0: added to each pre gate */
+    float post_mult;    /* finite: post = post_mult * sigmoid(l[4:8]) */
+} mhc_params;
+
+MHC_API mhc_params mhc_default_params(void);
+
+/*
+ * mhc_pre -- the fused pre-map (steps: sum of squares -> rstd; projection; logit affine and gates;
+ * Sinkhorn; aggregate). "FlashInfer mHC module deep dive" §3.4 and §5.2; rwkv-ops mhc_pre_op.
+ *
+ *   R        [T][4][H] bf16   residual streams; the row of token t flattened as k = i*H + h
+ *   hc_fn    [4H][24]  fp32   projection (row k, logit j)
+ *   hc_scale [3]       fp32   logit scales of pre, post, comb, in that order
+ *   hc_base  [24]      fp32   logit biases
+ *   y        [T][H]    bf16   out: sum_i pre_i * R[t][i][:], fp32 accumulate, rounded to nearest even
+ *   pre      [T][4]    fp32   out
+ *   post     [T][4]    fp32   out
+ *   comb     [T][4][4] fp32   out, [old][new]: comb[o][n] weighs old stream o into new stream n
+ *   workspace / workspace_bytes: caller-allocated device scratch of at least
+ *            mhc_pre_workspace_bytes(T, H) bytes, 256-byte aligned; its contents on entry do not
+ *            matter and on return are unspecified. May be NULL when that size is 0.
+ *   p        host pointer to parameters; NULL selects mhc_default_params().
+ *
+ * Errors: MHC_ERR_INVALID_ARG for a null array, T < 0, H <= 0, or a parameter outside its range;
+ * MHC_ERR_WORKSPACE_TOO_SMALL; MHC_ERR_ALIAS when y, pre, post or comb overlaps R or one another.
+ * Any H >= 1 is accepted (FlashInfer requires H % 8 == 0; here other H take a scalar path), as is
+ * any alignment of the arrays.
+ */
+MHC_API int mhc_pre(const uint16_t* R, const float* hc_fn, const float* hc_scale, const float* hc_base,
+            uint16_t* y, float* pre, float* post, float* comb, void* workspace,
+            size_t workspace_bytes, int64_t T, int64_t H, const mhc_params* p,
+            mhc_stream_t stream);
+
+/* Bytes of workspace mhc_pre needs for (T, H): enough for every path mhc_pre or
+ * mhc_pre_with_path may take at that size. 0 when T <= 0 or H <= 0. */
+MHC_API size_t mhc_pre_workspace_bytes(int64_t T, int64_t H);
+
+/*
+ * mhc_post -- the post-map. "FlashInfer mHC module deep dive" §2.1-2.3; glm5next_mhc.rs
+ * glm_hc_post; hyper_connection_dispatch.rs hc_post_site.
+ *
+ *   x     [T][H]     bf16   layer output
+ *   R     [T][4][H]  bf16   residual streams
+ *   post  [T][4]     fp32   (a [T][4][1] tensor has the same layout)
+ *   comb  [T][4][4]  fp32   [old][new]
+ *   out   [T][4][H]  bf16   out[t][n][h] = bf16_rn(x*post[n] + sum_o R[o]*comb[o][n]), fp32 math
+ *
+ * out may be exactly R (in place): each element's four streams are read before it is written.
+ * Errors: MHC_ERR_INVALID_ARG (null array, T < 0, H <= 0); MHC_ERR_ALIAS when out overlaps R
+ * without being equal to it, or overlaps x, post or comb.
+ */
+MHC_API int mhc_post(const uint16_t* x, const uint16_t* R, const float* post, const float* comb,
+             uint16_t* out, int64_t T, int64_t H, mhc_stream_t stream);
+
+/*
+ * mhc_sinkhorn -- the Sinkhorn step on its own. "FlashInfer mHC module deep dive" §3.4 (softmax
+ * with row-max shift, then row -> column rounds) and §5.2; rwkv-ops sinkhorn_knopp.
+ *
+ *   logits [T][4][4] fp32   pre-exp logits, [old][new]
+ *   comb   [T][4][4] fp32   out: A = exp(l - rowmax); `iters` times { rows /= (rowsum + eps);
+ *                           columns /= (colsum + eps) }; may be equal to logits (in place)
+ *   H_unused               ignored (kept so every entry takes T and H)
+ *
+ * Errors: MHC_ERR_INVALID_ARG (null array, T < 0, iters < 1, eps <= 0 or not finite);
+ * MHC_ERR_ALIAS when comb overlaps logits without being equal to it.
+ */
+MHC_API int mhc_sinkhorn(const float* logits, float* comb, int64_t T, int64_t H_unused, int iters,
+                 float eps, mhc_stream_t stream);
+
+/* Kernel-path selectors for mhc_pre_with_path / mhc_post_with_path (tests and benchmarks use them
+ * to exercise each kernel; mhc_pre / mhc_post are MHC_PATH_AUTO). A forced path that cannot run
+ * on the given sizes or alignment returns MHC_ERR_UNSUPPORTED before any launch. */
+enum mhc_path {
+    MHC_PATH_AUTO = 0,
+    /* pre */
+    MHC_PRE_PATH_CUDA_CORE = 1, /* fp32 CUDA-core split-K projection + finish kernel */
+    MHC_PRE_PATH_TENSOR = 2,    /* tcgen05 projection (bf16 x3 split of hc_fn) fused pre */
+    /* post */
+    MHC_POST_PATH_VEC8 = 11,       /* 16-byte vector loads/stores; H % 8 == 0, 16-byte aligned */
+    MHC_POST_PATH_PERSISTENT = 12, /* persistent, bulk-copy (TMA) staged; same requirements */
+    MHC_POST_PATH_SCALAR = 13,     /* element-wise; any H and alignment */
+};
+
+MHC_API int mhc_pre_with_path(const uint16_t* R, const float* hc_fn, const float* hc_scale,
+                      const float* hc_base, uint16_t* y, float* pre, float* post, float* comb,
+                      void* workspace, size_t workspace_bytes, int64_t T, int64_t H,
+                      const mhc_params* p, int path, mhc_stream_t stream);
+
+MHC_API int mhc_post_with_path(const uint16_t* x, const uint16_t* R, const float* post, const float* comb,
+                       uint16_t* out, int64_t T, int64_t H, int path, mhc_stream_t stream);
+
+/* Reads and clears the device-side status word that bounded waits inside the kernels set when
+ * they give up (MHC_OK or MHC_ERR_TIMEOUT). Synchronises `stream` first. Kernels never trap. */
+MHC_API int mhc_device_status(mhc_stream_t stream);
+
+/* Number of kernel launches this process has enqueued through the library so far (all devices,
+ * all threads). A diagnostic counter for benchmarks: take the difference around a region. */
+MHC_API uint64_t mhc_launch_count(void);
+
+/* Static name of a status code ("MHC_OK", "MHC_ERR_ALIAS", ...). */
+MHC_API const char* mhc_status_string(int status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+MHC_API int mhc_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MHC_H */

@@ -1,0 +1,233 @@
+// C ABI of libmhc.so (declared in include/mhc.h): host-side validation, alias checks, device
+// binding and kernel dispatch. Nothing is launched before every check has passed
+// (glm5next_mhc.rs glm_hc_pre: refuse before launching; "FlashInfer mHC module deep dive" §2.3:
+// an empty input returns without a launch, §3.2: eps > 0 and sinkhorn_repeat >= 1).
+#include <math.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "mhc.h"
+#include "mhc_device.cuh"
+#include "mhc_internal.h"
+
+namespace mhc {
+
+namespace {
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices] = {};
+int g_cc[kMaxDevices] = {};
+std::mutex g_mu;
+
+void query_device(int dev) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_sm_count[dev] != 0) return;
+  int sms = 0, major = 0, minor = 0;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  g_cc[dev] = major * 10 + minor;
+  g_sm_count[dev] = sms > 0 ? sms : 1;
+}
+}  // namespace
+
+static std::atomic<uint64_t> g_launches{0};
+void note_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+
+int current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
+
+int device_sm_count() {
+  const int dev = current_device();
+  if (dev < 0) return 1;
+  if (g_sm_count[dev] == 0) query_device(dev);
+  return g_sm_count[dev];
+}
+
+int device_cc() {
+  const int dev = current_device();
+  if (dev < 0) return 0;
+  if (g_sm_count[dev] == 0) query_device(dev);
+  return g_cc[dev];
+}
+
+// Make this runtime's current device the one that owns `p` (the caller's framework may have a
+// different device current), and check that `p` is device memory and the device is sm_100.
+static int bind_device(const void* p) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return MHC_ERR_INVALID_ARG;
+  }
+  if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged) return MHC_ERR_INVALID_ARG;
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) return MHC_ERR_CUDA;
+  if (cur != at.device && cudaSetDevice(at.device) != cudaSuccess) return MHC_ERR_CUDA;
+  if (device_cc() / 10 != 10) return MHC_ERR_UNSUPPORTED;
+  return MHC_OK;
+}
+
+// Byte ranges [a, a+na) and [b, b+nb) intersect.
+static bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return na > 0 && nb > 0 && x < y + nb && y < x + na;
+}
+
+static bool mul_ok(int64_t a, int64_t b, int64_t limit) { return a >= 0 && b >= 0 && (b == 0 || a <= limit / b); }
+
+}  // namespace mhc
+
+using namespace mhc;
+
+extern "C" {
+
+mhc_params mhc_default_params(void) {
+  mhc_params p;
+  p.sinkhorn_iters = 20;
+  p.sinkhorn_eps = 1e-6f;
+  p.rms_eps = 1e-6f;
+  p.pre_eps = 0.0f;
+  p.post_mult = 2.0f;
+  return p;
+}
+
+const char* mhc_status_string(int status) {
+  switch (status) {
+    case MHC_OK: return "MHC_OK";
+    case MHC_ERR_INVALID_ARG: return "MHC_ERR_INVALID_ARG";
+    case MHC_ERR_WORKSPACE_TOO_SMALL: return "MHC_ERR_WORKSPACE_TOO_SMALL";
+    case MHC_ERR_ALIAS: return "MHC_ERR_ALIAS";
+    case MHC_ERR_CUDA: return "MHC_ERR_CUDA";
+    case MHC_ERR_UNSUPPORTED: return "MHC_ERR_UNSUPPORTED";
+    case MHC_ERR_TIMEOUT: return "MHC_ERR_TIMEOUT";
+    default: return "MHC_ERR_UNKNOWN";
+  }
+}
+
+int mhc_version(void) { return 100; }
+
+uint64_t mhc_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+size_t mhc_pre_workspace_bytes(int64_t T, int64_t H) {
+  if (T <= 0 || H <= 0) return 0;
+  size_t a = pre_cc_workspace_bytes(T, H);
+  size_t b = pre_tc_workspace_bytes(T, H);
+  size_t m = a > b ? a : b;
+  return (m + 255) / 256 * 256;
+}
+
+int mhc_post_with_path(const uint16_t* x, const uint16_t* R, const float* post, const float* comb,
+                       uint16_t* out, int64_t T, int64_t H, int path, mhc_stream_t stream) {
+  if (T < 0 || H <= 0) return MHC_ERR_INVALID_ARG;
+  if (!mul_ok(T, 4 * H, INT64_MAX / 4)) return MHC_ERR_INVALID_ARG;
+  if (T == 0) return MHC_OK;
+  if (!x || !R || !post || !comb || !out) return MHC_ERR_INVALID_ARG;
+  const size_t nR = static_cast<size_t>(T) * 4 * H * 2, nx = static_cast<size_t>(T) * H * 2;
+  if (static_cast<const void*>(out) != static_cast<const void*>(R) && overlaps(out, nR, R, nR))
+    return MHC_ERR_ALIAS;
+  if (overlaps(out, nR, x, nx) || overlaps(out, nR, post, T * 16) || overlaps(out, nR, comb, T * 64))
+    return MHC_ERR_ALIAS;
+  const bool vec_ok = (H % 8 == 0) && aligned16(x) && aligned16(R) && aligned16(out) &&
+                      aligned16(post) && aligned16(comb);
+  if (path == MHC_PATH_AUTO) {
+    path = vec_ok ? MHC_POST_PATH_VEC8 : MHC_POST_PATH_SCALAR;
+  } else if (path == MHC_POST_PATH_VEC8 || path == MHC_POST_PATH_PERSISTENT) {
+    if (!vec_ok) return MHC_ERR_UNSUPPORTED;
+  } else if (path != MHC_POST_PATH_SCALAR) {
+    return MHC_ERR_INVALID_ARG;
+  }
+  int st = bind_device(R);
+  if (st != MHC_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (path == MHC_POST_PATH_VEC8) return launch_post_vec8(x, R, post, comb, out, T, H, s);
+  if (path == MHC_POST_PATH_PERSISTENT) return launch_post_persistent(x, R, post, comb, out, T, H, s);
+  return launch_post_scalar(x, R, post, comb, out, T, H, s);
+}
+
+int mhc_post(const uint16_t* x, const uint16_t* R, const float* post, const float* comb,
+             uint16_t* out, int64_t T, int64_t H, mhc_stream_t stream) {
+  return mhc_post_with_path(x, R, post, comb, out, T, H, MHC_PATH_AUTO, stream);
+}
+
+int mhc_sinkhorn(const float* logits, float* comb, int64_t T, int64_t H_unused, int iters,
+                 float eps, mhc_stream_t stream) {
+  (void)H_unused;
+  if (T < 0 || iters < 1 || !(eps > 0.0f) || !isfinite(eps)) return MHC_ERR_INVALID_ARG;
+  if (!mul_ok(T, 64, INT64_MAX)) return MHC_ERR_INVALID_ARG;
+  if (T == 0) return MHC_OK;
+  if (!logits || !comb) return MHC_ERR_INVALID_ARG;
+  const size_t n = static_cast<size_t>(T) * 64;
+  if (static_cast<const void*>(comb) != static_cast<const void*>(logits) && overlaps(comb, n, logits, n))
+    return MHC_ERR_ALIAS;
+  int st = bind_device(logits);
+  if (st != MHC_OK) return st;
+  return launch_sinkhorn(logits, comb, T, iters, eps, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int mhc_pre_with_path(const uint16_t* R, const float* hc_fn, const float* hc_scale,
+                      const float* hc_base, uint16_t* y, float* pre, float* post, float* comb,
+                      void* workspace, size_t workspace_bytes, int64_t T, int64_t H,
+                      const mhc_params* p, int path, mhc_stream_t stream) {
+  const mhc_params prm = p ? *p : mhc_default_params();
+  if (T < 0 || H <= 0) return MHC_ERR_INVALID_ARG;
+  if (!mul_ok(T, 4 * H, INT64_MAX / 4)) return MHC_ERR_INVALID_ARG;
+  if (prm.sinkhorn_iters < 1 || !(prm.sinkhorn_eps > 0.0f) || !isfinite(prm.sinkhorn_eps) ||
+      !(prm.rms_eps > 0.0f) || !isfinite(prm.rms_eps) || !(prm.pre_eps >= 0.0f) ||
+      !isfinite(prm.pre_eps) || !isfinite(prm.post_mult))
+    return MHC_ERR_INVALID_ARG;
+  if (path != MHC_PATH_AUTO && path != MHC_PRE_PATH_CUDA_CORE && path != MHC_PRE_PATH_TENSOR)
+    return MHC_ERR_INVALID_ARG;
+  if (T == 0) return MHC_OK;
+  if (!R || !hc_fn || !hc_scale || !hc_base || !y || !pre || !post || !comb)
+    return MHC_ERR_INVALID_ARG;
+  const size_t need = mhc_pre_workspace_bytes(T, H);
+  if (workspace_bytes < need || (need > 0 && workspace == nullptr)) return MHC_ERR_WORKSPACE_TOO_SMALL;
+  const size_t nR = static_cast<size_t>(T) * 4 * H * 2, ny = static_cast<size_t>(T) * H * 2;
+  const size_t n4 = static_cast<size_t>(T) * 16, n16 = static_cast<size_t>(T) * 64;
+  const void* outs[4] = {y, pre, post, comb};
+  const size_t outn[4] = {ny, n4, n4, n16};
+  const void* ins[5] = {R, hc_fn, hc_scale, hc_base, workspace};
+  const size_t inn[5] = {nR, static_cast<size_t>(H) * 4 * 24 * 4, 12, 96, need};
+  for (int i = 0; i < 4; ++i) {
+    for (int j = 0; j < 5; ++j)
+      if (ins[j] && overlaps(outs[i], outn[i], ins[j], inn[j])) return MHC_ERR_ALIAS;
+    for (int j = i + 1; j < 4; ++j)
+      if (overlaps(outs[i], outn[i], outs[j], outn[j])) return MHC_ERR_ALIAS;
+  }
+  if (workspace && (overlaps(workspace, need, R, nR) || overlaps(workspace, need, hc_fn, inn[1])))
+    return MHC_ERR_ALIAS;
+  if (path == MHC_PATH_AUTO) {
+    path = pre_tc_supported(T, H) ? MHC_PRE_PATH_TENSOR : MHC_PRE_PATH_CUDA_CORE;
+  } else if (path == MHC_PRE_PATH_TENSOR && !pre_tc_supported(T, H)) {
+    return MHC_ERR_UNSUPPORTED;
+  }
+  int st = bind_device(R);
+  if (st != MHC_OK) return st;
+  PreArgs a{R, hc_fn, hc_scale, hc_base, y, pre, post, comb, workspace, workspace_bytes, T, H,
+            prm.sinkhorn_iters, prm.sinkhorn_eps, prm.rms_eps, prm.pre_eps, prm.post_mult};
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (path == MHC_PRE_PATH_TENSOR) return launch_pre_tc(a, s);
+  return launch_pre_cc(a, s);
+}
+
+int mhc_pre(const uint16_t* R, const float* hc_fn, const float* hc_scale, const float* hc_base,
+            uint16_t* y, float* pre, float* post, float* comb, void* workspace,
+            size_t workspace_bytes, int64_t T, int64_t H, const mhc_params* p,
+            mhc_stream_t stream) {
+  return mhc_pre_with_path(R, hc_fn, hc_scale, hc_base, y, pre, post, comb, workspace,
+                           workspace_bytes, T, H, p, MHC_PATH_AUTO, stream);
+}
+
+int mhc_device_status(mhc_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MHC_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return MHC_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return MHC_ERR_CUDA;
+  return v;
+}
+
+}  // extern "C"

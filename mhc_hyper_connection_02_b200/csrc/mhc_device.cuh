@@ -1,0 +1,166 @@
+// Device-side helpers shared by the mHC kernels (sm_100a): bf16 packing, 16-byte global
+// loads/stores with cache hints, mbarrier and bulk-copy wrappers with bounded waits, and the
+// per-token coefficient math (gates and the 4x4 Sinkhorn).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mhc {
+
+constexpr int kHC = 4;
+constexpr int kMix = 24;
+
+// Status word that bounded waits set when they give up; read and cleared by mhc_device_status().
+// Defined here: the library is a single translation unit (libmhc.cu).
+__device__ int g_device_status = 0;
+
+// Bounded waits give up after this many nanoseconds of %globaltimer.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ unsigned long long global_timer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void report_timeout(int where) {
+  atomicCAS(&g_device_status, 0, -6 /* MHC_ERR_TIMEOUT */);
+  (void)where;
+}
+
+// ------------------------------------------------------------------------------ bf16 packing
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+__device__ __forceinline__ float bf16_to_f32(uint16_t v) {
+  return __uint_as_float(static_cast<uint32_t>(v) << 16);
+}
+
+// Round two floats to bf16 (nearest even) and pack them, `a` in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ uint16_t f32_to_bf16(float a) {
+  __nv_bfloat16 v = __float2bfloat16_rn(a);
+  return *reinterpret_cast<uint16_t*>(&v);
+}
+
+// ------------------------------------------------------------------------------ 16-byte memory ops
+
+// Streaming read-only load (data not written by this kernel): non-coherent path, no L1 allocation.
+__device__ __forceinline__ uint4 ld_stream_ro(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+// Streaming load of data this kernel may later overwrite (in-place): coherent path.
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_stream(void* p, uint4 v) {
+  asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void st_plain(void* p, uint4 v) {
+  asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+
+// ------------------------------------------------------------------------------ mbarrier + bulk copy
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+__device__ __forceinline__ void fence_mbarrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile(
+      "{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
+          smem_u32(bar)),
+      "r"(bytes)
+      : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Wait for the phase with the given parity to complete. Returns false (and records a timeout) if
+// it has not completed within kWaitLimitNs; the caller then stops using the pipeline.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int where) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+      report_timeout(where);
+      return false;
+    }
+  }
+}
+
+// 1-D bulk copy global -> shared (TMA engine), completion counted on `bar` in bytes. Both
+// addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// ------------------------------------------------------------------------------ coefficient math
+
+__device__ __forceinline__ float sigmoidf_ieee(float v) { return 1.0f / (1.0f + expf(-v)); }
+
+// Sinkhorn on one 4x4 block held as 4 rows by 4 cooperating lanes: lane q (= lane & 3 within its
+// quad) owns row q. Row max shift and exp, then `iters` rounds of (row /= rowsum + eps,
+// column /= colsum + eps). Column sums reduce across the quad with xor shuffles. All 32 lanes of
+// the warp must call it (inactive quads pass any finite values).
+__device__ __forceinline__ void sinkhorn_quad(float (&a)[4], int iters, float eps) {
+  float m = fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3]));
+#pragma unroll
+  for (int n = 0; n < 4; ++n) a[n] = expf(a[n] - m);
+  for (int it = 0; it < iters; ++it) {
+    const float rs = ((a[0] + a[1]) + a[2]) + a[3] + eps;
+#pragma unroll
+    for (int n = 0; n < 4; ++n) a[n] = __fdiv_rn(a[n], rs);
+#pragma unroll
+    for (int n = 0; n < 4; ++n) {
+      float c = a[n] + __shfl_xor_sync(0xffffffffu, a[n], 1);
+      c = c + __shfl_xor_sync(0xffffffffu, c, 2);
+      a[n] = __fdiv_rn(a[n], c + eps);
+    }
+  }
+}
+
+}  // namespace mhc

@@ -1,0 +1,64 @@
+// Host-side declarations shared by the library's translation units (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cstddef>
+
+namespace mhc {
+
+// Device of the calling thread (this runtime instance), or -1 on error.
+int current_device();
+// Streaming multiprocessors of the current device (cached per device).
+int device_sm_count();
+// Compute capability major*10+minor of the current device (cached per device).
+int device_cc();
+
+// Counts kernel launches enqueued through the library (mhc_launch_count).
+void note_launches(int n);
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Launchers return 0 or a negative MHC_ERR_* code.
+int launch_post_vec8(const uint16_t* x, const uint16_t* R, const float* post, const float* comb,
+                     uint16_t* out, int64_t T, int64_t H, cudaStream_t s);
+int launch_post_scalar(const uint16_t* x, const uint16_t* R, const float* post, const float* comb,
+                       uint16_t* out, int64_t T, int64_t H, cudaStream_t s);
+int launch_post_persistent(const uint16_t* x, const uint16_t* R, const float* post,
+                           const float* comb, uint16_t* out, int64_t T, int64_t H,
+                           cudaStream_t s);
+
+int launch_sinkhorn(const float* logits, float* comb, int64_t T, int iters, float eps,
+                    cudaStream_t s);
+
+struct PreArgs {
+  const uint16_t* R;
+  const float* hc_fn;
+  const float* hc_scale;
+  const float* hc_base;
+  uint16_t* y;
+  float* pre;
+  float* post;
+  float* comb;
+  void* workspace;
+  size_t workspace_bytes;
+  int64_t T;
+  int64_t H;
+  int iters;
+  float sinkhorn_eps;
+  float rms_eps;
+  float pre_eps;
+  float post_mult;
+};
+
+// CUDA-core split-K path.
+size_t pre_cc_workspace_bytes(int64_t T, int64_t H);
+int launch_pre_cc(const PreArgs& a, cudaStream_t s);
+
+// Tensor-core path.
+size_t pre_tc_workspace_bytes(int64_t T, int64_t H);
+bool pre_tc_supported(int64_t T, int64_t H);
+int launch_pre_tc(const PreArgs& a, cudaStream_t s);
+
+}  // namespace mhc

@@ -1,0 +1,58 @@
+"""GPU parity of the standalone Sinkhorn entry (mhc_sinkhorn) against the fp64 oracle:
+A = exp(l - rowmax), then `iters` rounds of (rows /= rowsum + eps, columns /= colsum + eps)
+("FlashInfer mHC module deep dive" §3.4; rwkv-ops sinkhorn_knopp). Coefficient bar: 1e-5."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import mhc_hyper_connection_02_b200 as mhc
+from tolerance import check_coef
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("T", [1, 3, 1000, 4097])
+@pytest.mark.parametrize("std,iters", [(1.0, 1), (1.0, 20), (3.0, 50)])
+def test_sinkhorn_matches_oracle(T, std, iters):
+    rng = np.random.default_rng(T * 7 + iters)
+    logits = (rng.standard_normal((T, 4, 4)) * std).astype(np.float32)
+    got = mhc.sinkhorn(torch.from_numpy(logits).cuda(), iters=iters, eps=1e-6)
+    torch.cuda.synchronize()
+    ref = oracle.sinkhorn(logits.astype(np.float64), iters=iters, eps=1e-6)
+    d = check_coef(got.cpu().numpy(), ref, f"sinkhorn T={T} iters={iters}")
+    print(f"[sinkhorn T={T} std={std} iters={iters}] max|d|={d:.2e}")
+
+
+def test_sinkhorn_in_place_and_unaligned():
+    rng = np.random.default_rng(3)
+    logits = rng.standard_normal((257, 4, 4)).astype(np.float32)
+    ref = oracle.sinkhorn(logits.astype(np.float64), iters=20, eps=1e-6)
+    a = torch.from_numpy(logits).cuda()
+    mhc.sinkhorn(a, comb=a, iters=20, eps=1e-6)            # in place
+    big = torch.zeros(257 * 16 + 1, device="cuda")
+    big[1:] = torch.from_numpy(logits).cuda().view(-1)
+    u = big[1:].view(257, 4, 4)                            # 4-byte offset: scalar loads
+    got_u = mhc.sinkhorn(u, iters=20, eps=1e-6)
+    torch.cuda.synchronize()
+    check_coef(a.cpu().numpy(), ref, "in place")
+    check_coef(got_u.cpu().numpy(), ref, "unaligned")
+
+
+def test_sinkhorn_rank_one_is_uniform_and_doubly_stochastic():
+    rng = np.random.default_rng(4)
+    a, b = rng.standard_normal((64, 4, 1)), rng.standard_normal((64, 1, 4))
+    got = mhc.sinkhorn(torch.from_numpy((a + b).astype(np.float32)).cuda(), iters=20, eps=1e-6)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(got.cpu().numpy(), 0.25, atol=1e-5)
+
+
+def test_sinkhorn_large_eps_and_many_rounds():
+    rng = np.random.default_rng(5)
+    logits = (rng.standard_normal((999, 4, 4)) * 2).astype(np.float32)
+    for iters, eps in ((200, 1e-6), (7, 0.5)):
+        got = mhc.sinkhorn(torch.from_numpy(logits).cuda(), iters=iters, eps=eps)
+        torch.cuda.synchronize()
+        check_coef(got.cpu().numpy(), oracle.sinkhorn(logits.astype(np.float64), iters, eps),
+                   f"iters={iters} eps={eps}")
