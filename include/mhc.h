@@ -72,6 +72,7 @@ enum mhc_status {
     MHC_ERR_CUDA = -4,                /* a CUDA runtime call or a launch failed */
     MHC_ERR_UNSUPPORTED = -5,         /* device is not sm_100, or a forced path cannot run */
     MHC_ERR_TIMEOUT = -6,             /* a bounded device-side wait gave up (see mhc_device_status) */
+    MHC_ERR_SCRATCH_LIMIT = -7,       /* mhc_pre_noalloc: the size needs more than its fixed scratch */
 };
 
 /* Pre-map parameters. Defaults (mhc_default_params): sinkhorn_iters 20 and sinkhorn_eps 1e-6
@@ -176,6 +177,35 @@ MHC_API int mhc_post_with_path(const uint16_t* x, const uint16_t* R, const float
 /* Reads and clears the device-side status word that bounded waits inside the kernels set when
  * they give up (MHC_OK or MHC_ERR_TIMEOUT). Synchronises `stream` first. Kernels never trap. */
 MHC_API int mhc_device_status(mhc_stream_t stream);
+
+/*
+ * mhc_pre_noalloc -- mhc_pre for callers that cannot allocate device memory. No counterpart on the
+ * pages: it is an addition of this library.
+ *
+ * Some callers cannot call cudaMalloc or hand the library a workspace: plugins whose host framework
+ * owns every device allocation and whose plugin interface has no workspace argument, and serving
+ * loops that must not allocate per call (an allocation can synchronise the device and adds latency
+ * to every decode step). This entry computes exactly what mhc_pre computes on its CUDA-core path,
+ * but keeps that path's scratch (the split-K partial records, nsplit x T x 128 bytes) in a fixed
+ * array of MHC_NOALLOC_SCRATCH_BYTES bytes inside the library's device image instead of a
+ * caller workspace. The caller still passes every input and output.
+ *
+ *   - Sizes whose scratch would exceed MHC_NOALLOC_SCRATCH_BYTES return MHC_ERR_SCRATCH_LIMIT
+ *     before anything is launched (every T up to 16384 tokens fits for H up to 16392; other
+ *     arguments and errors are those of mhc_pre). It calls no cudaMalloc, cudaFree or allocating library routine.
+ *   - The array exists on every GPU that loads the library and is held until the process exits.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
+ *     that device current) and caches it; make that first call before any stream capture.
+ *   - All calls on a device share the one array, which keeps the last call's contents; every record
+ *     a call reads is written earlier in the same call, so nothing needs clearing. Calls whose
+ *     kernels can overlap on the GPU (different streams without ordering between them) race on the
+ *     array and give wrong results; order them on one stream.
+ */
+#define MHC_NOALLOC_SCRATCH_BYTES (4u << 20)
+MHC_API int mhc_pre_noalloc(const uint16_t* R, const float* hc_fn, const float* hc_scale,
+                            const float* hc_base, uint16_t* y, float* pre, float* post,
+                            float* comb, int64_t T, int64_t H, const mhc_params* p,
+                            mhc_stream_t stream);
 
 /* Number of kernel launches this process has enqueued through the library so far (all devices,
  * all threads). A diagnostic counter for benchmarks: take the difference around a region. */

@@ -25,6 +25,8 @@ MHC_ERR_ALIAS = -3
 MHC_ERR_CUDA = -4
 MHC_ERR_UNSUPPORTED = -5
 MHC_ERR_TIMEOUT = -6
+MHC_ERR_SCRATCH_LIMIT = -7
+NOALLOC_SCRATCH_BYTES = 4 << 20
 
 PATH_AUTO = 0
 PRE_PATH_CUDA_CORE = 1
@@ -36,7 +38,7 @@ POST_PATH_SCALAR = 13
 EXPORTED_SYMBOLS = (
     "mhc_default_params", "mhc_pre", "mhc_pre_workspace_bytes", "mhc_post", "mhc_sinkhorn",
     "mhc_pre_with_path", "mhc_post_with_path", "mhc_device_status", "mhc_status_string",
-    "mhc_version", "mhc_launch_count",
+    "mhc_version", "mhc_launch_count", "mhc_pre_noalloc",
 )
 
 
@@ -89,6 +91,9 @@ def lib() -> ctypes.CDLL:
     L.mhc_status_string.argtypes = [ctypes.c_int]
     L.mhc_version.restype = ctypes.c_int
     L.mhc_version.argtypes = []
+    L.mhc_pre_noalloc.restype = ctypes.c_int
+    L.mhc_pre_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64,
+                                  ctypes.POINTER(Params), _P]
     L.mhc_launch_count.restype = ctypes.c_uint64
     L.mhc_launch_count.argtypes = []
     _lib = L

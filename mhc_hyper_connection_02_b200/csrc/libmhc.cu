@@ -6,3 +6,4 @@
 #include "mhc_sinkhorn.cu"
 #include "mhc_pre_cc.cu"
 #include "mhc_pre_tc.cu"
+#include "mhc_pre_noalloc.cu"

@@ -103,6 +103,7 @@ const char* mhc_status_string(int status) {
     case MHC_ERR_CUDA: return "MHC_ERR_CUDA";
     case MHC_ERR_UNSUPPORTED: return "MHC_ERR_UNSUPPORTED";
     case MHC_ERR_TIMEOUT: return "MHC_ERR_TIMEOUT";
+    case MHC_ERR_SCRATCH_LIMIT: return "MHC_ERR_SCRATCH_LIMIT";
     default: return "MHC_ERR_UNKNOWN";
   }
 }

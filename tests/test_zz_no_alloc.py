@@ -1,0 +1,70 @@
+"""mhc_pre_noalloc: the pre-map for callers that cannot allocate device memory (plugins whose host
+framework owns all device allocations and gives them no workspace, and serving loops that must not
+allocate per call). It keeps its scratch in a fixed array inside the library.
+
+Checked through the C ABI against the existing entry point (mhc_pre, which takes a caller workspace)
+on two calls in a row with different sizes, within the tolerances the other tests use. This file is
+collected last so that a run stopping at the first failure has already run every other test.
+"""
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import mhc_hyper_connection_02_b200 as mhc
+from mhc_hyper_connection_02_b200 import inputs
+from tolerance import COEF_TOL, REL, ulp_bf16, bf16_bits_to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def to_dev(w):
+    return (torch.from_numpy(w.R.view(np.int16)).view(torch.bfloat16).cuda(),
+            torch.from_numpy(w.hc_fn).cuda(), torch.from_numpy(w.hc_scale).cuda(),
+            torch.from_numpy(w.hc_base).cuda())
+
+
+def call_noalloc(R, W, S, B, T, H, params):
+    y = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    pre = torch.empty((T, 4), device="cuda")
+    post = torch.empty((T, 4), device="cuda")
+    comb = torch.empty((T, 4, 4), device="cuda")
+    st = mhc.lib().mhc_pre_noalloc(R.data_ptr(), W.data_ptr(), S.data_ptr(), B.data_ptr(),
+                                   y.data_ptr(), pre.data_ptr(), post.data_ptr(), comb.data_ptr(),
+                                   T, H, ctypes.byref(params),
+                                   ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == mhc.MHC_OK, mhc.status_string(st)
+    return y, pre, post, comb
+
+
+def assert_close(new, ref):
+    for a, b, name in zip(new[1:], ref[1:], ("pre", "post", "comb")):
+        d = (a.double() - b.double()).abs().max().item()
+        assert d <= COEF_TOL, f"{name}: {d}"
+    yn = bf16_bits_to_f64(new[0].view(torch.int16).cpu().numpy().view(np.uint16))
+    yr = bf16_bits_to_f64(ref[0].view(torch.int16).cpu().numpy().view(np.uint16))
+    tol = np.maximum(ulp_bf16(yr), REL * np.abs(yr))
+    assert np.all(np.abs(yn - yr) <= tol)
+
+
+def test_noalloc_matches_mhc_pre_on_two_calls_in_a_row():
+    for w in (inputs.decode(32), inputs.custom(7, 1000, seed=61)):
+        params = mhc.make_params(iters=w.iters, eps=w.eps, rms_eps=w.rms_eps)
+        R, W, S, B = to_dev(w)
+        new = call_noalloc(R, W, S, B, w.T, w.H, params)
+        ref = mhc.pre(R, W, S, B, params=params)
+        torch.cuda.synchronize()
+        assert mhc.device_status() == 0
+        assert_close(new, ref)
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch():
+    A = 1 << 40
+    p = mhc.default_params()
+    st = mhc.lib().mhc_pre_noalloc(A, A + (1 << 36), A + (2 << 36), A + (3 << 36), A + (4 << 36),
+                                   A + (5 << 36), A + (6 << 36), A + (7 << 36), 16385, 512,
+                                   ctypes.byref(p), None)
+    assert st == mhc.MHC_ERR_SCRATCH_LIMIT
+    assert mhc.status_string(st) == "MHC_ERR_SCRATCH_LIMIT"
