@@ -159,7 +159,10 @@ enum mhc_path {
     MHC_PATH_AUTO = 0,
     /* pre */
     MHC_PRE_PATH_CUDA_CORE = 1, /* fp32 CUDA-core split-K projection + finish kernel */
-    MHC_PRE_PATH_TENSOR = 2,    /* tcgen05 projection (bf16 x3 split of hc_fn) fused pre */
+    MHC_PRE_PATH_TENSOR = 2,    /* tcgen05 projection (exact bf16 x3 split of hc_fn): the
+                                   persistent fused kernel when H % 8 == 0 and R, y, pre and the
+                                   workspace are 16-byte aligned, else the split pair below */
+    MHC_PRE_PATH_TENSOR_SPLIT = 3, /* tcgen05 projection kernel + finish kernel; H even */
     /* post */
     MHC_POST_PATH_VEC8 = 11,       /* 16-byte vector loads/stores; H % 8 == 0, 16-byte aligned */
     MHC_POST_PATH_PERSISTENT = 12, /* persistent, bulk-copy (TMA) staged; same requirements */

@@ -6,4 +6,5 @@
 #include "mhc_sinkhorn.cu"
 #include "mhc_pre_cc.cu"
 #include "mhc_pre_tc.cu"
+#include "mhc_pre_fused.cu"
 #include "mhc_pre_noalloc.cu"

@@ -76,6 +76,10 @@ static bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   return na > 0 && nb > 0 && x < y + nb && y < x + na;
 }
 
+constexpr int64_t kPreTensorMinTokens = 128;
+constexpr int64_t kPostPersistentMinH = 2048;
+constexpr int64_t kPostPersistentMinElems = int64_t(1) << 22;
+
 static bool mul_ok(int64_t a, int64_t b, int64_t limit) { return a >= 0 && b >= 0 && (b == 0 || a <= limit / b); }
 
 }  // namespace mhc
@@ -114,9 +118,10 @@ uint64_t mhc_launch_count(void) { return g_launches.load(std::memory_order_relax
 
 size_t mhc_pre_workspace_bytes(int64_t T, int64_t H) {
   if (T <= 0 || H <= 0) return 0;
-  size_t a = pre_cc_workspace_bytes(T, H);
-  size_t b = pre_tc_workspace_bytes(T, H);
-  size_t m = a > b ? a : b;
+  size_t m = pre_cc_workspace_bytes(T, H);
+  const size_t b = pre_tc_workspace_bytes(T, H), c = pre_fused_workspace_bytes(T, H);
+  if (b > m) m = b;
+  if (c > m) m = c;
   return (m + 255) / 256 * 256;
 }
 
@@ -134,7 +139,10 @@ int mhc_post_with_path(const uint16_t* x, const uint16_t* R, const float* post, 
   const bool vec_ok = (H % 8 == 0) && aligned16(x) && aligned16(R) && aligned16(out) &&
                       aligned16(post) && aligned16(comb);
   if (path == MHC_PATH_AUTO) {
-    path = vec_ok ? MHC_POST_PATH_VEC8 : MHC_POST_PATH_SCALAR;
+    // The bulk-copy staged persistent kernel streams best once rows are long (one 1024-element
+    // chunk per tile row) and the call is large; short rows and small calls take vec8.
+    const bool big = H >= kPostPersistentMinH && T * H >= kPostPersistentMinElems;
+    path = !vec_ok ? MHC_POST_PATH_SCALAR : (big ? MHC_POST_PATH_PERSISTENT : MHC_POST_PATH_VEC8);
   } else if (path == MHC_POST_PATH_VEC8 || path == MHC_POST_PATH_PERSISTENT) {
     if (!vec_ok) return MHC_ERR_UNSUPPORTED;
   } else if (path != MHC_POST_PATH_SCALAR) {
@@ -179,7 +187,8 @@ int mhc_pre_with_path(const uint16_t* R, const float* hc_fn, const float* hc_sca
       !(prm.rms_eps > 0.0f) || !isfinite(prm.rms_eps) || !(prm.pre_eps >= 0.0f) ||
       !isfinite(prm.pre_eps) || !isfinite(prm.post_mult))
     return MHC_ERR_INVALID_ARG;
-  if (path != MHC_PATH_AUTO && path != MHC_PRE_PATH_CUDA_CORE && path != MHC_PRE_PATH_TENSOR)
+  if (path != MHC_PATH_AUTO && path != MHC_PRE_PATH_CUDA_CORE && path != MHC_PRE_PATH_TENSOR &&
+      path != MHC_PRE_PATH_TENSOR_SPLIT)
     return MHC_ERR_INVALID_ARG;
   if (T == 0) return MHC_OK;
   if (!R || !hc_fn || !hc_scale || !hc_base || !y || !pre || !post || !comb)
@@ -200,9 +209,17 @@ int mhc_pre_with_path(const uint16_t* R, const float* hc_fn, const float* hc_sca
   }
   if (workspace && (overlaps(workspace, need, R, nR) || overlaps(workspace, need, hc_fn, inn[1])))
     return MHC_ERR_ALIAS;
+  // The tensor path reads R and its split hc_fn copy (in the workspace) with TMA: 16-byte aligned
+  // bases. Below kPreTensorMinTokens the CUDA-core path, which reads hc_fn once in fp32, is faster.
+  const bool tc_ok = pre_tc_supported(T, H) && aligned16(R) && aligned16(workspace);
+  // The fused kernel also uses 16-byte accesses on y, pre and comb.
+  const bool fused_ok = tc_ok && pre_fused_supported(T, H) && aligned16(y) && aligned16(pre) &&
+                        aligned16(comb);
   if (path == MHC_PATH_AUTO) {
-    path = pre_tc_supported(T, H) ? MHC_PRE_PATH_TENSOR : MHC_PRE_PATH_CUDA_CORE;
-  } else if (path == MHC_PRE_PATH_TENSOR && !pre_tc_supported(T, H)) {
+    path = (tc_ok && T >= kPreTensorMinTokens) ? MHC_PRE_PATH_TENSOR : MHC_PRE_PATH_CUDA_CORE;
+  } else if (path == MHC_PRE_PATH_TENSOR_SPLIT && !tc_ok) {
+    return MHC_ERR_UNSUPPORTED;
+  } else if (path == MHC_PRE_PATH_TENSOR && !tc_ok) {
     return MHC_ERR_UNSUPPORTED;
   }
   int st = bind_device(R);
@@ -210,7 +227,11 @@ int mhc_pre_with_path(const uint16_t* R, const float* hc_fn, const float* hc_sca
   PreArgs a{R, hc_fn, hc_scale, hc_base, y, pre, post, comb, workspace, workspace_bytes, T, H,
             prm.sinkhorn_iters, prm.sinkhorn_eps, prm.rms_eps, prm.pre_eps, prm.post_mult};
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (path == MHC_PRE_PATH_TENSOR) return launch_pre_tc(a, s);
+  if (path == MHC_PRE_PATH_TENSOR && fused_ok) {
+    const int r = launch_pre_fused(a, s);
+    if (r <= 0) return r;  // 1: grid cannot be co-scheduled here, take the split pair
+  }
+  if (path == MHC_PRE_PATH_TENSOR || path == MHC_PRE_PATH_TENSOR_SPLIT) return launch_pre_tc(a, s);
   return launch_pre_cc(a, s);
 }
 

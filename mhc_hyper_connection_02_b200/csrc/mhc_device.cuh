@@ -120,9 +120,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int wh
   const unsigned long long t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
-      report_timeout(where);
-      return false;
+    if ((i & 255u) == 0) {
+      if (*reinterpret_cast<volatile int*>(&g_device_status) != 0) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        report_timeout(where);
+        return false;
+      }
     }
   }
 }
@@ -142,23 +145,35 @@ __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, u
 
 __device__ __forceinline__ float sigmoidf_ieee(float v) { return 1.0f / (1.0f + expf(-v)); }
 
+// 1/s for a positive normal s: the hardware approximate reciprocal refined by one Newton-Raphson
+// step r1 = r0 + r0 * (1 - s * r0) (the textbook iteration for 1/s, e.g. Muller et al.,
+// "Handbook of Floating-Point Arithmetic", ch. 5), which roughly doubles the correct bits of r0;
+// the result is within about an ulp of the correctly rounded reciprocal.
+__device__ __forceinline__ float recip_nr(float s) {
+  float r0;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r0) : "f"(s));
+  const float e = fmaf(-s, r0, 1.0f);
+  return fmaf(r0, e, r0);
+}
+
 // Sinkhorn on one 4x4 block held as 4 rows by 4 cooperating lanes: lane q (= lane & 3 within its
 // quad) owns row q. Row max shift and exp, then `iters` rounds of (row /= rowsum + eps,
-// column /= colsum + eps). Column sums reduce across the quad with xor shuffles. All 32 lanes of
-// the warp must call it (inactive quads pass any finite values).
+// column /= colsum + eps), each division done as a multiplication by recip_nr of the sum.
+// Column sums reduce across the quad with xor shuffles. All 32 lanes of the warp must call it
+// (inactive quads pass any finite values).
 __device__ __forceinline__ void sinkhorn_quad(float (&a)[4], int iters, float eps) {
   float m = fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3]));
 #pragma unroll
   for (int n = 0; n < 4; ++n) a[n] = expf(a[n] - m);
   for (int it = 0; it < iters; ++it) {
-    const float rs = ((a[0] + a[1]) + a[2]) + a[3] + eps;
+    const float rr = recip_nr(((a[0] + a[1]) + a[2]) + a[3] + eps);
 #pragma unroll
-    for (int n = 0; n < 4; ++n) a[n] = __fdiv_rn(a[n], rs);
+    for (int n = 0; n < 4; ++n) a[n] *= rr;
 #pragma unroll
     for (int n = 0; n < 4; ++n) {
       float c = a[n] + __shfl_xor_sync(0xffffffffu, a[n], 1);
       c = c + __shfl_xor_sync(0xffffffffu, c, 2);
-      a[n] = __fdiv_rn(a[n], c + eps);
+      a[n] *= recip_nr(c + eps);
     }
   }
 }

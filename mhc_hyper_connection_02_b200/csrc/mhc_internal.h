@@ -56,7 +56,13 @@ struct PreArgs {
 size_t pre_cc_workspace_bytes(int64_t T, int64_t H);
 int launch_pre_cc(const PreArgs& a, cudaStream_t s);
 
-// Tensor-core path.
+// Tensor-core path: persistent fused kernel (launch returns 1 when the device cannot co-schedule
+// its grid; the caller then takes the split pair).
+bool pre_fused_supported(int64_t T, int64_t H);
+size_t pre_fused_workspace_bytes(int64_t T, int64_t H);
+int launch_pre_fused(const PreArgs& a, cudaStream_t s);
+
+// Tensor-core path, split pair (projection kernel + finish kernel).
 size_t pre_tc_workspace_bytes(int64_t T, int64_t H);
 bool pre_tc_supported(int64_t T, int64_t H);
 int launch_pre_tc(const PreArgs& a, cudaStream_t s);

@@ -19,7 +19,8 @@ from tolerance import COEF_TOL, U32, bf16_bits_to_f64, check_bf16, check_coef
 
 pytestmark = pytest.mark.gpu
 
-PRE_PATHS = {"cuda_core": mhc.PRE_PATH_CUDA_CORE, "tensor": mhc.PRE_PATH_TENSOR}
+PRE_PATHS = {"cuda_core": mhc.PRE_PATH_CUDA_CORE, "tensor": mhc.PRE_PATH_TENSOR,
+             "tensor_split": mhc.PRE_PATH_TENSOR_SPLIT}
 
 
 def run_pre(w, path=mhc.PATH_AUTO, params=None, R_dev=None):
@@ -53,7 +54,7 @@ def compare_pre(w, outs, rows=None, label="", pre_eps=None, post_mult=None, iter
     return max(dp, dq, dc)
 
 
-@pytest.mark.parametrize("path", ["cuda_core", "tensor"])
+@pytest.mark.parametrize("path", ["cuda_core", "tensor", "tensor_split"])
 def test_pre_small_workload(path):
     w = inputs.small()
     try:
@@ -70,6 +71,25 @@ def test_pre_shapes(T, H):
     w = inputs.custom(T, H, seed=T + H)
     compare_pre(w, run_pre(w), label=f"T={T} H={H}")
     compare_pre(w, run_pre(w, mhc.PRE_PATH_CUDA_CORE), label=f"T={T} H={H} cuda_core")
+    if H % 2 == 0:
+        compare_pre(w, run_pre(w, mhc.PRE_PATH_TENSOR), label=f"T={T} H={H} tensor")
+        compare_pre(w, run_pre(w, mhc.PRE_PATH_TENSOR_SPLIT), label=f"T={T} H={H} tensor-split")
+
+
+@pytest.mark.parametrize("T,H", [(300, 7168), (129, 1000), (1, 4096), (520, 512)])
+def test_pre_tensor_path_agrees_with_cuda_core_path(T, H):
+    """Two GPU implementations of the projection (tcgen05 bf16x3 vs fp32 CUDA cores) agree within
+    the coefficient tolerance, and each matches the oracle."""
+    w = inputs.custom(T, H, seed=3 * T + H)
+    a = run_pre(w, mhc.PRE_PATH_TENSOR)
+    b = run_pre(w, mhc.PRE_PATH_CUDA_CORE)
+    c = run_pre(w, mhc.PRE_PATH_TENSOR_SPLIT)
+    for other, oname in ((b, "cuda_core"), (c, "tensor-split")):
+        for x, y, name in zip(a[1:], other[1:], ("pre", "post", "comb")):
+            d = (x.double() - y.double()).abs().max().item()
+            print(f"[tensor vs {oname} T={T} H={H}] {name} max|d| = {d:.2e}")
+            assert d <= COEF_TOL
+    compare_pre(w, a, label=f"tensor T={T} H={H}")
 
 
 @pytest.mark.parametrize("T", [1, 4, 16, 32])
