@@ -159,10 +159,13 @@ enum mhc_path {
     MHC_PATH_AUTO = 0,
     /* pre */
     MHC_PRE_PATH_CUDA_CORE = 1, /* fp32 CUDA-core split-K projection + finish kernel */
-    MHC_PRE_PATH_TENSOR = 2,    /* tcgen05 projection (exact bf16 x3 split of hc_fn): the
-                                   persistent fused kernel when H % 8 == 0 and R, y, pre and the
-                                   workspace are 16-byte aligned, else the split pair below */
-    MHC_PRE_PATH_TENSOR_SPLIT = 3, /* tcgen05 projection kernel + finish kernel; H even */
+    MHC_PRE_PATH_TENSOR = 2,    /* tcgen05 projection (exact bf16 x3 split of hc_fn), the
+                                   fastest tensor-core variant: currently the split pair */
+    MHC_PRE_PATH_TENSOR_SPLIT = 3, /* tcgen05 split-K projection kernel, then a coefficient kernel
+                                      and a streaming aggregate kernel; H even */
+    MHC_PRE_PATH_TENSOR_FUSED = 4, /* one persistent kernel (projection, cross-CTA reduction,
+                                      coefficients, aggregate); H % 8 == 0 and R, y, pre, comb and
+                                      the workspace 16-byte aligned */
     /* post */
     MHC_POST_PATH_VEC8 = 11,       /* 16-byte vector loads/stores; H % 8 == 0, 16-byte aligned */
     MHC_POST_PATH_PERSISTENT = 12, /* persistent, bulk-copy (TMA) staged; same requirements */

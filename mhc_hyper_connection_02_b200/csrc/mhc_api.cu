@@ -188,7 +188,7 @@ int mhc_pre_with_path(const uint16_t* R, const float* hc_fn, const float* hc_sca
       !isfinite(prm.pre_eps) || !isfinite(prm.post_mult))
     return MHC_ERR_INVALID_ARG;
   if (path != MHC_PATH_AUTO && path != MHC_PRE_PATH_CUDA_CORE && path != MHC_PRE_PATH_TENSOR &&
-      path != MHC_PRE_PATH_TENSOR_SPLIT)
+      path != MHC_PRE_PATH_TENSOR_SPLIT && path != MHC_PRE_PATH_TENSOR_FUSED)
     return MHC_ERR_INVALID_ARG;
   if (T == 0) return MHC_OK;
   if (!R || !hc_fn || !hc_scale || !hc_base || !y || !pre || !post || !comb)
@@ -217,9 +217,9 @@ int mhc_pre_with_path(const uint16_t* R, const float* hc_fn, const float* hc_sca
                         aligned16(comb);
   if (path == MHC_PATH_AUTO) {
     path = (tc_ok && T >= kPreTensorMinTokens) ? MHC_PRE_PATH_TENSOR : MHC_PRE_PATH_CUDA_CORE;
-  } else if (path == MHC_PRE_PATH_TENSOR_SPLIT && !tc_ok) {
+  } else if ((path == MHC_PRE_PATH_TENSOR || path == MHC_PRE_PATH_TENSOR_SPLIT) && !tc_ok) {
     return MHC_ERR_UNSUPPORTED;
-  } else if (path == MHC_PRE_PATH_TENSOR && !tc_ok) {
+  } else if (path == MHC_PRE_PATH_TENSOR_FUSED && !fused_ok) {
     return MHC_ERR_UNSUPPORTED;
   }
   int st = bind_device(R);
@@ -227,11 +227,11 @@ int mhc_pre_with_path(const uint16_t* R, const float* hc_fn, const float* hc_sca
   PreArgs a{R, hc_fn, hc_scale, hc_base, y, pre, post, comb, workspace, workspace_bytes, T, H,
             prm.sinkhorn_iters, prm.sinkhorn_eps, prm.rms_eps, prm.pre_eps, prm.post_mult};
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (path == MHC_PRE_PATH_TENSOR && fused_ok) {
+  if (path == MHC_PRE_PATH_TENSOR_FUSED) {
     const int r = launch_pre_fused(a, s);
     if (r <= 0) return r;  // 1: grid cannot be co-scheduled here, take the split pair
   }
-  if (path == MHC_PRE_PATH_TENSOR || path == MHC_PRE_PATH_TENSOR_SPLIT) return launch_pre_tc(a, s);
+  if (path != MHC_PRE_PATH_CUDA_CORE) return launch_pre_tc(a, s);
   return launch_pre_cc(a, s);
 }
 

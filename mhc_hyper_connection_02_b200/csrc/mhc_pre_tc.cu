@@ -37,7 +37,7 @@ constexpr int kTcStageBytes = kTcABytes + kTcBBytes;  // 26624 = 26 x 1024
 constexpr int kTcThreads = 192;
 constexpr int kTcTmemCols = 128;
 constexpr int kTcSmem = 1024 + kTcStages * kTcStageBytes + 256;
-constexpr int64_t kTcPlanCtas = 444;               // 3 x 148: target CTAs of the split plan
+constexpr int64_t kTcSms = 148;                    // SM count the split plan is tuned for (B200)
 
 struct TcPlan {
   int64_t ntiles, kblocks, kbps, nsplit;
@@ -49,10 +49,25 @@ static TcPlan tc_plan(int64_t T, int64_t H) {
   const int64_t K = 4 * H;
   p.ntiles = (T + kTcM - 1) / kTcM;
   p.kblocks = (K + kTcKB - 1) / kTcKB;
-  int64_t ns = (kTcPlanCtas + p.ntiles - 1) / p.ntiles;
-  if (ns < 1) ns = 1;
-  if (ns > p.kblocks) ns = p.kblocks;
-  p.kbps = (p.kblocks + ns - 1) / ns;
+  // Splits per tile: at least 3 waves of CTAs (one CTA per SM); then the fewest splits whose last
+  // wave is at least 90% full (each CTA's pipeline fill is exposed, so longer CTAs are better),
+  // else the fullest last wave seen.
+  const int64_t ns_min = (3 * kTcSms + p.ntiles - 1) / p.ntiles;
+  int64_t best_ns = ns_min > p.kblocks ? p.kblocks : (ns_min < 1 ? 1 : ns_min);
+  double best_eff = -1.0;
+  for (int64_t ns = best_ns; ns <= ns_min + 16 && ns <= p.kblocks; ++ns) {
+    const int64_t kbps = (p.kblocks + ns - 1) / ns;
+    const int64_t nsplit = (p.kblocks + kbps - 1) / kbps;
+    const int64_t ctas = nsplit * p.ntiles;
+    const int64_t waves = (ctas + kTcSms - 1) / kTcSms;
+    const double eff = static_cast<double>(ctas) / static_cast<double>(waves * kTcSms);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best_ns = ns;
+    }
+    if (eff >= 0.9) break;
+  }
+  p.kbps = (p.kblocks + best_ns - 1) / best_ns;
   p.nsplit = (p.kblocks + p.kbps - 1) / p.kbps;
   p.bw_bytes = (static_cast<size_t>(kTcN) * K * 2 + 1023) / 1024 * 1024;
   return p;
@@ -308,6 +323,89 @@ __global__ void __launch_bounds__(kTcThreads, 1) pre_tc_proj_kernel(
   }
 }
 
+// Coefficients from the split records [split][t][32] (raw[0..23], ss): one token per lane quad,
+// 8 tokens per warp. Lane r of a quad sums, over the splits in order, the components it needs
+// (pre r, post r, comb row r, ss) and runs its row of the Sinkhorn.
+__global__ void __launch_bounds__(256) pre_tc_coef_kernel(const float* __restrict__ part,
+                                                          int64_t nsplit,
+                                                          const float* __restrict__ scale,
+                                                          const float* __restrict__ base,
+                                                          float* __restrict__ pre,
+                                                          float* __restrict__ post,
+                                                          float* __restrict__ comb, int64_t T,
+                                                          int64_t K, FinishParams fp) {
+  const int lane = threadIdx.x & 31;
+  const int r = lane & 3;
+  const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 2;
+  const bool live = t < T;
+  const int64_t tt = live ? t : 0;
+  float4 g0 = make_float4(0.f, 0.f, 0.f, 0.f), g1 = g0, gc = g0, g6 = g0;
+  for (int64_t s = 0; s < nsplit; ++s) {
+    const float4* rec = reinterpret_cast<const float4*>(part + (s * T + tt) * 32);
+    const float4 a0 = __ldg(rec), a1 = __ldg(rec + 1), ac = __ldg(rec + 2 + r), a6 = __ldg(rec + 6);
+    g0.x += a0.x, g0.y += a0.y, g0.z += a0.z, g0.w += a0.w;
+    g1.x += a1.x, g1.y += a1.y, g1.z += a1.z, g1.w += a1.w;
+    gc.x += ac.x, gc.y += ac.y, gc.z += ac.z, gc.w += ac.w;
+    g6.x += a6.x;
+  }
+  const float p0[4] = {g0.x, g0.y, g0.z, g0.w};
+  const float p1[4] = {g1.x, g1.y, g1.z, g1.w};
+  const float rstd =
+      __fdiv_rn(1.0f, __fsqrt_rn(__fdiv_rn(g6.x, static_cast<float>(K)) + fp.rms_eps));
+  const float lp = fmaf(p0[r] * rstd, __ldg(scale), __ldg(base + r));
+  const float lq = fmaf(p1[r] * rstd, __ldg(scale + 1), __ldg(base + 4 + r));
+  const float s2 = __ldg(scale + 2);
+  float cr[4] = {fmaf(gc.x * rstd, s2, __ldg(base + 8 + 4 * r)),
+                 fmaf(gc.y * rstd, s2, __ldg(base + 9 + 4 * r)),
+                 fmaf(gc.z * rstd, s2, __ldg(base + 10 + 4 * r)),
+                 fmaf(gc.w * rstd, s2, __ldg(base + 11 + 4 * r))};
+  sinkhorn_quad(cr, fp.iters, fp.sinkhorn_eps);  // every lane takes part
+  if (live) {
+    pre[t * 4 + r] = sigmoidf_ieee(lp) + fp.pre_eps;
+    post[t * 4 + r] = fp.post_mult * sigmoidf_ieee(lq);
+    float* dst = comb + t * 16 + r * 4;
+    dst[0] = cr[0], dst[1] = cr[1], dst[2] = cr[2], dst[3] = cr[3];
+  }
+}
+
+// y = bf16_rn(sum_i pre_i * R_i): one thread per (token, 8 columns), a streaming pass (R read once,
+// y written once). Requires H % 8 == 0 and 16-byte aligned R and y.
+__global__ void __launch_bounds__(256) pre_agg_vec8_kernel(const uint16_t* __restrict__ R,
+                                                           const float* __restrict__ pre,
+                                                           uint16_t* __restrict__ y, int64_t T,
+                                                           int64_t H8) {
+  const int64_t total = T * H8;
+  const int64_t H = H8 * 8;
+  for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < total;
+       u += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = u / H8;
+    const int64_t v = u - t * H8;
+    const uint16_t* rr = R + t * 4 * H + v * 8;
+    uint4 rv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) rv[i] = ld_stream_ro(rr + i * H);
+    const float4 p4 = __ldg(reinterpret_cast<const float4*>(pre + t * 4));
+    const uint32_t* r0 = &rv[0].x;
+    const uint32_t* r1 = &rv[1].x;
+    const uint32_t* r2 = &rv[2].x;
+    const uint32_t* r3 = &rv[3].x;
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float lo = p4.x * bf16_lo(r0[e]);
+      lo = fmaf(p4.y, bf16_lo(r1[e]), lo);
+      lo = fmaf(p4.z, bf16_lo(r2[e]), lo);
+      lo = fmaf(p4.w, bf16_lo(r3[e]), lo);
+      float hi = p4.x * bf16_hi(r0[e]);
+      hi = fmaf(p4.y, bf16_hi(r1[e]), hi);
+      hi = fmaf(p4.z, bf16_hi(r2[e]), hi);
+      hi = fmaf(p4.w, bf16_hi(r3[e]), hi);
+      o[e] = pack_bf16x2(lo, hi);
+    }
+    st_plain(y + t * H + v * 8, make_uint4(o[0], o[1], o[2], o[3]));
+  }
+}
+
 // ------------------------------------------------------------------------------ host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -378,18 +476,29 @@ int launch_pre_tc(const PreArgs& a, cudaStream_t s) {
   note_launches(1);
   if (cudaGetLastError() != cudaSuccess) return -4;
 
-  const int64_t nhb = (a.H + kAggCols - 1) / kAggCols;
-  if (a.T > 0x7fffffff || 1 + nhb > 65535) return -5;
-  const dim3 g2(static_cast<unsigned>(a.T), static_cast<unsigned>(1 + nhb));
   const FinishParams fp{a.iters, a.sinkhorn_eps, a.rms_eps, a.pre_eps, a.post_mult};
-  const bool vec = aligned16(a.R) && aligned16(a.y) && (a.H % 8 == 0);
-  if (vec)
-    pre_cc_finish_kernel<true><<<g2, 256, 0, s>>>(a.R, part, plan.nsplit, a.hc_scale, a.hc_base,
-                                                  a.y, a.pre, a.post, a.comb, a.T, a.H, fp);
-  else
+  const bool vec = aligned16(a.R) && aligned16(a.y) && aligned16(a.pre) && (a.H % 8 == 0);
+  if (vec) {
+    // Coefficients for all tokens, then one streaming pass for y.
+    const int64_t cb = (4 * a.T + 255) / 256;
+    if (cb > 0x7fffffff) return -5;
+    pre_tc_coef_kernel<<<static_cast<unsigned>(cb), 256, 0, s>>>(
+        part, plan.nsplit, a.hc_scale, a.hc_base, a.pre, a.post, a.comb, a.T, 4 * a.H, fp);
+    note_launches(1);
+    if (cudaGetLastError() != cudaSuccess) return -4;
+    const int64_t units = a.T * (a.H / 8);
+    int64_t ab = (units + 255) / 256;
+    const int64_t cap = static_cast<int64_t>(device_sm_count()) * 16;
+    if (ab > cap) ab = cap;
+    pre_agg_vec8_kernel<<<static_cast<unsigned>(ab), 256, 0, s>>>(a.R, a.pre, a.y, a.T, a.H / 8);
+  } else {
+    const int64_t nhb = (a.H + kAggCols - 1) / kAggCols;
+    if (a.T > 0x7fffffff || 1 + nhb > 65535) return -5;
+    const dim3 g2(static_cast<unsigned>(a.T), static_cast<unsigned>(1 + nhb));
     pre_cc_finish_kernel<false><<<g2, 256, 0, s>>>(a.R, part, plan.nsplit, a.hc_scale,
                                                    a.hc_base, a.y, a.pre, a.post, a.comb, a.T,
                                                    a.H, fp);
+  }
   note_launches(1);
   return cudaGetLastError() == cudaSuccess ? 0 : -4;
 }

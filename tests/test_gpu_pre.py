@@ -20,7 +20,7 @@ from tolerance import COEF_TOL, U32, bf16_bits_to_f64, check_bf16, check_coef
 pytestmark = pytest.mark.gpu
 
 PRE_PATHS = {"cuda_core": mhc.PRE_PATH_CUDA_CORE, "tensor": mhc.PRE_PATH_TENSOR,
-             "tensor_split": mhc.PRE_PATH_TENSOR_SPLIT}
+             "tensor_split": mhc.PRE_PATH_TENSOR_SPLIT, "tensor_fused": mhc.PRE_PATH_TENSOR_FUSED}
 
 
 def run_pre(w, path=mhc.PATH_AUTO, params=None, R_dev=None):
@@ -54,7 +54,7 @@ def compare_pre(w, outs, rows=None, label="", pre_eps=None, post_mult=None, iter
     return max(dp, dq, dc)
 
 
-@pytest.mark.parametrize("path", ["cuda_core", "tensor", "tensor_split"])
+@pytest.mark.parametrize("path", ["cuda_core", "tensor", "tensor_split", "tensor_fused"])
 def test_pre_small_workload(path):
     w = inputs.small()
     try:
@@ -74,6 +74,8 @@ def test_pre_shapes(T, H):
     if H % 2 == 0:
         compare_pre(w, run_pre(w, mhc.PRE_PATH_TENSOR), label=f"T={T} H={H} tensor")
         compare_pre(w, run_pre(w, mhc.PRE_PATH_TENSOR_SPLIT), label=f"T={T} H={H} tensor-split")
+    if H % 8 == 0 and 448 < H <= 9472:
+        compare_pre(w, run_pre(w, mhc.PRE_PATH_TENSOR_FUSED), label=f"T={T} H={H} tensor-fused")
 
 
 @pytest.mark.parametrize("T,H", [(300, 7168), (129, 1000), (1, 4096), (520, 512)])
@@ -84,7 +86,10 @@ def test_pre_tensor_path_agrees_with_cuda_core_path(T, H):
     a = run_pre(w, mhc.PRE_PATH_TENSOR)
     b = run_pre(w, mhc.PRE_PATH_CUDA_CORE)
     c = run_pre(w, mhc.PRE_PATH_TENSOR_SPLIT)
-    for other, oname in ((b, "cuda_core"), (c, "tensor-split")):
+    others = [(b, "cuda_core"), (c, "tensor-split")]
+    if H % 8 == 0 and 448 < H <= 9472:
+        others.append((run_pre(w, mhc.PRE_PATH_TENSOR_FUSED), "tensor-fused"))
+    for other, oname in others:
         for x, y, name in zip(a[1:], other[1:], ("pre", "post", "comb")):
             d = (x.double() - y.double()).abs().max().item()
             print(f"[tensor vs {oname} T={T} H={H}] {name} max|d| = {d:.2e}")
