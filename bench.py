@@ -176,12 +176,19 @@ def load_traffic():
         return {}
 
 
-def source_digest():
+# Source files that define each map's kernels; a recorded DRAM traffic figure is used only while
+# their digest matches the one it was recorded with.
+KERNEL_SOURCES = {
+    "post": ["mhc_post.cu", "mhc_device.cuh", "mhc_internal.h"],
+    "pre": ["mhc_pre_tc.cu", "mhc_pre_cc.cu", "mhc_device.cuh", "mhc_internal.h"],
+}
+
+
+def source_digest(kernel):
     import hashlib
-    from mhc_hyper_connection_02_b200 import build
     h = hashlib.sha256()
-    for s in build.sources():
-        with open(s, "rb") as f:
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "mhc_hyper_connection_02_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
@@ -197,6 +204,10 @@ def main():
     ap.add_argument("--pre-path", type=int, default=0)
     ap.add_argument("--post-path", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--only", default="both", choices=["both", "pre", "post"],
+                    help="time one map only (profiling); the JSON line is for the full step")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the workload's token count (profiling smaller cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -216,7 +227,7 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
 
-    w = inputs.WORKLOADS[args.workload]()
+    w = inputs.WORKLOADS[args.workload](T=args.tokens) if args.tokens else inputs.WORKLOADS[args.workload]()
     T, H = w.T, w.H
     dev = torch.device("cuda", local)
     R = torch.from_numpy(w.R.view(np.int16)).view(torch.bfloat16).to(dev)
@@ -235,10 +246,18 @@ def main():
                              post_mult=w.post_mult)
     stream = torch.cuda.current_stream(dev)
 
+    do_pre, do_post = args.only in ("both", "pre"), args.only in ("both", "post")
+
     def step():
+        if do_pre:
+            mhc.pre(R, hc_fn, scale, base, y=y, pre=pre, post=post, comb=comb, workspace=workspace,
+                    params=params, path=args.pre_path, stream=stream)
+        if do_post:
+            mhc.post(x, R, post, comb, out=out, path=args.post_path, stream=stream)
+
+    if not do_pre:  # post-only timing still needs valid coefficients
         mhc.pre(R, hc_fn, scale, base, y=y, pre=pre, post=post, comb=comb, workspace=workspace,
-                params=params, path=args.pre_path, stream=stream)
-        mhc.post(x, R, post, comb, out=out, path=args.post_path, stream=stream)
+                params=params, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -258,10 +277,12 @@ def main():
     start.record(stream)
     for i in range(args.steps):
         ev[i][0].record(stream)
-        mhc.pre(R, hc_fn, scale, base, y=y, pre=pre, post=post, comb=comb, workspace=workspace,
-                params=params, path=args.pre_path, stream=stream)
+        if do_pre:
+            mhc.pre(R, hc_fn, scale, base, y=y, pre=pre, post=post, comb=comb,
+                    workspace=workspace, params=params, path=args.pre_path, stream=stream)
         ev[i][1].record(stream)
-        mhc.post(x, R, post, comb, out=out, path=args.post_path, stream=stream)
+        if do_post:
+            mhc.post(x, R, post, comb, out=out, path=args.post_path, stream=stream)
         ev[i][2].record(stream)
     stop.record(stream)
     torch.cuda.synchronize()
@@ -282,7 +303,7 @@ def main():
     # End to end through the public API with host buffers: pinned H2D of the step's inputs, the
     # two calls, D2H of the step's results, all inside the timed region.
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and args.only == "both":
         hR = torch.from_numpy(w.R.view(np.int16)).view(torch.bfloat16).pin_memory()
         hx = torch.from_numpy(w.x.view(np.int16)).view(torch.bfloat16).pin_memory()
         hW = torch.from_numpy(w.hc_fn).pin_memory()
@@ -332,12 +353,15 @@ def main():
         post_avg_s = statistics.mean(post_ms) / 1e3
         pre_avg_s = statistics.mean(pre_ms) / 1e3
         pb, qb = post_bytes(T, H), pre_bytes(T, H)
-        post_gbs = pb / post_avg_s / 1e9
-        pre_gbs = qb / pre_avg_s / 1e9
-        dominant = "post" if post_avg_s >= pre_avg_s else "pre"
+        post_gbs = pb / post_avg_s / 1e9 if do_post else 0.0
+        pre_gbs = qb / pre_avg_s / 1e9 if do_pre else 0.0
+        # The roofline object describes one kernel: the post-map is a single launch and the
+        # longest kernel of the step (the split pre-map is a chain of four shorter launches,
+        # reported as a whole call under "kernels").
+        dominant = "post" if do_post else "pre"
         traffic_rec = load_traffic().get(f"{dominant}:{args.workload}")
         traffic = None
-        if traffic_rec and traffic_rec.get("source") == source_digest():
+        if traffic_rec and traffic_rec.get("source") == source_digest(dominant):
             traffic = traffic_rec.get("bytes_per_launch")
         ach = post_gbs if dominant == "post" else pre_gbs
         line = {
@@ -353,18 +377,21 @@ def main():
             "roofline": {"bound": "hbm", "kernel": f"mhc_{dominant}", "achieved": ach,
                          "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "traffic": traffic,
                          "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)"},
-            "kernels": {
-                "pre": {"us": pre_avg_s * 1e6, "algo_bytes": qb, "GBps": pre_gbs,
-                        "frac_measured": pre_gbs / hbm, "frac_8TBps": pre_gbs / 8000.0,
-                        "path": args.pre_path},
-                "post": {"us": post_avg_s * 1e6, "algo_bytes": pb, "GBps": post_gbs,
-                         "frac_measured": post_gbs / hbm, "frac_8TBps": post_gbs / 8000.0,
-                         "path": args.post_path},
-            },
+            "kernels": {},
             "gpu_launches": int(launches),
             "clocks": clocks,
             "e2e": e2e,
         }
+        if do_pre:
+            line["kernels"]["pre"] = {
+                "us": pre_avg_s * 1e6, "algo_bytes": qb, "GBps": pre_gbs,
+                "frac_measured": pre_gbs / hbm, "frac_8TBps": pre_gbs / 8000.0,
+                "path": args.pre_path}
+        if do_post:
+            line["kernels"]["post"] = {
+                "us": post_avg_s * 1e6, "algo_bytes": pb, "GBps": post_gbs,
+                "frac_measured": post_gbs / hbm, "frac_8TBps": post_gbs / 8000.0,
+                "path": args.post_path}
         if not args.no_cpu_baseline and ws == 1:
             line["cpu_baseline"] = cpu_baseline(w)
         print(json.dumps(line), flush=True)

@@ -30,6 +30,18 @@ __device__ __forceinline__ void report_timeout(int where) {
   (void)where;
 }
 
+// ------------------------------------------------------------------------------ dependent launch
+
+// Programmatic dependent launch. pdl_wait blocks until every grid this one depends on in the stream
+// has completed and its memory operations are visible (it returns at once for a grid launched
+// without the programmatic-serialisation attribute); every thread calls it before its first access
+// to global memory. pdl_trigger lets the next grid in the stream start launching once all CTAs of
+// this one have triggered or exited; that grid still waits in its own pdl_wait.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------------------ bf16 packing
 
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }

@@ -5,8 +5,28 @@
 #include <stdint.h>
 
 #include <cstddef>
+#include <utility>
 
 namespace mhc {
+
+// Launches `kernel` on stream s with programmatic stream serialisation: the grid may begin
+// launching while the previous grid in the stream finishes; the kernel orders itself behind that
+// grid with pdl_wait (mhc_device.cuh) before touching global memory.
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Device of the calling thread (this runtime instance), or -1 on error.
 int current_device();

@@ -164,6 +164,8 @@ __global__ void __launch_bounds__(kPostThreads) post_persistent_kernel(
     fence_mbarrier_init();
   }
   __syncthreads();
+  pdl_wait();  // launched as a programmatic dependent of the previous grid in the stream
+  pdl_trigger();
 
   if (tid >= kPostConsumers) {
     // Producer warp: lane 0 issues the copies.
@@ -281,10 +283,11 @@ int launch_post_persistent(const uint16_t* x, const uint16_t* R, const float* po
   const int64_t tiles = T * ((H + kPostChunk - 1) / kPostChunk);
   int64_t blocks = static_cast<int64_t>(device_sm_count()) * 3;  // 3 x 61 KB of stages per SM
   if (blocks > tiles) blocks = tiles;
-  post_persistent_kernel<<<static_cast<int>(blocks), kPostThreads, kPostSmem, s>>>(
-      x, R, post, comb, out, T, H);
+  if (launch_pdl(post_persistent_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kPostThreads),
+                 static_cast<size_t>(kPostSmem), s, x, R, post, comb, out, T, H) != cudaSuccess)
+    return -4;
   note_launches(1);
-  return cudaGetLastError() == cudaSuccess ? 0 : -4;
+  return 0;
 }
 
 }  // namespace mhc

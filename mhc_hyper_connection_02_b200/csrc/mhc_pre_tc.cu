@@ -8,16 +8,25 @@
 // columns [hi | mid | lo] padded to N = 80. Products are exact in the fp32 accumulator; the three
 // column groups are summed as (lo + mid) + hi in the epilogue.
 //
-// Kernels (one call):
+// Kernels (one call, chained with programmatic dependent launch):
 //   split   hc_fn [4H][24] fp32 -> Bw [80][4H] bf16 (K contiguous) in the workspace.
-//   proj    grid (token tiles of 128, K splits). Warp 0 issues TMA loads of R [128 x 64] and
-//           Bw [80 x 64] tiles (128-byte swizzle) into a 6-stage ring; warp 1 issues
-//           tcgen05.mma M=128 N=80 K=16 (four per 64-wide K block) into a TMEM accumulator;
-//           warps 2-5 sum the squares of their token rows from the same shared-memory tiles and,
-//           after the last block, read the accumulator (tcgen05.ld) and write the split record
-//           [split][t][32] = raw[0..23], ss -- the record format of the CUDA-core path.
-//   finish  the CUDA-core path's finish kernel: sums the split records in a fixed order, forms
-//           rstd, the logits, gates and Sinkhorn, and aggregates y.
+//   proj    persistent, one CTA per SM. The work is the (token tile of 256, 64-wide K block)
+//           grid flattened tile-major and cut into equal contiguous ranges, one per CTA, so every
+//           CTA streams the same number of blocks; a range covers pieces (tile, K interval). Warp 0
+//           issues TMA loads of two R sub-tiles [128 x 64] and one Bw tile [80 x 64] (128-byte
+//           swizzle) per stage into a 4-stage ring that runs on across pieces; warp 1 issues
+//           tcgen05.mma M=128 N=80 K=16 (four per 64-wide K block and sub-tile) into two TMEM
+//           accumulators sharing the B tile, double-buffered across pieces (512 columns), so the
+//           epilogue of one piece overlaps the loads of the next; warps 2-5 sum the squares of
+//           their token rows from the same shared-memory tiles and, after a piece, read its
+//           accumulators (tcgen05.ld) and write the record [slot][t][32] = raw[0..23], ss, slot =
+//           the piece's rank among its tile's pieces. The CTA holding a tile's last piece writes
+//           zero records into the tile's unused slots, so readers sum a fixed number of slots.
+//   coef    one token per lane quad: sums the slots in order, forms rstd, the logits, the gates
+//           and the Sinkhorn comb.
+//   agg     y = bf16_rn(sum_i pre_i R_i), one thread per (token, 8 columns): R read once more,
+//           y written once. (Unaligned R / y / pre or H % 8 != 0: the CUDA-core path's finish
+//           kernel replaces coef + agg, on the same records.)
 #include <cuda.h>
 
 #include <mutex>
@@ -27,62 +36,60 @@
 
 namespace mhc {
 
-constexpr int kTcM = 128;                          // tokens per tile (MMA M)
+constexpr int kTcM = 128;                          // tokens per MMA (M)
+constexpr int kTcSub = 2;                          // MMA sub-tiles per CTA tile sharing one B tile
+constexpr int kTcTile = kTcM * kTcSub;             // 256 tokens per CTA tile
 constexpr int kTcN = 80;                           // 3 x 24 split columns + 8 zero rows
 constexpr int kTcKB = 64;                          // K per block: one 128-byte swizzled row
-constexpr int kTcStages = 6;
-constexpr int kTcABytes = kTcM * kTcKB * 2;        // 16384
+constexpr int kTcStages = 4;
+constexpr int kTcABytes = kTcM * kTcKB * 2;        // 16384 per sub-tile
 constexpr int kTcBBytes = kTcN * kTcKB * 2;        // 10240
-constexpr int kTcStageBytes = kTcABytes + kTcBBytes;  // 26624 = 26 x 1024
+constexpr int kTcStageBytes = kTcSub * kTcABytes + kTcBBytes;  // 43008 = 42 x 1024
 constexpr int kTcThreads = 192;
-constexpr int kTcTmemCols = 128;
+constexpr int kTcTmemCols = 512;                   // 2 buffers x 2 sub-tiles x 128 columns
 constexpr int kTcSmem = 1024 + kTcStages * kTcStageBytes + 256;
-constexpr int64_t kTcSms = 148;                    // SM count the split plan is tuned for (B200)
+constexpr int64_t kTcSms = 148;                    // CTAs of the projection (B200's SM count)
+constexpr int64_t kTcMinBlocks = 8;                // K blocks per CTA at least (pipeline fill)
 
+// Work plan of the projection: W = ntiles * kblocks block-tiles over P CTAs; CTA c takes
+// [c W / P, (c + 1) W / P). A tile's K range is cut into at most S pieces.
 struct TcPlan {
-  int64_t ntiles, kblocks, kbps, nsplit;
+  int64_t ntiles, kblocks, W, P, S;
   size_t bw_bytes;  // workspace bytes of Bw, rounded to 1 KB
 };
 
 static TcPlan tc_plan(int64_t T, int64_t H) {
   TcPlan p;
   const int64_t K = 4 * H;
-  p.ntiles = (T + kTcM - 1) / kTcM;
+  p.ntiles = (T + kTcTile - 1) / kTcTile;
   p.kblocks = (K + kTcKB - 1) / kTcKB;
-  // Splits per tile: at least 3 waves of CTAs (one CTA per SM); then the fewest splits whose last
-  // wave is at least 90% full (each CTA's pipeline fill is exposed, so longer CTAs are better),
-  // else the fullest last wave seen.
-  const int64_t ns_min = (3 * kTcSms + p.ntiles - 1) / p.ntiles;
-  int64_t best_ns = ns_min > p.kblocks ? p.kblocks : (ns_min < 1 ? 1 : ns_min);
-  double best_eff = -1.0;
-  for (int64_t ns = best_ns; ns <= ns_min + 16 && ns <= p.kblocks; ++ns) {
-    const int64_t kbps = (p.kblocks + ns - 1) / ns;
-    const int64_t nsplit = (p.kblocks + kbps - 1) / kbps;
-    const int64_t ctas = nsplit * p.ntiles;
-    const int64_t waves = (ctas + kTcSms - 1) / kTcSms;
-    const double eff = static_cast<double>(ctas) / static_cast<double>(waves * kTcSms);
-    if (eff > best_eff + 1e-9) {
-      best_eff = eff;
-      best_ns = ns;
-    }
-    if (eff >= 0.9) break;
-  }
-  p.kbps = (p.kblocks + best_ns - 1) / best_ns;
-  p.nsplit = (p.kblocks + p.kbps - 1) / p.kbps;
+  p.W = p.ntiles * p.kblocks;
+  p.P = p.W / kTcMinBlocks;
+  if (p.P > kTcSms) p.P = kTcSms;
+  if (p.P < 1) p.P = 1;
+  // A tile spans kblocks consecutive units; a CTA range holds at least floor(W / P) of them, so a
+  // tile meets at most floor(kblocks P / W) + 2 ranges.
+  p.S = p.kblocks * p.P / p.W + 2;
+  if (p.S > p.P) p.S = p.P;
   p.bw_bytes = (static_cast<size_t>(kTcN) * K * 2 + 1023) / 1024 * 1024;
   return p;
 }
 
+// First CTA whose range contains flattened unit x.
+__host__ __device__ __forceinline__ int64_t tc_first_cta(int64_t x, int64_t P, int64_t W) {
+  return ((x + 1) * P - 1) / W;
+}
+
 bool pre_tc_supported(int64_t T, int64_t H) {
   // TMA needs 16-byte global strides: rows of R (8H bytes) and of Bw (8H bytes).
-  return T >= 1 && H >= 2 && H % 2 == 0 && tc_plan(T, H).nsplit <= 65535 &&
-         (T + kTcM - 1) / kTcM <= 0x7fffffff;
+  return T >= 1 && H >= 2 && H % 2 == 0 && (T + kTcTile - 1) / kTcTile <= 0x7fffffff &&
+         (4 * H + kTcKB - 1) / kTcKB <= 0x7fffffff;
 }
 
 size_t pre_tc_workspace_bytes(int64_t T, int64_t H) {
   if (T <= 0 || H <= 0 || H % 2 != 0) return 0;
   const TcPlan p = tc_plan(T, H);
-  return p.bw_bytes + static_cast<size_t>(p.nsplit) * static_cast<size_t>(T) * 32 * sizeof(float);
+  return p.bw_bytes + static_cast<size_t>(p.S) * static_cast<size_t>(T) * 32 * sizeof(float);
 }
 
 // ------------------------------------------------------------------------------ device helpers
@@ -152,6 +159,8 @@ __device__ __forceinline__ void tmem_wait_ld() {
 // 72..79 are zero.
 __global__ void __launch_bounds__(256) pre_tc_split_kernel(const float* __restrict__ W,
                                                            uint16_t* __restrict__ Bw, int64_t K) {
+  pdl_wait();  // the previous call's projection may still read Bw
+  pdl_trigger();
   for (int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; k < K;
        k += (int64_t)gridDim.x * blockDim.x) {
 #pragma unroll 4
@@ -173,28 +182,34 @@ __global__ void __launch_bounds__(256) pre_tc_split_kernel(const float* __restri
 
 __global__ void __launch_bounds__(kTcThreads, 1) pre_tc_proj_kernel(
     const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmB,
-    float* __restrict__ part, int64_t T, int kblocks, int kbps) {
+    float* __restrict__ part, int64_t T, int64_t W, int KB, int S) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTcStages * kTcStageBytes);
   uint64_t* empty = full + kTcStages;
-  uint64_t* accum = empty + kTcStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  uint64_t* afull = empty + kTcStages;  // [2] accumulator buffer b complete (MMA commit)
+  uint64_t* aempty = afull + 2;         // [2] accumulator buffer b read out (4 warps)
+  uint64_t* done = aempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  static_assert((2 * kTcStages + 5) * 8 + 4 <= 256, "barrier area");
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int tile = blockIdx.x;
-  const int split = blockIdx.y;
-  const int kb0 = split * kbps;
-  const int nkb = min(kblocks, kb0 + kbps) - kb0;  // >= 1 by the plan
+  const int64_t P = gridDim.x;
+  const int64_t c = blockIdx.x;
+  const int64_t lo = c * W / P, hi = (c + 1) * W / P;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1 + 4);  // MMA commit + one arrival per sum-of-squares warp
     }
-    mbar_init(accum, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&afull[b], 1);
+      mbar_init(&aempty[b], 4);
+    }
+    mbar_init(done, 1);
     fence_mbarrier_init();
   }
   if (warp == 1) {
@@ -208,109 +223,176 @@ __global__ void __launch_bounds__(kTcThreads, 1) pre_tc_proj_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
-      int issued = 0;
+      int64_t n = 0;
       bool ok = true;
-      for (int i = 0; i < nkb; ++i) {
-        const int s = i % kTcStages;
-        const uint32_t ph = static_cast<uint32_t>(i / kTcStages) & 1u;
-        if (i >= kTcStages && !mbar_wait(&empty[s], ph ^ 1u, 10)) {
-          ok = false;
-          break;
+      for (int64_t u = lo; u < hi && ok;) {
+        const int64_t tile = u / KB;
+        const int kbs = static_cast<int>(u - tile * KB);
+        const int kbe = static_cast<int>(min(static_cast<int64_t>(KB), kbs + (hi - u)));
+        for (int kb = kbs; kb < kbe; ++kb, ++n) {
+          const int s = static_cast<int>(n % kTcStages);
+          const uint32_t ph = static_cast<uint32_t>(n / kTcStages) & 1u;
+          if (n >= kTcStages && !mbar_wait(&empty[s], ph ^ 1u, 10)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * kTcStageBytes;
+          mbar_arrive_expect_tx(&full[s], kTcStageBytes);
+#pragma unroll
+          for (int v = 0; v < kTcSub; ++v)
+            tma_load_2d(st + v * kTcABytes, &tmR, kb * kTcKB,
+                        static_cast<int>(tile * kTcTile + v * kTcM), &full[s]);
+          tma_load_2d(st + kTcSub * kTcABytes, &tmB, kb * kTcKB, 0, &full[s]);
         }
-        uint8_t* st = smem + s * kTcStageBytes;
-        mbar_arrive_expect_tx(&full[s], kTcStageBytes);
-        tma_load_2d(st, &tmR, (kb0 + i) * kTcKB, tile * kTcM, &full[s]);
-        tma_load_2d(st + kTcABytes, &tmB, (kb0 + i) * kTcKB, 0, &full[s]);
-        ++issued;
+        u += kbe - kbs;
       }
       if (!ok) {  // do not leave while copies into shared memory are in flight
-        for (int i = issued - kTcStages; i < issued; ++i)
+        for (int64_t i = n - kTcStages; i < n; ++i)
           if (i >= 0)
             mbar_wait(&full[i % kTcStages], static_cast<uint32_t>(i / kTcStages) & 1u, 15);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
+      int64_t n = 0;
+      int64_t p = 0;
       bool ok = true;
-      for (int i = 0; i < nkb; ++i) {
-        const int s = i % kTcStages;
-        const uint32_t ph = static_cast<uint32_t>(i / kTcStages) & 1u;
-        if (!mbar_wait(&full[s], ph, 11)) {
+      for (int64_t u = lo; u < hi && ok; ++p) {
+        const int64_t tile = u / KB;
+        const int kbs = static_cast<int>(u - tile * KB);
+        const int kbe = static_cast<int>(min(static_cast<int64_t>(KB), kbs + (hi - u)));
+        const int b = static_cast<int>(p & 1);
+        if (p >= 2 && !mbar_wait(&aempty[b], static_cast<uint32_t>((p >> 1) - 1) & 1u, 16)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t a = smem_u32(smem + s * kTcStageBytes);
-        const uint64_t adesc = sw128_desc(a);
-        const uint64_t bdesc = sw128_desc(a + kTcABytes);
+        const uint32_t dt = tmem + static_cast<uint32_t>(b * kTcSub * kTcM);
+        for (int kb = kbs; kb < kbe; ++kb, ++n) {
+          const int s = static_cast<int>(n % kTcStages);
+          const uint32_t ph = static_cast<uint32_t>(n / kTcStages) & 1u;
+          if (!mbar_wait(&full[s], ph, 11)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a = smem_u32(smem + s * kTcStageBytes);
+          const uint64_t bdesc = sw128_desc(a + kTcSub * kTcABytes);
 #pragma unroll
-        for (int k = 0; k < kTcKB / 16; ++k)  // +32 bytes along the swizzled row per K=16 step
-          umma_bf16(tmem, adesc + 2 * k, bdesc + 2 * k, (i > 0 || k > 0) ? 1u : 0u);
-        umma_commit(&empty[s]);
+          for (int v = 0; v < kTcSub; ++v) {
+            const uint64_t adesc = sw128_desc(a + v * kTcABytes);
+#pragma unroll
+            for (int k = 0; k < kTcKB / 16; ++k)  // +32 bytes along the swizzled row per K=16 step
+              umma_bf16(dt + static_cast<uint32_t>(v * kTcM), adesc + 2 * k, bdesc + 2 * k,
+                        (kb > kbs || k > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        umma_commit(&afull[b]);
+        u += kbe - kbs;
       }
-      umma_commit(accum);
-      if (!ok) mbar_wait(accum, 0, 14);
+      // Every issued MMA has finished before TMEM is released.
+      umma_commit(done);
+      mbar_wait(done, 0, 14);
     }
   } else {
-    // Warps 2..5: TMEM lane quarter q = warp % 4 holds accumulator rows 32q..32q+31; the same
-    // thread sums the squares of that row.
+    // Warps 2..5: TMEM lane quarter q = warp % 4 holds rows 32q..32q+31 of each sub-tile's
+    // accumulator; the same thread sums the squares of those rows (one per sub-tile).
     const int q = warp & 3;
     const int row = q * 32 + lane;
-    float ss0 = 0.f, ss1 = 0.f;
+    int64_t n = 0;
+    int64_t p = 0;
     bool ok = true;
-    for (int i = 0; i < nkb; ++i) {
-      const int s = i % kTcStages;
-      const uint32_t ph = static_cast<uint32_t>(i / kTcStages) & 1u;
-      // Every lane waits; the warp continues only if all of them saw the stage (warp-uniform, so
-      // the __syncwarp and the .sync.aligned TMEM loads below are never reached divergently).
-      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, 12))) {
+    for (int64_t u = lo; u < hi && ok; ++p) {
+      const int64_t tile = u / KB;
+      const int kbs = static_cast<int>(u - tile * KB);
+      const int kbe = static_cast<int>(min(static_cast<int64_t>(KB), kbs + (hi - u)));
+      float ss0[kTcSub], ss1[kTcSub];
+#pragma unroll
+      for (int v = 0; v < kTcSub; ++v) ss0[v] = ss1[v] = 0.f;
+      for (int kb = kbs; kb < kbe; ++kb, ++n) {
+        const int s = static_cast<int>(n % kTcStages);
+        const uint32_t ph = static_cast<uint32_t>(n / kTcStages) & 1u;
+        // Every lane waits; the warp continues only if all of them saw the stage (warp-uniform,
+        // so the __syncwarp and the .sync.aligned TMEM loads below are never reached divergently).
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, 12))) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int v = 0; v < kTcSub; ++v) {
+          // Row `row` of the swizzled tile is its own 128 contiguous bytes (chunks permuted within
+          // it), and a sum does not depend on element order. Each lane starts at a different
+          // 16-byte chunk, so the 8 lanes of a load phase hit 8 different bank groups.
+          const uint4* rp = reinterpret_cast<const uint4*>(smem + s * kTcStageBytes +
+                                                           v * kTcABytes + row * 128);
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc) {
+            const uint4 w = rp[cc ^ (lane & 7)];
+            const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float x0 = bf16_lo(w4[e]), x1 = bf16_hi(w4[e]);
+              ss0[v] = fmaf(x0, x0, ss0[v]);
+              ss1[v] = fmaf(x1, x1, ss1[v]);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
+      if (!ok) break;
+      const int b = static_cast<int>(p & 1);
+      if (!__all_sync(0xffffffffu, mbar_wait(&afull[b], static_cast<uint32_t>(p >> 1) & 1u, 13))) {
         ok = false;
         break;
       }
-      // Row `row` of the swizzled tile is its own 128 contiguous bytes (chunks permuted within
-      // it), and a sum does not depend on element order. Each lane starts at a different 16-byte
-      // chunk, so the 8 lanes of a load phase hit 8 different bank groups.
-      const uint4* rp = reinterpret_cast<const uint4*>(smem + s * kTcStageBytes + row * 128);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 v = rp[c ^ (lane & 7)];
-        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a = bf16_lo(u[e]), b = bf16_hi(u[e]);
-          ss0 = fmaf(a, a, ss0);
-          ss1 = fmaf(b, b, ss1);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-    }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(accum, 0, 13))) {
       tc_fence_after();
-      uint32_t d[5][16];
-      const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      const int64_t slot = c - tc_first_cta(tile * KB, P, W);
+      const bool last_piece = (kbe == KB);
 #pragma unroll
-      for (int c = 0; c < 5; ++c) tmem_ld16(tbase + c * 16, d[c]);
-      tmem_wait_ld();
-      const int64_t t = static_cast<int64_t>(tile) * kTcM + row;
-      if (t < T) {
-        float raw[kMix];
+      for (int v = 0; v < kTcSub; ++v) {
+        uint32_t d[5][16];
+        const uint32_t tbase = tmem + static_cast<uint32_t>((b * kTcSub + v) * kTcM) +
+                               (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll
-        for (int j = 0; j < kMix; ++j) {
-          const float hi = __uint_as_float(d[j / 16][j % 16]);
-          const float mid = __uint_as_float(d[(kMix + j) / 16][(kMix + j) % 16]);
-          const float lo = __uint_as_float(d[(2 * kMix + j) / 16][(2 * kMix + j) % 16]);
-          raw[j] = (lo + mid) + hi;
+        for (int cc = 0; cc < 5; ++cc) tmem_ld16(tbase + cc * 16, d[cc]);
+        tmem_wait_ld();
+        const int64_t t = tile * kTcTile + v * kTcM + row;
+        if (t < T) {
+          float raw[kMix];
+#pragma unroll
+          for (int j = 0; j < kMix; ++j) {
+            const float hi3 = __uint_as_float(d[j / 16][j % 16]);
+            const float mid = __uint_as_float(d[(kMix + j) / 16][(kMix + j) % 16]);
+            const float lo3 = __uint_as_float(d[(2 * kMix + j) / 16][(2 * kMix + j) % 16]);
+            raw[j] = (lo3 + mid) + hi3;
+          }
+          float4* rec = reinterpret_cast<float4*>(part + (slot * T + t) * 32);
+#pragma unroll
+          for (int w = 0; w < 6; ++w)
+            rec[w] = make_float4(raw[4 * w], raw[4 * w + 1], raw[4 * w + 2], raw[4 * w + 3]);
+          rec[6] = make_float4(ss0[v] + ss1[v], 0.f, 0.f, 0.f);
+          if (last_piece) {
+            const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int64_t sl = slot + 1; sl < S; ++sl) {
+              float4* zr = reinterpret_cast<float4*>(part + (sl * T + t) * 32);
+#pragma unroll
+              for (int w = 0; w < 7; ++w) zr[w] = z;
+            }
+          }
         }
-        float4* rec = reinterpret_cast<float4*>(part + (static_cast<int64_t>(split) * T + t) * 32);
-#pragma unroll
-        for (int v = 0; v < 6; ++v)
-          rec[v] = make_float4(raw[4 * v], raw[4 * v + 1], raw[4 * v + 2], raw[4 * v + 3]);
-        rec[6] = make_float4(ss0 + ss1, 0.f, 0.f, 0.f);
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&aempty[b]);
+      u += kbe - kbs;
     }
   }
   tc_fence_before();
@@ -323,11 +405,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) pre_tc_proj_kernel(
   }
 }
 
-// Coefficients from the split records [split][t][32] (raw[0..23], ss): one token per lane quad,
-// 8 tokens per warp. Lane r of a quad sums, over the splits in order, the components it needs
-// (pre r, post r, comb row r, ss) and runs its row of the Sinkhorn.
+// Coefficients from the records [slot][t][32] (raw[0..23], ss): one token per lane quad, 8 tokens
+// per warp. Lane r of a quad sums, over the slots in order, the components it needs (pre r, post
+// r, comb row r, ss) and runs its row of the Sinkhorn.
 __global__ void __launch_bounds__(256) pre_tc_coef_kernel(const float* __restrict__ part,
-                                                          int64_t nsplit,
+                                                          int nslot,
                                                           const float* __restrict__ scale,
                                                           const float* __restrict__ base,
                                                           float* __restrict__ pre,
@@ -339,43 +421,48 @@ __global__ void __launch_bounds__(256) pre_tc_coef_kernel(const float* __restric
   const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 2;
   const bool live = t < T;
   const int64_t tt = live ? t : 0;
-  float4 g0 = make_float4(0.f, 0.f, 0.f, 0.f), g1 = g0, gc = g0, g6 = g0;
-  for (int64_t s = 0; s < nsplit; ++s) {
+  pdl_wait();
+  pdl_trigger();
+  float4 g0 = make_float4(0.f, 0.f, 0.f, 0.f), g1 = g0, gc = g0;
+  float g6 = 0.f;
+#pragma unroll 2
+  for (int s = 0; s < nslot; ++s) {
     const float4* rec = reinterpret_cast<const float4*>(part + (s * T + tt) * 32);
-    const float4 a0 = __ldg(rec), a1 = __ldg(rec + 1), ac = __ldg(rec + 2 + r), a6 = __ldg(rec + 6);
+    const float4 a0 = __ldg(rec), a1 = __ldg(rec + 1), ac = __ldg(rec + 2 + r);
+    const float a6 = __ldg(reinterpret_cast<const float*>(rec + 6));
     g0.x += a0.x, g0.y += a0.y, g0.z += a0.z, g0.w += a0.w;
     g1.x += a1.x, g1.y += a1.y, g1.z += a1.z, g1.w += a1.w;
     gc.x += ac.x, gc.y += ac.y, gc.z += ac.z, gc.w += ac.w;
-    g6.x += a6.x;
+    g6 += a6;
   }
-  const float p0[4] = {g0.x, g0.y, g0.z, g0.w};
-  const float p1[4] = {g1.x, g1.y, g1.z, g1.w};
-  const float rstd =
-      __fdiv_rn(1.0f, __fsqrt_rn(__fdiv_rn(g6.x, static_cast<float>(K)) + fp.rms_eps));
-  const float lp = fmaf(p0[r] * rstd, __ldg(scale), __ldg(base + r));
-  const float lq = fmaf(p1[r] * rstd, __ldg(scale + 1), __ldg(base + 4 + r));
+  const float rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fdiv_rn(g6, static_cast<float>(K)) + fp.rms_eps));
+  const float g0r = r == 0 ? g0.x : r == 1 ? g0.y : r == 2 ? g0.z : g0.w;
+  const float g1r = r == 0 ? g1.x : r == 1 ? g1.y : r == 2 ? g1.z : g1.w;
+  const float lp = fmaf(g0r * rstd, __ldg(scale), __ldg(base + r));
+  const float lq = fmaf(g1r * rstd, __ldg(scale + 1), __ldg(base + 4 + r));
   const float s2 = __ldg(scale + 2);
   float cr[4] = {fmaf(gc.x * rstd, s2, __ldg(base + 8 + 4 * r)),
                  fmaf(gc.y * rstd, s2, __ldg(base + 9 + 4 * r)),
                  fmaf(gc.z * rstd, s2, __ldg(base + 10 + 4 * r)),
                  fmaf(gc.w * rstd, s2, __ldg(base + 11 + 4 * r))};
+  if (live) pre[t * 4 + r] = sigmoidf_ieee(lp) + fp.pre_eps;
   sinkhorn_quad(cr, fp.iters, fp.sinkhorn_eps);  // every lane takes part
   if (live) {
-    pre[t * 4 + r] = sigmoidf_ieee(lp) + fp.pre_eps;
     post[t * 4 + r] = fp.post_mult * sigmoidf_ieee(lq);
-    float* dst = comb + t * 16 + r * 4;
-    dst[0] = cr[0], dst[1] = cr[1], dst[2] = cr[2], dst[3] = cr[3];
+    *reinterpret_cast<float4*>(comb + t * 16 + r * 4) = make_float4(cr[0], cr[1], cr[2], cr[3]);
   }
 }
 
 // y = bf16_rn(sum_i pre_i * R_i): one thread per (token, 8 columns), a streaming pass (R read once,
-// y written once). Requires H % 8 == 0 and 16-byte aligned R and y.
+// y written once). Requires H % 8 == 0 and 16-byte aligned R, y and pre.
 __global__ void __launch_bounds__(256) pre_agg_vec8_kernel(const uint16_t* __restrict__ R,
                                                            const float* __restrict__ pre,
                                                            uint16_t* __restrict__ y, int64_t T,
                                                            int64_t H8) {
   const int64_t total = T * H8;
   const int64_t H = H8 * 8;
+  pdl_wait();
+  pdl_trigger();
   for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < total;
        u += (int64_t)gridDim.x * blockDim.x) {
     const int64_t t = u / H8;
@@ -392,15 +479,15 @@ __global__ void __launch_bounds__(256) pre_agg_vec8_kernel(const uint16_t* __res
     uint32_t o[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      float lo = p4.x * bf16_lo(r0[e]);
-      lo = fmaf(p4.y, bf16_lo(r1[e]), lo);
-      lo = fmaf(p4.z, bf16_lo(r2[e]), lo);
-      lo = fmaf(p4.w, bf16_lo(r3[e]), lo);
-      float hi = p4.x * bf16_hi(r0[e]);
-      hi = fmaf(p4.y, bf16_hi(r1[e]), hi);
-      hi = fmaf(p4.z, bf16_hi(r2[e]), hi);
-      hi = fmaf(p4.w, bf16_hi(r3[e]), hi);
-      o[e] = pack_bf16x2(lo, hi);
+      float a = p4.x * bf16_lo(r0[e]);
+      a = fmaf(p4.y, bf16_lo(r1[e]), a);
+      a = fmaf(p4.z, bf16_lo(r2[e]), a);
+      a = fmaf(p4.w, bf16_lo(r3[e]), a);
+      float b = p4.x * bf16_hi(r0[e]);
+      b = fmaf(p4.y, bf16_hi(r1[e]), b);
+      b = fmaf(p4.z, bf16_hi(r2[e]), b);
+      b = fmaf(p4.w, bf16_hi(r3[e]), b);
+      o[e] = pack_bf16x2(a, b);
     }
     st_plain(y + t * H + v * 8, make_uint4(o[0], o[1], o[2], o[3]));
   }
@@ -465,39 +552,40 @@ int launch_pre_tc(const PreArgs& a, cudaStream_t s) {
 
   const int64_t sb = (K + 255) / 256;
   const int split_blocks = static_cast<int>(sb < 4096 ? sb : 4096);
-  pre_tc_split_kernel<<<split_blocks, 256, 0, s>>>(a.hc_fn, Bw, K);
+  if (launch_pdl(pre_tc_split_kernel, dim3(split_blocks), dim3(256), 0, s,
+                 static_cast<const float*>(a.hc_fn), Bw, K) != cudaSuccess)
+    return -4;
   note_launches(1);
-  if (cudaGetLastError() != cudaSuccess) return -4;
 
-  const dim3 grid(static_cast<unsigned>(plan.ntiles), static_cast<unsigned>(plan.nsplit));
-  pre_tc_proj_kernel<<<grid, kTcThreads, kTcSmem, s>>>(mR, mB, part, a.T,
-                                                       static_cast<int>(plan.kblocks),
-                                                       static_cast<int>(plan.kbps));
+  if (launch_pdl(pre_tc_proj_kernel, dim3(static_cast<unsigned>(plan.P)), dim3(kTcThreads),
+                 static_cast<size_t>(kTcSmem), s, mR, mB, part, a.T, plan.W,
+                 static_cast<int>(plan.kblocks), static_cast<int>(plan.S)) != cudaSuccess)
+    return -4;
   note_launches(1);
-  if (cudaGetLastError() != cudaSuccess) return -4;
 
   const FinishParams fp{a.iters, a.sinkhorn_eps, a.rms_eps, a.pre_eps, a.post_mult};
-  const bool vec = aligned16(a.R) && aligned16(a.y) && aligned16(a.pre) && (a.H % 8 == 0);
-  if (vec) {
-    // Coefficients for all tokens, then one streaming pass for y.
+  const bool vec = aligned16(a.R) && aligned16(a.y) && aligned16(a.comb) && (a.H % 8 == 0);
+  if (vec && aligned16(a.pre)) {
     const int64_t cb = (4 * a.T + 255) / 256;
     if (cb > 0x7fffffff) return -5;
-    pre_tc_coef_kernel<<<static_cast<unsigned>(cb), 256, 0, s>>>(
-        part, plan.nsplit, a.hc_scale, a.hc_base, a.pre, a.post, a.comb, a.T, 4 * a.H, fp);
+    if (launch_pdl(pre_tc_coef_kernel, dim3(static_cast<unsigned>(cb)), dim3(256), 0, s,
+                   static_cast<const float*>(part), static_cast<int>(plan.S), a.hc_scale,
+                   a.hc_base, a.pre, a.post, a.comb, a.T, 4 * a.H, fp) != cudaSuccess)
+      return -4;
     note_launches(1);
-    if (cudaGetLastError() != cudaSuccess) return -4;
     const int64_t units = a.T * (a.H / 8);
     int64_t ab = (units + 255) / 256;
     const int64_t cap = static_cast<int64_t>(device_sm_count()) * 16;
     if (ab > cap) ab = cap;
-    pre_agg_vec8_kernel<<<static_cast<unsigned>(ab), 256, 0, s>>>(a.R, a.pre, a.y, a.T, a.H / 8);
+    if (launch_pdl(pre_agg_vec8_kernel, dim3(static_cast<unsigned>(ab)), dim3(256), 0, s, a.R,
+                   static_cast<const float*>(a.pre), a.y, a.T, a.H / 8) != cudaSuccess)
+      return -4;
   } else {
     const int64_t nhb = (a.H + kAggCols - 1) / kAggCols;
     if (a.T > 0x7fffffff || 1 + nhb > 65535) return -5;
     const dim3 g2(static_cast<unsigned>(a.T), static_cast<unsigned>(1 + nhb));
-    pre_cc_finish_kernel<false><<<g2, 256, 0, s>>>(a.R, part, plan.nsplit, a.hc_scale,
-                                                   a.hc_base, a.y, a.pre, a.post, a.comb, a.T,
-                                                   a.H, fp);
+    pre_cc_finish_kernel<false><<<g2, 256, 0, s>>>(a.R, part, plan.S, a.hc_scale, a.hc_base,
+                                                   a.y, a.pre, a.post, a.comb, a.T, a.H, fp);
   }
   note_launches(1);
   return cudaGetLastError() == cudaSuccess ? 0 : -4;
