@@ -219,6 +219,7 @@ def main():
     import torch.distributed as dist
     import mhc_hyper_connection_02_b200 as mhc
     from mhc_hyper_connection_02_b200 import inputs
+    from mhc_hyper_connection_02_b200.shard import global_max, throughput
 
     ws, rank, local = dist_env()
     torch.cuda.set_device(local)
@@ -295,10 +296,7 @@ def main():
     total_ms = start.elapsed_time(stop)
     pre_ms = [a.elapsed_time(b) for a, b, _ in ev]
     post_ms = [b.elapsed_time(c) for _, b, c in ev]
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if ws > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = global_max(total_ms, device=dev)
 
     # End to end through the public API with host buffers: pinned H2D of the step's inputs, the
     # two calls, D2H of the step's results, all inside the timed region.
@@ -342,10 +340,8 @@ def main():
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        te = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
-        if ws > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": ws * T * e2e_steps / (float(te.item()) / 1e3), "unit": UNIT,
+        e2e = {"value": throughput(T, ws, e2e_steps, global_max(a.elapsed_time(b), device=dev)),
+               "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     if rank == 0:
@@ -366,7 +362,7 @@ def main():
         ach = post_gbs if dominant == "post" else pre_gbs
         line = {
             "metric": METRIC,
-            "value": ws * T * args.steps / (max_ms / 1e3),
+            "value": throughput(T, ws, args.steps, max_ms),
             "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
