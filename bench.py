@@ -193,6 +193,38 @@ def source_digest(kernel):
     return h.hexdigest()[:16]
 
 
+def time_extras(mhc, R, y, pre, post, comb, scale, base, params, stream, T, H, dev, reps=10):
+    """Device time of the pre-map entries that take an external projection (one split), on the
+    step's residual: algorithmic bytes R (8H) + y (2H) + dot_mix (96) + sqrsum (4, external only)
+    + pre/post/comb (96) per token."""
+    import torch
+    g = torch.Generator(device=dev).manual_seed(5)
+    dot = torch.randn((1, T, 24), generator=g, device=dev) * 0.01
+    sq = torch.full((1, T), float(4 * H), device=dev)
+    calls = {
+        "pre_big_fuse": (lambda: mhc.pre_big_fuse(dot, sq, R, scale, base, 4 * H, y=y, pre=pre,
+                                                  post=post, comb=comb, params=params,
+                                                  stream=stream), T * (10 * H + 196)),
+        "pre_big_fuse_with_prenorm": (lambda: mhc.pre_big_fuse_with_prenorm(
+            dot[0], R, scale, base, y=y, pre=pre, post=post, comb=comb, params=params,
+            stream=stream), T * (10 * H + 192)),
+    }
+    out = {}
+    for name, (fn, nbytes) in calls.items():
+        for _ in range(3):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        us = a.elapsed_time(b) / reps * 1e3
+        out[name] = {"us": us, "algo_bytes": nbytes, "GBps": nbytes / us / 1e3}
+    assert mhc.device_status() == 0
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -209,6 +241,8 @@ def main():
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the workload's token count (profiling smaller cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip timing the entries beside the step (pre from an external projection)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -344,6 +378,10 @@ def main():
                "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
+    extras = None
+    if not args.no_extras and args.only == "both":
+        extras = time_extras(mhc, R, y, pre, post, comb, scale, base, params, stream, T, H, dev)
+
     if rank == 0:
         hbm, tflops, peak_src = load_peaks()
         post_avg_s = statistics.mean(post_ms) / 1e3
@@ -388,6 +426,10 @@ def main():
                 "us": post_avg_s * 1e6, "algo_bytes": pb, "GBps": post_gbs,
                 "frac_measured": post_gbs / hbm, "frac_8TBps": post_gbs / 8000.0,
                 "path": args.post_path}
+        if extras:
+            for v in extras.values():
+                v["frac_measured"] = v["GBps"] / hbm
+            line["extras"] = extras
         if not args.no_cpu_baseline and ws == 1:
             line["cpu_baseline"] = cpu_baseline(w)
         print(json.dumps(line), flush=True)

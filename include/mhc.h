@@ -213,6 +213,43 @@ MHC_API int mhc_pre_noalloc(const uint16_t* R, const float* hc_fn, const float* 
                             float* comb, int64_t T, int64_t H, const mhc_params* p,
                             mhc_stream_t stream);
 
+/*
+ * mhc_pre_big_fuse -- the pre-map from a projection computed elsewhere ("FlashInfer mHC module deep
+ * dive" §3.1-3.4: mhc_pre_big_fuse; §5.2 reference math). The projection and the sum of squares
+ * arrive as num_splits partial sums (for instance from a split-K GEMM), summed here in split order:
+ *
+ *   dot_mix  [num_splits][T][24] fp32   raw projection partials, sum_k R_flat[t][k] * hc_fn[k][j]
+ *   sqrsum   [num_splits][T]     fp32   partials of sum_k R_flat[t][k]^2
+ *   num_splits                          1, 2, 4, 8 or 16 (the values the page allows)
+ *   k                                   RMS denominator (>= 1; 4H for the mHC row):
+ *                                       rstd = 1 / sqrt(sum(sqrsum) / k + rms_eps)
+ *   R, hc_scale, hc_base, y, pre, post, comb, p: as mhc_pre (pre is an output here too, although
+ *                                       FlashInfer's entry does not return it)
+ *
+ * logits l = sum(dot_mix) * rstd * hc_scale[group] + hc_base, then gates, Sinkhorn and y as in
+ * mhc_pre. Needs no workspace. Any H >= 1 and alignment (H % 8 == 0 with 16-byte aligned R and y
+ * takes 16-byte accesses; FlashInfer requires H % 8 == 0).
+ * Errors: MHC_ERR_INVALID_ARG (null array, T < 0, H <= 0, num_splits not in {1,2,4,8,16}, k < 1,
+ * a parameter outside its range); MHC_ERR_ALIAS when y, pre, post or comb overlaps an input or
+ * one another.
+ */
+MHC_API int mhc_pre_big_fuse(const float* dot_mix, const float* sqrsum, int num_splits, int64_t k,
+                             const uint16_t* R, const float* hc_scale, const float* hc_base,
+                             uint16_t* y, float* pre, float* post, float* comb, int64_t T,
+                             int64_t H, const mhc_params* p, mhc_stream_t stream);
+
+/*
+ * mhc_pre_big_fuse_with_prenorm -- as mhc_pre_big_fuse with one split, but the sum of squares is
+ * formed here from R and k is 4H ("FlashInfer mHC module deep dive" §4).
+ *
+ *   dot_mix  [T][24] fp32   raw projection (a [1][T][24] tensor has the same layout)
+ */
+MHC_API int mhc_pre_big_fuse_with_prenorm(const float* dot_mix, const uint16_t* R,
+                                          const float* hc_scale, const float* hc_base,
+                                          uint16_t* y, float* pre, float* post, float* comb,
+                                          int64_t T, int64_t H, const mhc_params* p,
+                                          mhc_stream_t stream);
+
 /* Number of kernel launches this process has enqueued through the library so far (all devices,
  * all threads). A diagnostic counter for benchmarks: take the difference around a region. */
 MHC_API uint64_t mhc_launch_count(void);

@@ -40,7 +40,8 @@ POST_PATH_SCALAR = 13
 EXPORTED_SYMBOLS = (
     "mhc_default_params", "mhc_pre", "mhc_pre_workspace_bytes", "mhc_post", "mhc_sinkhorn",
     "mhc_pre_with_path", "mhc_post_with_path", "mhc_device_status", "mhc_status_string",
-    "mhc_version", "mhc_launch_count", "mhc_pre_noalloc",
+    "mhc_version", "mhc_launch_count", "mhc_pre_noalloc", "mhc_pre_big_fuse",
+    "mhc_pre_big_fuse_with_prenorm",
 )
 
 
@@ -96,6 +97,12 @@ def lib() -> ctypes.CDLL:
     L.mhc_pre_noalloc.restype = ctypes.c_int
     L.mhc_pre_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64,
                                   ctypes.POINTER(Params), _P]
+    L.mhc_pre_big_fuse.restype = ctypes.c_int
+    L.mhc_pre_big_fuse.argtypes = [_P, _P, ctypes.c_int, _I64, _P, _P, _P, _P, _P, _P, _P, _I64,
+                                   _I64, ctypes.POINTER(Params), _P]
+    L.mhc_pre_big_fuse_with_prenorm.restype = ctypes.c_int
+    L.mhc_pre_big_fuse_with_prenorm.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64,
+                                                ctypes.POINTER(Params), _P]
     L.mhc_launch_count.restype = ctypes.c_uint64
     L.mhc_launch_count.argtypes = []
     _lib = L
@@ -186,6 +193,71 @@ def pre(R, hc_fn, hc_scale, hc_base, *, y=None, pre=None, post=None, comb=None, 
                                  _ptr(pre), _ptr(post), _ptr(comb), _ptr(workspace), wsb, T, H,
                                  ctypes.byref(p), int(path), _stream(stream))
     _check(st, "mhc_pre")
+    return y, pre, post, comb
+
+
+def _pre_outputs(R, y, pre, post, comb):
+    import torch
+    T, _, H = R.shape
+    dev = R.device
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=dev) if y is None else y
+    pre = torch.empty((T, 4), dtype=torch.float32, device=dev) if pre is None else pre
+    post = torch.empty((T, 4), dtype=torch.float32, device=dev) if post is None else post
+    comb = torch.empty((T, 4, 4), dtype=torch.float32, device=dev) if comb is None else comb
+    _need(y, torch.bfloat16, (T, H), "y")
+    _need(pre, torch.float32, (T, 4), "pre")
+    _need(post, torch.float32, None, "post")
+    if post.numel() != T * 4:
+        raise ValueError("post must hold T*4 values ([T,4] or [T,4,1])")
+    _need(comb, torch.float32, (T, 4, 4), "comb")
+    return y, pre, post, comb
+
+
+def pre_big_fuse(dot_mix, sqrsum, R, hc_scale, hc_base, k: int, *, num_splits: int = 1, y=None,
+                 pre=None, post=None, comb=None, params: Params | None = None, stream=None):
+    """Pre-map from an external projection: dot_mix [num_splits,T,24] (or [T,24] for one split)
+    and sqrsum [num_splits,T] (or [T]) fp32 partials, R [T,4,H] bf16, RMS denominator k.
+    Returns (y, pre, post, comb)."""
+    import torch
+    _need(R, torch.bfloat16, None, "R")
+    T, hc, H = R.shape
+    if hc != 4:
+        raise ValueError("R.shape[-2] (HC) must be 4")
+    _need(dot_mix, torch.float32, None, "dot_mix")
+    _need(sqrsum, torch.float32, None, "sqrsum")
+    if dot_mix.numel() != num_splits * T * 24 or sqrsum.numel() != num_splits * T:
+        raise ValueError("dot_mix must hold num_splits*T*24 values and sqrsum num_splits*T")
+    _need(hc_scale, torch.float32, (3,), "hc_scale")
+    _need(hc_base, torch.float32, (24,), "hc_base")
+    y, pre, post, comb = _pre_outputs(R, y, pre, post, comb)
+    p = params if params is not None else default_params()
+    st = lib().mhc_pre_big_fuse(_ptr(dot_mix), _ptr(sqrsum), int(num_splits), int(k), _ptr(R),
+                                _ptr(hc_scale), _ptr(hc_base), _ptr(y), _ptr(pre), _ptr(post),
+                                _ptr(comb), T, H, ctypes.byref(p), _stream(stream))
+    _check(st, "mhc_pre_big_fuse")
+    return y, pre, post, comb
+
+
+def pre_big_fuse_with_prenorm(dot_mix, R, hc_scale, hc_base, *, y=None, pre=None, post=None,
+                              comb=None, params: Params | None = None, stream=None):
+    """Pre-map from an external projection dot_mix [T,24] (or [1,T,24]); the sum of squares is
+    formed from R and the RMS denominator is 4H. Returns (y, pre, post, comb)."""
+    import torch
+    _need(R, torch.bfloat16, None, "R")
+    T, hc, H = R.shape
+    if hc != 4:
+        raise ValueError("R.shape[-2] (HC) must be 4")
+    _need(dot_mix, torch.float32, None, "dot_mix")
+    if dot_mix.numel() != T * 24:
+        raise ValueError("dot_mix must hold T*24 values")
+    _need(hc_scale, torch.float32, (3,), "hc_scale")
+    _need(hc_base, torch.float32, (24,), "hc_base")
+    y, pre, post, comb = _pre_outputs(R, y, pre, post, comb)
+    p = params if params is not None else default_params()
+    st = lib().mhc_pre_big_fuse_with_prenorm(_ptr(dot_mix), _ptr(R), _ptr(hc_scale),
+                                             _ptr(hc_base), _ptr(y), _ptr(pre), _ptr(post),
+                                             _ptr(comb), T, H, ctypes.byref(p), _stream(stream))
+    _check(st, "mhc_pre_big_fuse_with_prenorm")
     return y, pre, post, comb
 
 

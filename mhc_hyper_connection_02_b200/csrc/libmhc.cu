@@ -8,3 +8,4 @@
 #include "mhc_pre_tc.cu"
 #include "mhc_pre_fused.cu"
 #include "mhc_pre_noalloc.cu"
+#include "mhc_pre_bigfuse.cu"

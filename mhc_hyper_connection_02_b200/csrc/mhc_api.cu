@@ -243,6 +243,63 @@ int mhc_pre(const uint16_t* R, const float* hc_fn, const float* hc_scale, const 
                            workspace_bytes, T, H, p, MHC_PATH_AUTO, stream);
 }
 
+static int pre_big_fuse_common(const float* dot_mix, const float* sqrsum, int num_splits,
+                               double k, const uint16_t* R, const float* hc_scale,
+                               const float* hc_base, uint16_t* y, float* pre, float* post,
+                               float* comb, int64_t T, int64_t H, const mhc_params* p,
+                               mhc_stream_t stream) {
+  const mhc_params prm = p ? *p : mhc_default_params();
+  if (T < 0 || H <= 0) return MHC_ERR_INVALID_ARG;
+  if (!mul_ok(T, 4 * H, INT64_MAX / 4) || !mul_ok(T, 96 * num_splits, INT64_MAX)) return MHC_ERR_INVALID_ARG;
+  if (num_splits != 1 && num_splits != 2 && num_splits != 4 && num_splits != 8 && num_splits != 16)
+    return MHC_ERR_INVALID_ARG;
+  if (!(k > 0.0) || !(k < 3.0e38)) return MHC_ERR_INVALID_ARG;
+  if (prm.sinkhorn_iters < 1 || !(prm.sinkhorn_eps > 0.0f) || !isfinite(prm.sinkhorn_eps) ||
+      !(prm.rms_eps > 0.0f) || !isfinite(prm.rms_eps) || !(prm.pre_eps >= 0.0f) ||
+      !isfinite(prm.pre_eps) || !isfinite(prm.post_mult))
+    return MHC_ERR_INVALID_ARG;
+  if (T == 0) return MHC_OK;
+  if (!dot_mix || !R || !hc_scale || !hc_base || !y || !pre || !post || !comb)
+    return MHC_ERR_INVALID_ARG;
+  const size_t nR = static_cast<size_t>(T) * 4 * H * 2, ny = static_cast<size_t>(T) * H * 2;
+  const size_t n4 = static_cast<size_t>(T) * 16, n16 = static_cast<size_t>(T) * 64;
+  const size_t nd = static_cast<size_t>(T) * 96 * num_splits, ns = static_cast<size_t>(T) * 4 * num_splits;
+  const void* outs[4] = {y, pre, post, comb};
+  const size_t outn[4] = {ny, n4, n4, n16};
+  const void* ins[5] = {dot_mix, sqrsum, R, hc_scale, hc_base};
+  const size_t inn[5] = {nd, ns, nR, 12, 96};
+  for (int i = 0; i < 4; ++i) {
+    for (int j = 0; j < 5; ++j)
+      if (ins[j] && overlaps(outs[i], outn[i], ins[j], inn[j])) return MHC_ERR_ALIAS;
+    for (int j = i + 1; j < 4; ++j)
+      if (overlaps(outs[i], outn[i], outs[j], outn[j])) return MHC_ERR_ALIAS;
+  }
+  int st = bind_device(R);
+  if (st != MHC_OK) return st;
+  BigFuseArgs a{dot_mix, sqrsum, num_splits, static_cast<float>(k), R, hc_scale, hc_base, y, pre,
+                post, comb, T, H, prm.sinkhorn_iters, prm.sinkhorn_eps, prm.rms_eps, prm.pre_eps,
+                prm.post_mult};
+  return launch_pre_bigfuse(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int mhc_pre_big_fuse(const float* dot_mix, const float* sqrsum, int num_splits, int64_t k,
+                     const uint16_t* R, const float* hc_scale, const float* hc_base, uint16_t* y,
+                     float* pre, float* post, float* comb, int64_t T, int64_t H,
+                     const mhc_params* p, mhc_stream_t stream) {
+  if (!sqrsum && T > 0) return MHC_ERR_INVALID_ARG;
+  if (k < 1) return MHC_ERR_INVALID_ARG;
+  return pre_big_fuse_common(dot_mix, sqrsum, num_splits, static_cast<double>(k), R, hc_scale,
+                             hc_base, y, pre, post, comb, T, H, p, stream);
+}
+
+int mhc_pre_big_fuse_with_prenorm(const float* dot_mix, const uint16_t* R, const float* hc_scale,
+                                  const float* hc_base, uint16_t* y, float* pre, float* post,
+                                  float* comb, int64_t T, int64_t H, const mhc_params* p,
+                                  mhc_stream_t stream) {
+  return pre_big_fuse_common(dot_mix, nullptr, 1, 4.0 * static_cast<double>(H), R, hc_scale,
+                             hc_base, y, pre, post, comb, T, H, p, stream);
+}
+
 int mhc_device_status(mhc_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return MHC_ERR_CUDA;

@@ -82,6 +82,30 @@ bool pre_fused_supported(int64_t T, int64_t H);
 size_t pre_fused_workspace_bytes(int64_t T, int64_t H);
 int launch_pre_fused(const PreArgs& a, cudaStream_t s);
 
+// Pre-map from an external projection (mhc_pre_big_fuse; sqrsum == nullptr selects the variant
+// that forms the sum of squares from R, k = 4H).
+struct BigFuseArgs {
+  const float* dot_mix;  // [nsplit][T][24]
+  const float* sqrsum;   // [nsplit][T] or nullptr
+  int nsplit;
+  float k;               // RMS denominator
+  const uint16_t* R;
+  const float* hc_scale;
+  const float* hc_base;
+  uint16_t* y;
+  float* pre;
+  float* post;
+  float* comb;
+  int64_t T;
+  int64_t H;
+  int iters;
+  float sinkhorn_eps;
+  float rms_eps;
+  float pre_eps;
+  float post_mult;
+};
+int launch_pre_bigfuse(const BigFuseArgs& a, cudaStream_t s);
+
 // Tensor-core path, split pair (projection kernel + finish kernel).
 size_t pre_tc_workspace_bytes(int64_t T, int64_t H);
 bool pre_tc_supported(int64_t T, int64_t H);

@@ -115,4 +115,31 @@ def custom(T: int, H: int, seed: int, *, outliers=False, comb_std=1.0, iters=20)
                  iters=iters)
 
 
+@dataclasses.dataclass
+class Partials:
+    """Inputs of the pre-map from an external projection: split partials of the projection and of
+    the sum of squares, with the residual they belong to."""
+    T: int
+    H: int
+    R: np.ndarray        # uint16 bf16 bits [T,4,H]
+    dot_mix: np.ndarray  # float32 [S,T,24]
+    sqrsum: np.ndarray   # float32 [S,T]
+    hc_scale: np.ndarray  # float32 [3]
+    hc_base: np.ndarray   # float32 [24]
+
+
+def partials(T: int, H: int, num_splits: int, seed: int) -> Partials:
+    """The recipe of the FlashInfer article's minimal call (§5.1): R ~ N(0,1) bf16; per split
+    dot_mix ~ 0.01 N(0,1) and sqrsum ~ U(0,1) * k / num_splits (k = 4H); scale ~ 0.1 N(0,1),
+    base ~ 0.1 N(0,1). Draw order R, dot_mix, sqrsum, scale, base."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    R = torch.randn((T, HC, H), generator=g, dtype=torch.float32)
+    dot = torch.randn((num_splits, T, MIX), generator=g, dtype=torch.float32) * 0.01
+    sq = torch.rand((num_splits, T), generator=g, dtype=torch.float32) * float(4 * H / num_splits)
+    scale = torch.randn(3, generator=g, dtype=torch.float32) * 0.1
+    base = torch.randn(MIX, generator=g, dtype=torch.float32) * 0.1
+    return Partials(T=T, H=H, R=_bf16_bits(R), dot_mix=dot.numpy().copy(), sqrsum=sq.numpy().copy(),
+                    hc_scale=scale.numpy().copy(), hc_base=base.numpy().copy())
+
+
 WORKLOADS = {"small": small, "post4k": post4k, "large": large, "decode": decode, "tail": tail}

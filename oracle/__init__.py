@@ -26,3 +26,4 @@ from .c_oracle import (  # noqa: F401
     post,
     threads,
 )
+from .big_fuse import big_fuse, big_fuse_with_prenorm, sum_of_squares  # noqa: F401
