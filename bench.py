@@ -194,9 +194,10 @@ def source_digest(kernel):
 
 
 def time_extras(mhc, R, y, pre, post, comb, scale, base, params, stream, T, H, dev, reps=10):
-    """Device time of the pre-map entries that take an external projection (one split), on the
-    step's residual: algorithmic bytes R (8H) + y (2H) + dot_mix (96) + sqrsum (4, external only)
-    + pre/post/comb (96) per token."""
+    """Device time of the entries beside the step, on the step's residual. Algorithmic bytes per
+    token: pre from an external projection (one split): R (8H) + y (2H) + dot_mix (96) + sqrsum
+    (4, external only) + pre/post/comb (96); expand: hidden (2H) + streams (8H); head_mean: R (8H)
+    + y (2H); weighted head: R (8H) + y (2H) + weights (16), plus hc_fn (4H x 16) once."""
     import torch
     g = torch.Generator(device=dev).manual_seed(5)
     dot = torch.randn((1, T, 24), generator=g, device=dev) * 0.01
@@ -209,6 +210,17 @@ def time_extras(mhc, R, y, pre, post, comb, scale, base, params, stream, T, H, d
             dot[0], R, scale, base, y=y, pre=pre, post=post, comb=comb, params=params,
             stream=stream), T * (10 * H + 192)),
     }
+    hidden = y  # a [T,H] bf16 row buffer of the step
+    streams = torch.empty_like(R)
+    fn4 = torch.randn((4 * H, 4), generator=g, device=dev) * 0.02
+    s1 = torch.ones(1, device=dev)
+    b4 = torch.zeros(4, device=dev)
+    wts = torch.empty((T, 4), device=dev)
+    hws = torch.empty(mhc.head_workspace_bytes(T, H), dtype=torch.uint8, device=dev)
+    calls["expand"] = (lambda: mhc.expand(hidden, streams=streams, stream=stream), T * 10 * H)
+    calls["head_mean"] = (lambda: mhc.head_mean(R, y=hidden, stream=stream), T * 10 * H)
+    calls["head"] = (lambda: mhc.head(R, fn4, s1, b4, y=hidden, weights=wts, workspace=hws,
+                                      stream=stream), T * (10 * H + 16) + 4 * H * 16)
     out = {}
     for name, (fn, nbytes) in calls.items():
         for _ in range(3):

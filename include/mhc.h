@@ -250,6 +250,36 @@ MHC_API int mhc_pre_big_fuse_with_prenorm(const float* dot_mix, const uint16_t* 
                                           int64_t T, int64_t H, const mhc_params* p,
                                           mhc_stream_t stream);
 
+/*
+ * Model-boundary operations: the first layer's expand and the last layer's head. glm5next_mhc.rs
+ * glm_hc_expand and hc_head_mean; hyper_connection_dispatch.rs hc_head_site (weighted head).
+ * Streams are the library's bf16 [T][4][H] residual (the GLM page keeps them in fp32).
+ *
+ * mhc_expand     streams[t][i][:] = hidden[t][:] for each of the 4 streams (bitwise copies).
+ *                  hidden [T][H] bf16, streams [T][4][H] bf16 out.
+ * mhc_head_mean  y[t][:] = bf16_rn(mean_i streams[t][i][:]): the unweighted mean, fp32 sums.
+ *                  R [T][4][H] bf16, y [T][H] bf16 out.
+ * mhc_head       the weighted collapse: rstd = 1/sqrt(sum(R_flat^2)/(4H) + norm_eps);
+ *                  w_i = sigmoid((R_flat . hc_fn[:, i]) * rstd * hc_scale[0] + hc_base[i]) + hc_eps;
+ *                  y = bf16_rn(sum_i w_i R_i). The page shows this entry's arguments (hc_fn,
+ *                  hc_scale, hc_base, norm eps, hc_eps) but not its kernel; this is the reading in
+ *                  which the head is the pre-map's first gate group with its own weights.
+ *                  hc_fn [4H][4], hc_scale [1], hc_base [4] fp32; y [T][H] bf16 out; weights
+ *                  [T][4] fp32 out, or NULL; workspace of mhc_head_workspace_bytes(T, H) bytes,
+ *                  256-byte aligned (contents on entry do not matter).
+ * Errors: MHC_ERR_INVALID_ARG (null array, T < 0, H <= 0, norm_eps <= 0, hc_eps < 0, a misaligned
+ * workspace); MHC_ERR_WORKSPACE_TOO_SMALL; MHC_ERR_ALIAS when an output overlaps an input.
+ */
+MHC_API int mhc_expand(const uint16_t* hidden, uint16_t* streams, int64_t T, int64_t H,
+                       mhc_stream_t stream);
+MHC_API int mhc_head_mean(const uint16_t* R, uint16_t* y, int64_t T, int64_t H,
+                          mhc_stream_t stream);
+MHC_API size_t mhc_head_workspace_bytes(int64_t T, int64_t H);
+MHC_API int mhc_head(const uint16_t* R, const float* hc_fn, const float* hc_scale,
+                     const float* hc_base, uint16_t* y, float* weights, void* workspace,
+                     size_t workspace_bytes, int64_t T, int64_t H, float norm_eps, float hc_eps,
+                     mhc_stream_t stream);
+
 /* Number of kernel launches this process has enqueued through the library so far (all devices,
  * all threads). A diagnostic counter for benchmarks: take the difference around a region. */
 MHC_API uint64_t mhc_launch_count(void);

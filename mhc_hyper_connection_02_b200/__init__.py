@@ -41,7 +41,8 @@ EXPORTED_SYMBOLS = (
     "mhc_default_params", "mhc_pre", "mhc_pre_workspace_bytes", "mhc_post", "mhc_sinkhorn",
     "mhc_pre_with_path", "mhc_post_with_path", "mhc_device_status", "mhc_status_string",
     "mhc_version", "mhc_launch_count", "mhc_pre_noalloc", "mhc_pre_big_fuse",
-    "mhc_pre_big_fuse_with_prenorm",
+    "mhc_pre_big_fuse_with_prenorm", "mhc_expand", "mhc_head_mean", "mhc_head",
+    "mhc_head_workspace_bytes",
 )
 
 
@@ -103,6 +104,15 @@ def lib() -> ctypes.CDLL:
     L.mhc_pre_big_fuse_with_prenorm.restype = ctypes.c_int
     L.mhc_pre_big_fuse_with_prenorm.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64,
                                                 ctypes.POINTER(Params), _P]
+    L.mhc_expand.restype = ctypes.c_int
+    L.mhc_expand.argtypes = [_P, _P, _I64, _I64, _P]
+    L.mhc_head_mean.restype = ctypes.c_int
+    L.mhc_head_mean.argtypes = [_P, _P, _I64, _I64, _P]
+    L.mhc_head_workspace_bytes.restype = ctypes.c_size_t
+    L.mhc_head_workspace_bytes.argtypes = [_I64, _I64]
+    L.mhc_head.restype = ctypes.c_int
+    L.mhc_head.argtypes = [_P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I64, _I64,
+                           ctypes.c_float, ctypes.c_float, _P]
     L.mhc_launch_count.restype = ctypes.c_uint64
     L.mhc_launch_count.argtypes = []
     _lib = L
@@ -259,6 +269,63 @@ def pre_big_fuse_with_prenorm(dot_mix, R, hc_scale, hc_base, *, y=None, pre=None
                                              _ptr(comb), T, H, ctypes.byref(p), _stream(stream))
     _check(st, "mhc_pre_big_fuse_with_prenorm")
     return y, pre, post, comb
+
+
+def expand(hidden, *, streams=None, stream=None):
+    """First-layer expand: hidden [T,H] bf16 -> streams [T,4,H] bf16 (each stream a copy)."""
+    import torch
+    _need(hidden, torch.bfloat16, None, "hidden")
+    T, H = hidden.shape
+    streams = torch.empty((T, 4, H), dtype=torch.bfloat16, device=hidden.device) \
+        if streams is None else streams
+    _need(streams, torch.bfloat16, (T, 4, H), "streams")
+    _check(lib().mhc_expand(_ptr(hidden), _ptr(streams), T, H, _stream(stream)), "mhc_expand")
+    return streams
+
+
+def head_mean(R, *, y=None, stream=None):
+    """Last-layer unweighted head: y [T,H] = bf16(mean of the 4 streams of R [T,4,H])."""
+    import torch
+    _need(R, torch.bfloat16, None, "R")
+    T, hc, H = R.shape
+    if hc != 4:
+        raise ValueError("R.shape[-2] (HC) must be 4")
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=R.device) if y is None else y
+    _need(y, torch.bfloat16, (T, H), "y")
+    _check(lib().mhc_head_mean(_ptr(R), _ptr(y), T, H, _stream(stream)), "mhc_head_mean")
+    return y
+
+
+def head_workspace_bytes(T: int, H: int) -> int:
+    return int(lib().mhc_head_workspace_bytes(int(T), int(H)))
+
+
+def head(R, hc_fn, hc_scale, hc_base, *, norm_eps: float = 1e-6, hc_eps: float = 1e-6, y=None,
+         weights=None, workspace=None, stream=None):
+    """Last-layer weighted head: R [T,4,H] bf16, hc_fn [4H,4], hc_scale [1], hc_base [4] fp32.
+    Returns (y [T,H] bf16, weights [T,4] fp32)."""
+    import torch
+    _need(R, torch.bfloat16, None, "R")
+    T, hc, H = R.shape
+    if hc != 4:
+        raise ValueError("R.shape[-2] (HC) must be 4")
+    _need(hc_fn, torch.float32, (4 * H, 4), "hc_fn")
+    _need(hc_scale, torch.float32, (1,), "hc_scale")
+    _need(hc_base, torch.float32, (4,), "hc_base")
+    dev = R.device
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=dev) if y is None else y
+    weights = torch.empty((T, 4), dtype=torch.float32, device=dev) if weights is None else weights
+    _need(y, torch.bfloat16, (T, H), "y")
+    _need(weights, torch.float32, (T, 4), "weights")
+    nws = head_workspace_bytes(T, H)
+    if workspace is None and nws > 0:
+        workspace = torch.empty(nws, dtype=torch.uint8, device=dev)
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().mhc_head(_ptr(R), _ptr(hc_fn), _ptr(hc_scale), _ptr(hc_base), _ptr(y),
+                        _ptr(weights), _ptr(workspace), wsb, T, H, float(norm_eps), float(hc_eps),
+                        _stream(stream))
+    _check(st, "mhc_head")
+    return y, weights
 
 
 def post(x, R, post, comb, *, out=None, path: int = PATH_AUTO, stream=None):

@@ -9,3 +9,4 @@
 #include "mhc_pre_fused.cu"
 #include "mhc_pre_noalloc.cu"
 #include "mhc_pre_bigfuse.cu"
+#include "mhc_boundary.cu"

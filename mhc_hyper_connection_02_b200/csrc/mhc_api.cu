@@ -300,6 +300,94 @@ int mhc_pre_big_fuse_with_prenorm(const float* dot_mix, const uint16_t* R, const
                              hc_base, y, pre, post, comb, T, H, p, stream);
 }
 
+int mhc_expand(const uint16_t* hidden, uint16_t* streams, int64_t T, int64_t H,
+               mhc_stream_t stream) {
+  if (T < 0 || H <= 0 || !mul_ok(T, 4 * H, INT64_MAX / 4)) return MHC_ERR_INVALID_ARG;
+  if (T == 0) return MHC_OK;
+  if (!hidden || !streams) return MHC_ERR_INVALID_ARG;
+  if (overlaps(hidden, static_cast<size_t>(T) * H * 2, streams, static_cast<size_t>(T) * 8 * H))
+    return MHC_ERR_ALIAS;
+  int st = bind_device(hidden);
+  if (st != MHC_OK) return st;
+  return launch_expand(hidden, streams, T, H, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int mhc_head_mean(const uint16_t* R, uint16_t* y, int64_t T, int64_t H, mhc_stream_t stream) {
+  if (T < 0 || H <= 0 || !mul_ok(T, 4 * H, INT64_MAX / 4)) return MHC_ERR_INVALID_ARG;
+  if (T == 0) return MHC_OK;
+  if (!R || !y) return MHC_ERR_INVALID_ARG;
+  if (overlaps(R, static_cast<size_t>(T) * 8 * H, y, static_cast<size_t>(T) * H * 2))
+    return MHC_ERR_ALIAS;
+  int st = bind_device(R);
+  if (st != MHC_OK) return st;
+  return launch_head_mean(R, y, T, H, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// Workspace of mhc_head: [fn24: 4H x 24 fp32][scale3 + base24][pre, post, comb scratch: T x 24
+// fp32][mhc_pre workspace], each part 256-byte aligned.
+struct HeadLayout {
+  size_t fn, sb, coef, pre_ws, pre_ws_bytes, total;
+};
+static HeadLayout head_layout(int64_t T, int64_t H) {
+  HeadLayout l;
+  auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+  l.fn = 0;
+  l.sb = up(static_cast<size_t>(4 * H) * 24 * 4);
+  l.coef = l.sb + 256;
+  l.pre_ws = l.coef + up(static_cast<size_t>(T) * 24 * 4);
+  l.pre_ws_bytes = mhc_pre_workspace_bytes(T, H);
+  l.total = l.pre_ws + l.pre_ws_bytes;
+  return l;
+}
+
+size_t mhc_head_workspace_bytes(int64_t T, int64_t H) {
+  if (T <= 0 || H <= 0 || !mul_ok(T, 4 * H, INT64_MAX / 4)) return 0;
+  return head_layout(T, H).total;
+}
+
+int mhc_head(const uint16_t* R, const float* hc_fn, const float* hc_scale, const float* hc_base,
+             uint16_t* y, float* weights, void* workspace, size_t workspace_bytes, int64_t T,
+             int64_t H, float norm_eps, float hc_eps, mhc_stream_t stream) {
+  if (T < 0 || H <= 0 || !mul_ok(T, 4 * H, INT64_MAX / 4)) return MHC_ERR_INVALID_ARG;
+  if (!(norm_eps > 0.0f) || !isfinite(norm_eps) || !(hc_eps >= 0.0f) || !isfinite(hc_eps))
+    return MHC_ERR_INVALID_ARG;
+  if (T == 0) return MHC_OK;
+  if (!R || !hc_fn || !hc_scale || !hc_base || !y) return MHC_ERR_INVALID_ARG;
+  const HeadLayout l = head_layout(T, H);
+  if (workspace_bytes < l.total || !workspace) return MHC_ERR_WORKSPACE_TOO_SMALL;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MHC_ERR_INVALID_ARG;
+  const size_t nR = static_cast<size_t>(T) * 8 * H, ny = static_cast<size_t>(T) * H * 2;
+  const size_t nfn = static_cast<size_t>(4 * H) * 16;
+  if (overlaps(y, ny, R, nR) || overlaps(y, ny, hc_fn, nfn) || overlaps(y, ny, workspace, l.total))
+    return MHC_ERR_ALIAS;
+  if (overlaps(workspace, l.total, R, nR) || overlaps(workspace, l.total, hc_fn, nfn))
+    return MHC_ERR_ALIAS;
+  if (weights && (overlaps(weights, static_cast<size_t>(T) * 16, y, ny) ||
+                  overlaps(weights, static_cast<size_t>(T) * 16, R, nR) ||
+                  overlaps(weights, static_cast<size_t>(T) * 16, workspace, l.total)))
+    return MHC_ERR_ALIAS;
+  int st = bind_device(R);
+  if (st != MHC_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* fn24 = reinterpret_cast<float*>(ws + l.fn);
+  float* sb = reinterpret_cast<float*>(ws + l.sb);
+  float* coef = reinterpret_cast<float*>(ws + l.coef);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int r = launch_head_pad(hc_fn, hc_scale, hc_base, fn24, sb, H, s);
+  if (r != 0) return r;
+  // The pre-map with that padded projection: its pre gates are the head weights; post and comb
+  // (one Sinkhorn round) land in scratch.
+  mhc_params p;
+  p.sinkhorn_iters = 1;
+  p.sinkhorn_eps = 1e-6f;
+  p.rms_eps = norm_eps;
+  p.pre_eps = hc_eps;
+  p.post_mult = 1.0f;
+  float* pre_out = weights ? weights : coef;
+  return mhc_pre_with_path(R, fn24, sb, sb + 3, y, pre_out, coef + 4 * T, coef + 8 * T,
+                           ws + l.pre_ws, l.pre_ws_bytes, T, H, &p, MHC_PATH_AUTO, stream);
+}
+
 int mhc_device_status(mhc_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return MHC_ERR_CUDA;

@@ -106,6 +106,12 @@ struct BigFuseArgs {
 };
 int launch_pre_bigfuse(const BigFuseArgs& a, cudaStream_t s);
 
+// Model-boundary operations (mhc_boundary.cu).
+int launch_expand(const uint16_t* hidden, uint16_t* streams, int64_t T, int64_t H, cudaStream_t s);
+int launch_head_mean(const uint16_t* R, uint16_t* y, int64_t T, int64_t H, cudaStream_t s);
+int launch_head_pad(const float* fn4, const float* scale1, const float* base4, float* fn24,
+                    float* sb, int64_t H, cudaStream_t s);
+
 // Tensor-core path, split pair (projection kernel + finish kernel).
 size_t pre_tc_workspace_bytes(int64_t T, int64_t H);
 bool pre_tc_supported(int64_t T, int64_t H);
