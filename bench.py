@@ -193,11 +193,14 @@ def source_digest(kernel):
     return h.hexdigest()[:16]
 
 
-def time_extras(mhc, R, y, pre, post, comb, scale, base, params, stream, T, H, dev, reps=10):
+def time_extras(mhc, R, x, out, y, pre, post, comb, hc_fn, scale, base, params, stream, T, H, dev,
+                reps=10):
     """Device time of the entries beside the step, on the step's residual. Algorithmic bytes per
     token: pre from an external projection (one split): R (8H) + y (2H) + dot_mix (96) + sqrsum
     (4, external only) + pre/post/comb (96); expand: hidden (2H) + streams (8H); head_mean: R (8H)
-    + y (2H); weighted head: R (8H) + y (2H) + weights (16), plus hc_fn (4H x 16) once."""
+    + y (2H); weighted head: R (8H) + y (2H) + weights (16), plus hc_fn (4H x 16) once; post with
+    the next projection: the post-map's 18H + 80 plus S x 100 of partials; layer chain (that, then
+    the next pre-map from the partials): the post-map's bytes plus the pre-map's 10H + 96."""
     import torch
     g = torch.Generator(device=dev).manual_seed(5)
     dot = torch.randn((1, T, 24), generator=g, device=dev) * 0.01
@@ -221,6 +224,26 @@ def time_extras(mhc, R, y, pre, post, comb, scale, base, params, stream, T, H, d
     calls["head_mean"] = (lambda: mhc.head_mean(R, y=hidden, stream=stream), T * 10 * H)
     calls["head"] = (lambda: mhc.head(R, fn4, s1, b4, y=hidden, weights=wts, workspace=hws,
                                       stream=stream), T * (10 * H + 16) + 4 * H * 16)
+    S = mhc.post_project_splits(T, H)
+    if S > 0:
+        pdm = torch.empty((S, T, 24), device=dev)
+        psq = torch.empty((S, T), device=dev)
+        wsp = torch.empty(max(1, int(mhc.lib().mhc_post_project_workspace_bytes(T, H))),
+                          dtype=torch.uint8, device=dev)
+        pre2, post2 = torch.empty_like(pre), torch.empty_like(post)
+        comb2 = torch.empty_like(comb)
+
+        def post_project():
+            mhc.post_project(x, R, post, comb, hc_fn, out=out, dot_mix=pdm, sqrsum=psq,
+                             workspace=wsp, stream=stream)
+
+        def layer_chain():  # post of this site + the next site's pre-map on its output
+            post_project()
+            mhc.pre_big_fuse(pdm, psq, out, scale, base, 4 * H, num_splits=S, y=y, pre=pre2,
+                             post=post2, comb=comb2, params=params, stream=stream)
+
+        calls["post_project"] = (post_project, T * (18 * H + 80 + S * 100) + 4 * H * 96)
+        calls["layer_chain"] = (layer_chain, T * (18 * H + 80) + T * (10 * H + 96) + 4 * H * 96)
     out = {}
     for name, (fn, nbytes) in calls.items():
         for _ in range(3):
@@ -232,7 +255,8 @@ def time_extras(mhc, R, y, pre, post, comb, scale, base, params, stream, T, H, d
         b.record(stream)
         torch.cuda.synchronize()
         us = a.elapsed_time(b) / reps * 1e3
-        out[name] = {"us": us, "algo_bytes": nbytes, "GBps": nbytes / us / 1e3}
+        out[name] = {"us": us, "algo_bytes": nbytes, "GBps": nbytes / us / 1e3,
+                     "tokens_per_s": T / (us / 1e6)}
     assert mhc.device_status() == 0
     return out
 
@@ -392,7 +416,8 @@ def main():
 
     extras = None
     if not args.no_extras and args.only == "both":
-        extras = time_extras(mhc, R, y, pre, post, comb, scale, base, params, stream, T, H, dev)
+        extras = time_extras(mhc, R, x, out, y, pre, post, comb, hc_fn, scale, base, params,
+                             stream, T, H, dev)
 
     if rank == 0:
         hbm, tflops, peak_src = load_peaks()

@@ -251,6 +251,35 @@ MHC_API int mhc_pre_big_fuse_with_prenorm(const float* dot_mix, const uint16_t* 
                                           mhc_stream_t stream);
 
 /*
+ * mhc_post_project -- the post-map fused with the next site's projection partials. No entry of
+ * this shape is on the pages: pre and post alternate along the layer stack ("FlashInfer mHC
+ * module deep dive" §1; glm5next_mhc.rs: the streams glm_hc_post writes are the next residual),
+ * and the next pre-map's projection and sum of squares are sums over the new residual row, so
+ * they are formed here as split partials while that row is produced; mhc_pre_big_fuse (num_splits
+ * = mhc_post_project_splits(T, H), k = 4H) then finishes the next pre-map reading `out` once.
+ *
+ *   x, R, post, comb, out   as mhc_post; out is bitwise equal to mhc_post's result; out may be R
+ *   hc_fn_next  [4H][24] fp32   the next site's projection
+ *   dot_mix     [S][T][24] fp32 out: S = mhc_post_project_splits(T, H) (a power of two <= 16)
+ *                               partials of sum_k out_flat[t][k] * hc_fn_next[k][j], k = n*H + h,
+ *                               over the bf16 values of out; every split is written (zeros where
+ *                               a token's row has fewer pieces)
+ *   sqrsum      [S][T] fp32     out: partials of sum_k out_flat[t][k]^2
+ *   workspace   mhc_post_project_workspace_bytes(T, H) bytes, 256-byte aligned (the split
+ *               hc_fn_next operand)
+ *
+ * Requires H % 8 == 0 and 16-byte aligned x, R, out, post, comb and dot_mix (MHC_ERR_UNSUPPORTED
+ * otherwise; use mhc_post then mhc_pre). Errors: MHC_ERR_INVALID_ARG, MHC_ERR_WORKSPACE_TOO_SMALL,
+ * MHC_ERR_ALIAS (an output overlapping an input, other than out == R).
+ */
+MHC_API int mhc_post_project_splits(int64_t T, int64_t H);
+MHC_API size_t mhc_post_project_workspace_bytes(int64_t T, int64_t H);
+MHC_API int mhc_post_project(const uint16_t* x, const uint16_t* R, const float* post,
+                             const float* comb, uint16_t* out, const float* hc_fn_next,
+                             float* dot_mix, float* sqrsum, void* workspace,
+                             size_t workspace_bytes, int64_t T, int64_t H, mhc_stream_t stream);
+
+/*
  * Model-boundary operations: the first layer's expand and the last layer's head. glm5next_mhc.rs
  * glm_hc_expand and hc_head_mean; hyper_connection_dispatch.rs hc_head_site (weighted head).
  * Streams are the library's bf16 [T][4][H] residual (the GLM page keeps them in fp32).

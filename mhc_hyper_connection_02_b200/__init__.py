@@ -42,7 +42,8 @@ EXPORTED_SYMBOLS = (
     "mhc_pre_with_path", "mhc_post_with_path", "mhc_device_status", "mhc_status_string",
     "mhc_version", "mhc_launch_count", "mhc_pre_noalloc", "mhc_pre_big_fuse",
     "mhc_pre_big_fuse_with_prenorm", "mhc_expand", "mhc_head_mean", "mhc_head",
-    "mhc_head_workspace_bytes",
+    "mhc_head_workspace_bytes", "mhc_post_project", "mhc_post_project_splits",
+    "mhc_post_project_workspace_bytes",
 )
 
 
@@ -113,6 +114,13 @@ def lib() -> ctypes.CDLL:
     L.mhc_head.restype = ctypes.c_int
     L.mhc_head.argtypes = [_P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I64, _I64,
                            ctypes.c_float, ctypes.c_float, _P]
+    L.mhc_post_project_splits.restype = ctypes.c_int
+    L.mhc_post_project_splits.argtypes = [_I64, _I64]
+    L.mhc_post_project_workspace_bytes.restype = ctypes.c_size_t
+    L.mhc_post_project_workspace_bytes.argtypes = [_I64, _I64]
+    L.mhc_post_project.restype = ctypes.c_int
+    L.mhc_post_project.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I64,
+                                   _I64, _P]
     L.mhc_launch_count.restype = ctypes.c_uint64
     L.mhc_launch_count.argtypes = []
     _lib = L
@@ -269,6 +277,48 @@ def pre_big_fuse_with_prenorm(dot_mix, R, hc_scale, hc_base, *, y=None, pre=None
                                              _ptr(comb), T, H, ctypes.byref(p), _stream(stream))
     _check(st, "mhc_pre_big_fuse_with_prenorm")
     return y, pre, post, comb
+
+
+def post_project_splits(T: int, H: int) -> int:
+    """Splits S of the partials mhc_post_project writes for (T, H); 0 when unsupported."""
+    return int(lib().mhc_post_project_splits(int(T), int(H)))
+
+
+def post_project(x, R, post, comb, hc_fn_next, *, out=None, dot_mix=None, sqrsum=None,
+                 workspace=None, stream=None):
+    """Post-map fused with the next site's projection partials. Returns (out [T,4,H] bf16,
+    dot_mix [S,T,24], sqrsum [S,T]); finish the next pre-map with
+    pre_big_fuse(dot_mix, sqrsum, out, ..., k=4H, num_splits=S)."""
+    import torch
+    _need(R, torch.bfloat16, None, "R")
+    T, hc, H = R.shape
+    if hc != 4:
+        raise ValueError("R.shape[-2] (HC) must be 4")
+    _need(x, torch.bfloat16, (T, H), "x")
+    _need(post, torch.float32, None, "post")
+    if post.numel() != T * 4:
+        raise ValueError("post must hold T*4 values ([T,4] or [T,4,1])")
+    _need(comb, torch.float32, (T, 4, 4), "comb")
+    _need(hc_fn_next, torch.float32, (4 * H, 24), "hc_fn_next")
+    S = post_project_splits(T, H) if T > 0 else 1
+    if T > 0 and S == 0:
+        raise MhcError(MHC_ERR_UNSUPPORTED, "mhc_post_project")
+    dev = R.device
+    out = torch.empty_like(R) if out is None else out
+    dot_mix = torch.empty((S, T, 24), dtype=torch.float32, device=dev) if dot_mix is None else dot_mix
+    sqrsum = torch.empty((S, T), dtype=torch.float32, device=dev) if sqrsum is None else sqrsum
+    _need(out, torch.bfloat16, (T, 4, H), "out")
+    _need(dot_mix, torch.float32, (S, T, 24), "dot_mix")
+    _need(sqrsum, torch.float32, (S, T), "sqrsum")
+    nws = int(lib().mhc_post_project_workspace_bytes(T, H))
+    if workspace is None and nws > 0:
+        workspace = torch.empty(nws, dtype=torch.uint8, device=dev)
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().mhc_post_project(_ptr(x), _ptr(R), _ptr(post), _ptr(comb), _ptr(out),
+                                _ptr(hc_fn_next), _ptr(dot_mix), _ptr(sqrsum), _ptr(workspace),
+                                wsb, T, H, _stream(stream))
+    _check(st, "mhc_post_project")
+    return out, dot_mix, sqrsum
 
 
 def expand(hidden, *, streams=None, stream=None):

@@ -10,3 +10,4 @@
 #include "mhc_pre_noalloc.cu"
 #include "mhc_pre_bigfuse.cu"
 #include "mhc_boundary.cu"
+#include "mhc_post_project.cu"

@@ -300,6 +300,55 @@ int mhc_pre_big_fuse_with_prenorm(const float* dot_mix, const uint16_t* R, const
                              hc_base, y, pre, post, comb, T, H, p, stream);
 }
 
+int mhc_post_project_splits(int64_t T, int64_t H) {
+  if (T <= 0 || H <= 0 || !mul_ok(T, 4 * H, INT64_MAX / 4)) return 0;
+  return post_project_splits(T, H);
+}
+
+size_t mhc_post_project_workspace_bytes(int64_t T, int64_t H) {
+  if (T <= 0 || H <= 0 || !mul_ok(T, 4 * H, INT64_MAX / 4)) return 0;
+  const size_t b = post_project_workspace_bytes(T, H);
+  return (b + 255) / 256 * 256;
+}
+
+int mhc_post_project(const uint16_t* x, const uint16_t* R, const float* post, const float* comb,
+                     uint16_t* out, const float* hc_fn_next, float* dot_mix, float* sqrsum,
+                     void* workspace, size_t workspace_bytes, int64_t T, int64_t H,
+                     mhc_stream_t stream) {
+  if (T < 0 || H <= 0 || !mul_ok(T, 4 * H, INT64_MAX / 4)) return MHC_ERR_INVALID_ARG;
+  if (T == 0) return MHC_OK;
+  if (!x || !R || !post || !comb || !out || !hc_fn_next || !dot_mix || !sqrsum)
+    return MHC_ERR_INVALID_ARG;
+  if (!post_project_supported(T, H) || !aligned16(x) || !aligned16(R) || !aligned16(out) ||
+      !aligned16(post) || !aligned16(comb) || !aligned16(dot_mix))
+    return MHC_ERR_UNSUPPORTED;
+  const size_t need = mhc_post_project_workspace_bytes(T, H);
+  if (workspace_bytes < need || !workspace) return MHC_ERR_WORKSPACE_TOO_SMALL;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MHC_ERR_INVALID_ARG;
+  const int S = post_project_splits(T, H);
+  const size_t nR = static_cast<size_t>(T) * 8 * H, nx = static_cast<size_t>(T) * H * 2;
+  const size_t nd = static_cast<size_t>(S) * T * 96, ns = static_cast<size_t>(S) * T * 4;
+  const size_t nfn = static_cast<size_t>(4 * H) * 96;
+  if (static_cast<const void*>(out) != static_cast<const void*>(R) && overlaps(out, nR, R, nR))
+    return MHC_ERR_ALIAS;
+  const void* outs[4] = {out, dot_mix, sqrsum, workspace};
+  const size_t outn[4] = {nR, nd, ns, need};
+  const void* ins[5] = {x, post, comb, hc_fn_next, R};
+  const size_t inn[5] = {nx, static_cast<size_t>(T) * 16, static_cast<size_t>(T) * 64, nfn, nR};
+  for (int i = 0; i < 4; ++i) {
+    for (int j = 0; j < 5; ++j) {
+      if (i == 0 && j == 4) continue;  // out == R is allowed (checked above)
+      if (overlaps(outs[i], outn[i], ins[j], inn[j])) return MHC_ERR_ALIAS;
+    }
+    for (int j = i + 1; j < 4; ++j)
+      if (overlaps(outs[i], outn[i], outs[j], outn[j])) return MHC_ERR_ALIAS;
+  }
+  int st = bind_device(R);
+  if (st != MHC_OK) return st;
+  PostProjectArgs a{x, R, post, comb, out, hc_fn_next, dot_mix, sqrsum, workspace, T, H};
+  return launch_post_project(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int mhc_expand(const uint16_t* hidden, uint16_t* streams, int64_t T, int64_t H,
                mhc_stream_t stream) {
   if (T < 0 || H <= 0 || !mul_ok(T, 4 * H, INT64_MAX / 4)) return MHC_ERR_INVALID_ARG;

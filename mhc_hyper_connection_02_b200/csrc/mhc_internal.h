@@ -106,6 +106,25 @@ struct BigFuseArgs {
 };
 int launch_pre_bigfuse(const BigFuseArgs& a, cudaStream_t s);
 
+// Post-map fused with the next site's projection partials (mhc_post_project.cu).
+struct PostProjectArgs {
+  const uint16_t* x;
+  const uint16_t* R;
+  const float* post;
+  const float* comb;
+  uint16_t* out;
+  const float* hc_fn;  // the next site's [4H][24]
+  float* dot_mix;      // [S][T][24]
+  float* sqrsum;       // [S][T]
+  void* workspace;
+  int64_t T;
+  int64_t H;
+};
+bool post_project_supported(int64_t T, int64_t H);
+int post_project_splits(int64_t T, int64_t H);
+size_t post_project_workspace_bytes(int64_t T, int64_t H);
+int launch_post_project(const PostProjectArgs& a, cudaStream_t s);
+
 // Model-boundary operations (mhc_boundary.cu).
 int launch_expand(const uint16_t* hidden, uint16_t* streams, int64_t T, int64_t H, cudaStream_t s);
 int launch_head_mean(const uint16_t* R, uint16_t* y, int64_t T, int64_t H, cudaStream_t s);
