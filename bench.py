@@ -244,7 +244,7 @@ def time_extras(mhc, R, x, out, y, pre, post, comb, hc_fn, scale, base, params, 
 
         calls["post_project"] = (post_project, T * (18 * H + 80 + S * 100) + 4 * H * 96)
         calls["layer_chain"] = (layer_chain, T * (18 * H + 80) + T * (10 * H + 96) + 4 * H * 96)
-    out = {}
+    res = {}
     for name, (fn, nbytes) in calls.items():
         for _ in range(3):
             fn()
@@ -255,10 +255,10 @@ def time_extras(mhc, R, x, out, y, pre, post, comb, hc_fn, scale, base, params, 
         b.record(stream)
         torch.cuda.synchronize()
         us = a.elapsed_time(b) / reps * 1e3
-        out[name] = {"us": us, "algo_bytes": nbytes, "GBps": nbytes / us / 1e3,
+        res[name] = {"us": us, "algo_bytes": nbytes, "GBps": nbytes / us / 1e3,
                      "tokens_per_s": T / (us / 1e6)}
     assert mhc.device_status() == 0
-    return out
+    return res
 
 
 def main():

@@ -20,11 +20,12 @@
 //               of a column block into a 2-stage ring.
 //   warp 1      tcgen05.mma M=128 N=80 K=16: for each column block, 4 streams x 4 K-steps into
 //               the piece's TMEM accumulator (two, alternating between pieces).
-//   warps 2-9   the post-map: two threads per token, each 32 columns of the block; 16-byte loads
-//               of x and the four R streams, 16-byte stores of the four out streams to global and
-//               into the MMA A operand tiles in shared memory (128-byte swizzled rows); sum of
-//               squares of the rounded outputs. After a piece: the accumulator (tcgen05.ld) and
-//               the sums of squares become the split partials.
+//   warps 2-9   the post-map: 8 lanes per token row (one 16-byte chunk each), four tokens per
+//               thread. The four R streams arrive one block ahead by 16-byte asynchronous copies
+//               straight into the MMA A operand tiles (128-byte swizzled rows), x into registers;
+//               out is computed in place there (it becomes the A operand) and stored to global
+//               with 16-byte stores; sum of squares of the rounded outputs. After a piece they read the
+//               accumulator (tcgen05.ld) and, with the sums of squares, write the split partials.
 // Requires H % 8 == 0 and 16-byte aligned x, R, out, post, comb, dot_mix. out may be R.
 #include <cuda.h>
 
@@ -41,9 +42,13 @@ constexpr int kPpAStage = 4 * kPpABytes;           // 65536
 constexpr int kPpBStage = 4 * kPpBBytes;           // 40960
 constexpr int kPpStages = 2;
 constexpr int kPpXWarps = 8;                       // post-map warps (2..9)
+constexpr int kPpEpiWarps = 8;                     // of them, those that read TMEM (2..9)
+constexpr int kPpTokStride = 4 * kPpXWarps;        // a thread's tokens: tg + 32 i
+constexpr int kPpTokPerThread = kPpM / kPpTokStride;  // 4
 constexpr int kPpThreads = 64 + 32 * kPpXWarps;    // 320
 constexpr int kPpTmemCols = 256;                   // two accumulators of 128 columns
-constexpr int kPpSmem = 1024 + kPpStages * (kPpAStage + kPpBStage) + kPpM * 2 * 4 + 256;
+constexpr int kPpCoef = kPpM * 20 * 4;           // a tile's post / comb, 10 KB
+constexpr int kPpSmem = 1024 + kPpStages * (kPpAStage + kPpBStage) + kPpCoef + kPpM * 4 + 256;
 constexpr int64_t kPpSms = 148;
 constexpr int kPpMaxSplits = 16;
 
@@ -91,6 +96,50 @@ __device__ __forceinline__ float pp_raw(const uint32_t (&d)[5][16], int j) {
   return (l3 + m3) + h3;
 }
 
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_prior() {  // all groups but the newest
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// Issues one block's residual copies for this thread's chunk ch (8 columns) of tokens
+// tg + 32 i, i < 4, in all four streams, into stage s of the A tiles at their swizzled positions
+// (zeros where the token or the column is out of range), as one commit group; and loads the
+// block's x chunks into xn. The 8 lanes of a token cover one 128-byte row segment.
+__device__ __forceinline__ void pp_issue_block(int64_t g, int64_t hb, int s, uint8_t* Abuf,
+                                               const uint16_t* R, const uint16_t* x, int64_t T,
+                                               int64_t H, int C, int tg, int ch,
+                                               uint4 (&xn)[kPpTokPerThread]) {
+  const int64_t t0 = (g / C) * kPpM;
+  const int64_t h = hb * kPpHB + ch * 8;
+#pragma unroll
+  for (int i = 0; i < kPpTokPerThread; ++i) {
+    const int r = tg + kPpTokStride * i;
+    const int64_t t = t0 + r;
+    uint8_t* dst = Abuf + s * kPpAStage + r * 128 + ((ch ^ (r & 7)) << 4);
+    if (t < T && h < H) {
+#pragma unroll
+      for (int m = 0; m < 4; ++m) cp_async16(dst + m * kPpABytes, R + (t * 4 + m) * H + h);
+      xn[i] = __ldg(reinterpret_cast<const uint4*>(x + t * H + h));
+    } else {
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        *reinterpret_cast<uint4*>(dst + m * kPpABytes) = make_uint4(0u, 0u, 0u, 0u);
+      xn[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  cp_async_commit();
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -105,8 +154,9 @@ __global__ void __launch_bounds__(kPpThreads, 1) post_project_kernel(
   uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
   uint8_t* Abuf = smem;                                   // [2][4][128 x 128 B]
   uint8_t* Bbuf = smem + kPpStages * kPpAStage;           // [2][4][80 x 128 B]
-  float* ss_s = reinterpret_cast<float*>(Bbuf + kPpStages * kPpBStage);  // [128][2]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ss_s + kPpM * 2);
+  float* coef_s = reinterpret_cast<float*>(Bbuf + kPpStages * kPpBStage);  // [128][20]
+  float* ss_s = coef_s + kPpM * 20;                                            // [128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ss_s + kPpM);
   uint64_t* afull = bars;        // [2] 8 post-map warps wrote the A tiles
   uint64_t* aempty = bars + 2;   // [2] MMAs done with them
   uint64_t* bfull = bars + 4;    // [2] TMA bytes
@@ -129,7 +179,7 @@ __global__ void __launch_bounds__(kPpThreads, 1) post_project_kernel(
       mbar_init(&bfull[s], 1);
       mbar_init(&bempty[s], 1);
       mbar_init(&accfull[s], 1);
-      mbar_init(&accempty[s], kPpXWarps);
+      mbar_init(&accempty[s], kPpEpiWarps);
     }
     mbar_init(done, 1);
     fence_mbarrier_init();
@@ -219,69 +269,87 @@ __global__ void __launch_bounds__(kPpThreads, 1) post_project_kernel(
   } else {
     // ------------------------------------------------------------------ post-map warps
     const int xt = threadIdx.x - 64;  // 0..255
-    const int r = xt >> 1;            // token row in the tile
-    const int half = xt & 1;          // columns 32*half .. +31 of the block
+    const int ch = xt & 7;            // 8-column chunk of the block
+    const int tg = xt >> 3;           // tokens tg + 32 i, i < 4
     const int xw = warp - 2;          // 0..7
     int64_t n = 0, p = 0;
     bool dead = false;
+    // Block n's residual arrives in stage n & 1 by 16-byte asynchronous copies issued one block
+    // ahead (each thread copies, and later reads, only its own rows and chunk); its x chunks are
+    // loaded into registers one block ahead too. The post-map then overwrites the stage in place
+    // with out, which is the MMA's A operand.
+    uint4 xnext[kPpTokPerThread];
+    if (lo < hi) pp_issue_block(lo, (lo % C) * L, 0, Abuf, R, x, T, H, C, tg, ch, xnext);
     for (int64_t g = lo; g < hi; ++g, ++p) {
       const int64_t tile = g / C;
       const int64_t slot = g - tile * C;  // the chunk's rank in its tile: its split
       const int64_t hbs = slot * L;
       const int64_t hbe = min(static_cast<int64_t>(HB), hbs + L);
-      const int64_t t = tile * kPpM + r;
-      const bool live = t < T;
-      Coef20 k20;
-      if (live) {
-        k20 = load_coef<true>(post, comb, t);
-      } else {
-        k20.post = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int o = 0; o < 4; ++o) k20.c[o] = k20.post;
+      // The tile's post / comb into shared memory (the previous chunk's readers are past the
+      // epilogue's barriers): 128 tokens x 5 float4.
+      for (int e = xt; e < kPpM * 5; e += 32 * kPpXWarps) {
+        const int r = e / 5, v = e - r * 5;
+        const int64_t t = tile * kPpM + r;
+        float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (t < T)
+          val = v == 0 ? __ldg(reinterpret_cast<const float4*>(post + t * 4))
+                       : __ldg(reinterpret_cast<const float4*>(comb + t * 16 + (v - 1) * 4));
+        reinterpret_cast<float4*>(coef_s)[r * 5 + v] = val;
       }
-      float ss0 = 0.f, ss1 = 0.f;
+      dead = named_bar_or(1, 32 * kPpXWarps, dead);
+      float ss[kPpTokPerThread];
+#pragma unroll
+      for (int i = 0; i < kPpTokPerThread; ++i) ss[i] = 0.f;
       for (int64_t hb = hbs; hb < hbe; ++hb, ++n) {
         const int s = static_cast<int>(n & 1);
-        if (n >= kPpStages && !dead)
-          dead = !__all_sync(0xffffffffu,
-                             mbar_wait(&aempty[s], static_cast<uint32_t>((n >> 1) - 1) & 1u, 46));
-        if (dead) continue;
-        const int64_t h0 = hb * kPpHB + half * 32;
-        uint4 xv[4], rv[4][4];
+        uint4 xv[kPpTokPerThread];
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int64_t h = h0 + cc * 8;
-          if (live && h < H) {
-            xv[cc] = ld_stream_ro(x + t * H + h);
-#pragma unroll
-            for (int o = 0; o < 4; ++o) rv[cc][o] = ld_stream(R + (t * 4 + o) * H + h);
-          } else {
-            xv[cc] = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-            for (int o = 0; o < 4; ++o) rv[cc][o] = xv[cc];
-          }
+        for (int i = 0; i < kPpTokPerThread; ++i) xv[i] = xnext[i];
+        // Next block: into stage s ^ 1, once the MMAs of block n - 1 (its last user) are done.
+        const bool more = hb + 1 < hbe || g + 1 < hi;
+        if (more && n >= 1 && !dead)
+          dead = !__all_sync(0xffffffffu, mbar_wait(&aempty[s ^ 1],
+                                                   static_cast<uint32_t>((n - 1) >> 1) & 1u, 46));
+        if (more && !dead) {
+          if (hb + 1 < hbe)
+            pp_issue_block(g, hb + 1, s ^ 1, Abuf, R, x, T, H, C, tg, ch, xnext);
+          else
+            pp_issue_block(g + 1, ((g + 1) % C) * L, s ^ 1, Abuf, R, x, T, H, C, tg, ch, xnext);
+        } else {
+          cp_async_commit();  // an empty group keeps the group count per block
         }
-        uint8_t* As = Abuf + s * kPpAStage + r * 128;
+        cp_async_wait_prior();  // this block's copies (all groups but the newest) have landed
+        if (dead) continue;
+        const int64_t h = hb * kPpHB + ch * 8;
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int64_t h = h0 + cc * 8;
-          uint4 ov[4];
-          mix_vec8(xv[cc], rv[cc], k20, ov);
-          if (!(live && h < H)) {
+        for (int i = 0; i < kPpTokPerThread; ++i) {
+          const int r = tg + kPpTokStride * i;
+          const int64_t t = tile * kPpM + r;
+          const bool valid = t < T && h < H;
+          uint8_t* As = Abuf + s * kPpAStage + r * 128 + ((ch ^ (r & 7)) << 4);
+          const float4* cs = reinterpret_cast<const float4*>(coef_s) + r * 5;
+          Coef20 k20;
+          k20.post = cs[0];
+#pragma unroll
+          for (int o = 0; o < 4; ++o) k20.c[o] = cs[1 + o];
+          uint4 rv[4], ov[4];
+#pragma unroll
+          for (int m = 0; m < 4; ++m) rv[m] = *reinterpret_cast<const uint4*>(As + m * kPpABytes);
+          mix_vec8(xv[i], rv, k20, ov);
+          if (!valid) {
 #pragma unroll
             for (int m = 0; m < 4; ++m) ov[m] = make_uint4(0u, 0u, 0u, 0u);
           }
-          const int ch = half * 4 + cc;
 #pragma unroll
           for (int m = 0; m < 4; ++m) {
-            if (live && h < H) st_plain(out + (t * 4 + m) * H + h, ov[m]);
-            *reinterpret_cast<uint4*>(As + m * kPpABytes + ((ch ^ (r & 7)) << 4)) = ov[m];
+            if (valid) __stcg(reinterpret_cast<uint4*>(out + (t * 4 + m) * H + h), ov[m]);
+            *reinterpret_cast<uint4*>(As + m * kPpABytes) = ov[m];
             const uint32_t w4[4] = {ov[m].x, ov[m].y, ov[m].z, ov[m].w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const float a = bf16_lo(w4[q]), b = bf16_hi(w4[q]);
-              ss0 = fmaf(a, a, ss0);
-              ss1 = fmaf(b, b, ss1);
+              ss[i] = fmaf(a, a, ss[i]);
+              ss[i] = fmaf(b, b, ss[i]);
             }
           }
         }
@@ -290,13 +358,22 @@ __global__ void __launch_bounds__(kPpThreads, 1) post_project_kernel(
         if (lane == 0) mbar_arrive(&afull[s]);
       }
       // ---------------------------------------------------------------- piece epilogue
-      ss_s[r * 2 + half] = ss0 + ss1;
+      // A token's 8 chunk lanes are consecutive lanes: a fixed xor tree joins them.
+#pragma unroll
+      for (int i = 0; i < kPpTokPerThread; ++i) {
+        float v = ss[i];
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        if (ch == 0) ss_s[tg + kPpTokStride * i] = v;
+      }
       dead = named_bar_or(1, 32 * kPpXWarps, dead);
       const int b = static_cast<int>(p & 1);
-      if (!dead)
+      const bool epi = xw < kPpEpiWarps;  // warps 2..9 read the accumulator
+      if (epi && !dead)
         dead = !__all_sync(0xffffffffu,
                            mbar_wait(&accfull[b], static_cast<uint32_t>(p >> 1) & 1u, 47));
-      if (!dead) {
+      if (epi && !dead) {
         tc_fence_after();
         const int q = warp & 3;  // a warp reads TMEM lanes 32 * (warp % 4) .. + 31
         const int jh = xw >> 2;  // logits 12*jh .. 12*jh+11 (warps 2-5: 0, warps 6-9: 1)
@@ -321,7 +398,7 @@ __global__ void __launch_bounds__(kPpThreads, 1) post_project_kernel(
 #pragma unroll
           for (int v = 0; v < 3; ++v)
             dst[v] = make_float4(raw[4 * v], raw[4 * v + 1], raw[4 * v + 2], raw[4 * v + 3]);
-          if (jh == 0) sqrsum[slot * T + tr] = ss_s[row * 2] + ss_s[row * 2 + 1];
+          if (jh == 0) sqrsum[slot * T + tr] = ss_s[row];
           if (slot == C - 1) {  // the tile's last chunk: zero the splits beyond C
             const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
             for (int64_t sl = slot + 1; sl < S; ++sl) {
@@ -340,6 +417,7 @@ __global__ void __launch_bounds__(kPpThreads, 1) post_project_kernel(
       dead = named_bar_or(1, 32 * kPpXWarps, dead);
     }
   }
+  cp_async_wait_all();  // no copy into shared memory outlives the CTA
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -33,6 +33,7 @@ __device__ __forceinline__ BfSums bf_sum_splits(const float* __restrict__ dot_mi
                                                 const float* __restrict__ sqrsum, int nsplit,
                                                 int64_t T, int64_t t, int r) {
   BfSums a{0.f, 0.f, {0.f, 0.f, 0.f, 0.f}, 0.f};
+#pragma unroll 4
   for (int s = 0; s < nsplit; ++s) {
     const float* d = dot_mix + (static_cast<int64_t>(s) * T + t) * kMix;
     a.g0 += __ldg(d + r);
