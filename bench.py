@@ -261,6 +261,68 @@ def time_extras(mhc, R, x, out, y, pre, post, comb, hc_fn, scale, base, params, 
     return res
 
 
+def time_configs(mhc, inputs, dev, stream, reps=20):
+    """Per-call device time of the other workloads (small, post4k, decode T in {1,4,16,32}, tail),
+    each call timed alone with CUDA events. "flushed": a 256 MB buffer is written between calls
+    (outside the timed region) so no input is left in the 126 MB L2; "warm": no flush, inputs (and
+    for decode, hc_fn) L2-resident. Each call is queued behind a ~1 ms spin kernel so that the
+    host's time to issue it is not inside the events (device time; CUDA graphs remove that host
+    time in a serving loop). Returns {workload: {...}}."""
+    import torch
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def dev_bf16(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    def timed(fn, flushed):
+        fn()
+        ts = []
+        for _ in range(reps):
+            if flushed:
+                flush.fill_(1)
+            # Queue the call behind ~1 ms of spinning so that the host's time to issue it (Python,
+            # argument checks, launches) is not inside the events: device time only.
+            torch.cuda._sleep(2000000)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b) * 1e3)
+        return statistics.median(ts)
+
+    def one(w, do_pre=True):
+        R, x = dev_bf16(w.R), dev_bf16(w.x)
+        W, sc, bs = (torch.from_numpy(a).to(dev) for a in (w.hc_fn, w.hc_scale, w.hc_base))
+        prm = mhc.make_params(iters=w.iters, eps=w.eps, rms_eps=w.rms_eps, pre_eps=w.pre_eps,
+                              post_mult=w.post_mult)
+        ws = torch.empty(max(1, mhc.workspace_bytes(w.T, w.H)), dtype=torch.uint8, device=dev)
+        y, pre, post, comb = mhc.pre(R, W, sc, bs, workspace=ws, params=prm, stream=stream)
+        out = torch.empty_like(R)
+        rec = {"T": w.T, "H": w.H}
+        fp = lambda: mhc.pre(R, W, sc, bs, y=y, pre=pre, post=post, comb=comb, workspace=ws,
+                             params=prm, stream=stream)
+        fq = lambda: mhc.post(x, R, post, comb, out=out, stream=stream)
+        for flushed in (True, False):
+            tag = "flushed" if flushed else "warm"
+            if do_pre:
+                us = timed(fp, flushed)
+                rec[f"pre_us_{tag}"] = us
+                rec[f"pre_GBps_{tag}"] = pre_bytes(w.T, w.H) / us / 1e3
+            us = timed(fq, flushed)
+            rec[f"post_us_{tag}"] = us
+            rec[f"post_GBps_{tag}"] = post_bytes(w.T, w.H) / us / 1e3
+        return rec
+
+    res = {"small": one(inputs.small()), "post4k": one(inputs.post4k(), do_pre=False),
+           "tail": one(inputs.tail())}
+    for T in (1, 4, 16, 32):
+        res[f"decode_T{T}"] = one(inputs.decode(T))
+    assert mhc.device_status() == 0
+    del flush
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -278,7 +340,7 @@ def main():
                     help="override the workload's token count (profiling smaller cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
-                    help="skip timing the entries beside the step (pre from an external projection)")
+                    help="skip timing the entries beside the step and the other workloads")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -414,6 +476,9 @@ def main():
                "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
+    configs = None
+    if not args.no_extras and args.only == "both" and args.workload == "large":
+        configs = time_configs(mhc, inputs, dev, stream)
     extras = None
     if not args.no_extras and args.only == "both":
         extras = time_extras(mhc, R, x, out, y, pre, post, comb, hc_fn, scale, base, params,
@@ -467,6 +532,8 @@ def main():
             for v in extras.values():
                 v["frac_measured"] = v["GBps"] / hbm
             line["extras"] = extras
+        if configs:
+            line["configs"] = configs
         if not args.no_cpu_baseline and ws == 1:
             line["cpu_baseline"] = cpu_baseline(w)
         print(json.dumps(line), flush=True)
