@@ -28,3 +28,4 @@ from .c_oracle import (  # noqa: F401
 )
 from .big_fuse import big_fuse, big_fuse_with_prenorm, sum_of_squares  # noqa: F401
 from . import boundary  # noqa: F401
+from . import backward  # noqa: F401
