@@ -280,6 +280,41 @@ MHC_API int mhc_post_project(const uint16_t* x, const uint16_t* R, const float* 
                              size_t workspace_bytes, int64_t T, int64_t H, mhc_stream_t stream);
 
 /*
+ * Backward passes: the exact derivatives of the forward definitions. The pages name backward
+ * kernels (rwkv-ops mhu_jax.py: _mhc_post_op_ffi_bwd, mhc_pre_op's VJP) but print no formulas.
+ *
+ * mhc_post_backward  from d_out [T][4][H] bf16 and the forward's inputs x, R (bf16), post, comb:
+ *     d_x[h] = sum_n post[n] d_out[n][h]         (bf16 [T][H], fp32 math, one rounding)
+ *     d_R[o][h] = sum_n comb[o][n] d_out[n][h]   (bf16 [T][4][H])
+ *     d_post[n] = sum_h x[h] d_out[n][h]         (fp32 [T][4])
+ *     d_comb[o][n] = sum_h R[o][h] d_out[n][h]   (fp32 [T][4][4])
+ *   Sums over h are fixed-order (deterministic). Errors: MHC_ERR_INVALID_ARG, MHC_ERR_ALIAS (an
+ *   output overlapping an input or another output).
+ *
+ * mhc_pre_backward  from the upstream gradients of the pre-map's outputs -- d_y [T][H] bf16,
+ *   d_pre [T][4], d_post [T][4], d_comb [T][4][4] fp32, each optional (NULL = zero) -- and the
+ *   forward's inputs R, hc_fn, hc_scale, hc_base with the same params p:
+ *     d_R [T][4][H] bf16, d_hc_fn [4H][24] fp32, d_scale [3] fp32, d_base [24] fp32.
+ *   The projection is recomputed; gradients flow through the gates (sigmoid), the Sinkhorn rounds
+ *   (each normalisation Y = Z / (sum + eps) has dZ = (dY - sum(dY * Y)) / (sum + eps); the
+ *   row-max shift sends the row's sum of dA0 * A0, negated, to its first maximum), the logit
+ *   affine, rstd (d_ss = -rstd^3 / (8H) d_rstd) and the aggregate. Token sums are fixed-order.
+ *   workspace: mhc_pre_backward_workspace_bytes(T, H) bytes, 256-byte aligned.
+ *   Errors: MHC_ERR_INVALID_ARG, MHC_ERR_WORKSPACE_TOO_SMALL, MHC_ERR_ALIAS.
+ */
+MHC_API int mhc_post_backward(const uint16_t* d_out, const uint16_t* x, const uint16_t* R,
+                              const float* post, const float* comb, uint16_t* d_x, uint16_t* d_R,
+                              float* d_post, float* d_comb, int64_t T, int64_t H,
+                              mhc_stream_t stream);
+MHC_API size_t mhc_pre_backward_workspace_bytes(int64_t T, int64_t H);
+MHC_API int mhc_pre_backward(const uint16_t* d_y, const float* d_pre, const float* d_post,
+                             const float* d_comb, const uint16_t* R, const float* hc_fn,
+                             const float* hc_scale, const float* hc_base, uint16_t* d_R,
+                             float* d_hc_fn, float* d_scale, float* d_base, void* workspace,
+                             size_t workspace_bytes, int64_t T, int64_t H, const mhc_params* p,
+                             mhc_stream_t stream);
+
+/*
  * Model-boundary operations: the first layer's expand and the last layer's head. glm5next_mhc.rs
  * glm_hc_expand and hc_head_mean; hyper_connection_dispatch.rs hc_head_site (weighted head).
  * Streams are the library's bf16 [T][4][H] residual (the GLM page keeps them in fp32).

@@ -43,7 +43,8 @@ EXPORTED_SYMBOLS = (
     "mhc_version", "mhc_launch_count", "mhc_pre_noalloc", "mhc_pre_big_fuse",
     "mhc_pre_big_fuse_with_prenorm", "mhc_expand", "mhc_head_mean", "mhc_head",
     "mhc_head_workspace_bytes", "mhc_post_project", "mhc_post_project_splits",
-    "mhc_post_project_workspace_bytes",
+    "mhc_post_project_workspace_bytes", "mhc_post_backward", "mhc_pre_backward",
+    "mhc_pre_backward_workspace_bytes",
 )
 
 
@@ -121,6 +122,13 @@ def lib() -> ctypes.CDLL:
     L.mhc_post_project.restype = ctypes.c_int
     L.mhc_post_project.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I64,
                                    _I64, _P]
+    L.mhc_post_backward.restype = ctypes.c_int
+    L.mhc_post_backward.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _P]
+    L.mhc_pre_backward_workspace_bytes.restype = ctypes.c_size_t
+    L.mhc_pre_backward_workspace_bytes.argtypes = [_I64, _I64]
+    L.mhc_pre_backward.restype = ctypes.c_int
+    L.mhc_pre_backward.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                   ctypes.c_size_t, _I64, _I64, ctypes.POINTER(Params), _P]
     L.mhc_launch_count.restype = ctypes.c_uint64
     L.mhc_launch_count.argtypes = []
     _lib = L
@@ -319,6 +327,63 @@ def post_project(x, R, post, comb, hc_fn_next, *, out=None, dot_mix=None, sqrsum
                                 wsb, T, H, _stream(stream))
     _check(st, "mhc_post_project")
     return out, dot_mix, sqrsum
+
+
+def post_backward(d_out, x, R, post, comb, *, stream=None):
+    """Backward of the post-map. Returns (d_x [T,H] bf16, d_R [T,4,H] bf16, d_post [T,4],
+    d_comb [T,4,4] fp32)."""
+    import torch
+    _need(R, torch.bfloat16, None, "R")
+    T, hc, H = R.shape
+    _need(d_out, torch.bfloat16, (T, 4, H), "d_out")
+    _need(x, torch.bfloat16, (T, H), "x")
+    _need(post, torch.float32, None, "post")
+    _need(comb, torch.float32, (T, 4, 4), "comb")
+    dev = R.device
+    d_x = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    d_R = torch.empty_like(R)
+    d_post = torch.empty((T, 4), dtype=torch.float32, device=dev)
+    d_comb = torch.empty((T, 4, 4), dtype=torch.float32, device=dev)
+    st = lib().mhc_post_backward(_ptr(d_out), _ptr(x), _ptr(R), _ptr(post), _ptr(comb),
+                                 _ptr(d_x), _ptr(d_R), _ptr(d_post), _ptr(d_comb), T, H,
+                                 _stream(stream))
+    _check(st, "mhc_post_backward")
+    return d_x, d_R, d_post, d_comb
+
+
+def pre_backward(R, hc_fn, hc_scale, hc_base, *, d_y=None, d_pre=None, d_post=None, d_comb=None,
+                 params: Params | None = None, workspace=None, stream=None):
+    """Backward of the pre-map from the upstream gradients (any may be None). Returns
+    (d_R [T,4,H] bf16, d_hc_fn [4H,24], d_scale [3], d_base [24] fp32)."""
+    import torch
+    _need(R, torch.bfloat16, None, "R")
+    T, hc, H = R.shape
+    _need(hc_fn, torch.float32, (4 * H, 24), "hc_fn")
+    _need(hc_scale, torch.float32, (3,), "hc_scale")
+    _need(hc_base, torch.float32, (24,), "hc_base")
+    if d_y is not None:
+        _need(d_y, torch.bfloat16, (T, H), "d_y")
+    for name, tsr, n in (("d_pre", d_pre, 4), ("d_post", d_post, 4), ("d_comb", d_comb, 16)):
+        if tsr is not None:
+            _need(tsr, torch.float32, None, name)
+            if tsr.numel() != T * n:
+                raise ValueError(f"{name} must hold T*{n} values")
+    dev = R.device
+    d_R = torch.empty_like(R)
+    d_W = torch.empty((4 * H, 24), dtype=torch.float32, device=dev)
+    d_s = torch.empty(3, dtype=torch.float32, device=dev)
+    d_b = torch.empty(24, dtype=torch.float32, device=dev)
+    nws = int(lib().mhc_pre_backward_workspace_bytes(T, H))
+    if workspace is None and nws > 0:
+        workspace = torch.empty(nws, dtype=torch.uint8, device=dev)
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    p = params if params is not None else default_params()
+    st = lib().mhc_pre_backward(_ptr(d_y), _ptr(d_pre), _ptr(d_post), _ptr(d_comb), _ptr(R),
+                                _ptr(hc_fn), _ptr(hc_scale), _ptr(hc_base), _ptr(d_R), _ptr(d_W),
+                                _ptr(d_s), _ptr(d_b), _ptr(workspace), wsb, T, H, ctypes.byref(p),
+                                _stream(stream))
+    _check(st, "mhc_pre_backward")
+    return d_R, d_W, d_s, d_b
 
 
 def expand(hidden, *, streams=None, stream=None):

@@ -11,3 +11,4 @@
 #include "mhc_pre_bigfuse.cu"
 #include "mhc_boundary.cu"
 #include "mhc_post_project.cu"
+#include "mhc_backward.cu"

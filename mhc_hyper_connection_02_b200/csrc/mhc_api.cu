@@ -349,6 +349,73 @@ int mhc_post_project(const uint16_t* x, const uint16_t* R, const float* post, co
   return launch_post_project(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int mhc_post_backward(const uint16_t* d_out, const uint16_t* x, const uint16_t* R,
+                      const float* post, const float* comb, uint16_t* d_x, uint16_t* d_R,
+                      float* d_post, float* d_comb, int64_t T, int64_t H, mhc_stream_t stream) {
+  if (T < 0 || H <= 0 || !mul_ok(T, 4 * H, INT64_MAX / 4)) return MHC_ERR_INVALID_ARG;
+  if (T == 0) return MHC_OK;
+  if (!d_out || !x || !R || !post || !comb || !d_x || !d_R || !d_post || !d_comb)
+    return MHC_ERR_INVALID_ARG;
+  const size_t nR = static_cast<size_t>(T) * 8 * H, nx = static_cast<size_t>(T) * H * 2;
+  const void* outs[4] = {d_x, d_R, d_post, d_comb};
+  const size_t outn[4] = {nx, nR, static_cast<size_t>(T) * 16, static_cast<size_t>(T) * 64};
+  const void* ins[5] = {d_out, x, R, post, comb};
+  const size_t inn[5] = {nR, nx, nR, static_cast<size_t>(T) * 16, static_cast<size_t>(T) * 64};
+  for (int i = 0; i < 4; ++i) {
+    for (int j = 0; j < 5; ++j)
+      if (overlaps(outs[i], outn[i], ins[j], inn[j])) return MHC_ERR_ALIAS;
+    for (int j = i + 1; j < 4; ++j)
+      if (overlaps(outs[i], outn[i], outs[j], outn[j])) return MHC_ERR_ALIAS;
+  }
+  int st = bind_device(R);
+  if (st != MHC_OK) return st;
+  return launch_post_backward(d_out, x, R, post, comb, d_x, d_R, d_post, d_comb, T, H,
+                              reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t mhc_pre_backward_workspace_bytes(int64_t T, int64_t H) {
+  if (T <= 0 || H <= 0 || !mul_ok(T, 4 * H, INT64_MAX / 4)) return 0;
+  return pre_backward_workspace_bytes(T, H);
+}
+
+int mhc_pre_backward(const uint16_t* d_y, const float* d_pre, const float* d_post,
+                     const float* d_comb, const uint16_t* R, const float* hc_fn,
+                     const float* hc_scale, const float* hc_base, uint16_t* d_R, float* d_hc_fn,
+                     float* d_scale, float* d_base, void* workspace, size_t workspace_bytes,
+                     int64_t T, int64_t H, const mhc_params* p, mhc_stream_t stream) {
+  const mhc_params prm = p ? *p : mhc_default_params();
+  if (T < 0 || H <= 0 || !mul_ok(T, 4 * H, INT64_MAX / 4)) return MHC_ERR_INVALID_ARG;
+  if (prm.sinkhorn_iters < 1 || !(prm.sinkhorn_eps > 0.0f) || !isfinite(prm.sinkhorn_eps) ||
+      !(prm.rms_eps > 0.0f) || !isfinite(prm.rms_eps) || !(prm.pre_eps >= 0.0f) ||
+      !isfinite(prm.pre_eps) || !isfinite(prm.post_mult))
+    return MHC_ERR_INVALID_ARG;
+  if (T == 0) return MHC_OK;
+  if (!R || !hc_fn || !hc_scale || !hc_base || !d_R || !d_hc_fn || !d_scale || !d_base)
+    return MHC_ERR_INVALID_ARG;
+  const size_t need = mhc_pre_backward_workspace_bytes(T, H);
+  if (workspace_bytes < need || !workspace) return MHC_ERR_WORKSPACE_TOO_SMALL;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MHC_ERR_INVALID_ARG;
+  const size_t nR = static_cast<size_t>(T) * 8 * H, ny = static_cast<size_t>(T) * H * 2;
+  const size_t nfn = static_cast<size_t>(4 * H) * 96;
+  const void* outs[5] = {d_R, d_hc_fn, d_scale, d_base, workspace};
+  const size_t outn[5] = {nR, nfn, 12, 96, need};
+  const void* ins[8] = {d_y, d_pre, d_post, d_comb, R, hc_fn, hc_scale, hc_base};
+  const size_t inn[8] = {ny, static_cast<size_t>(T) * 16, static_cast<size_t>(T) * 16,
+                         static_cast<size_t>(T) * 64, nR, nfn, 12, 96};
+  for (int i = 0; i < 5; ++i) {
+    for (int j = 0; j < 8; ++j)
+      if (ins[j] && overlaps(outs[i], outn[i], ins[j], inn[j])) return MHC_ERR_ALIAS;
+    for (int j = i + 1; j < 5; ++j)
+      if (overlaps(outs[i], outn[i], outs[j], outn[j])) return MHC_ERR_ALIAS;
+  }
+  int st = bind_device(R);
+  if (st != MHC_OK) return st;
+  PreBwdArgs a{d_y, d_pre, d_post, d_comb, R, hc_fn, hc_scale, hc_base, d_R, d_hc_fn, d_scale,
+               d_base, workspace, T, H, prm.sinkhorn_iters, prm.sinkhorn_eps, prm.rms_eps,
+               prm.pre_eps, prm.post_mult};
+  return launch_pre_backward(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int mhc_expand(const uint16_t* hidden, uint16_t* streams, int64_t T, int64_t H,
                mhc_stream_t stream) {
   if (T < 0 || H <= 0 || !mul_ok(T, 4 * H, INT64_MAX / 4)) return MHC_ERR_INVALID_ARG;

@@ -1,0 +1,644 @@
+// Backward passes of the post-map and the pre-map: the exact derivatives of the forward
+// definitions ("FlashInfer mHC module deep dive" §2.1 post-map, §3.4 / §5.2 pre-map; rwkv-ops
+// mhu_jax.py names these backward kernels -- _mhc_post_op_ffi_bwd and mhc_pre_op's VJP -- without
+// formulas).
+//
+// post-map  d_x = sum_n post[n] d_out[n];  d_R[o] = sum_n comb[o][n] d_out[n];
+//           d_post[n] = sum_h x d_out[n];  d_comb[o][n] = sum_h R[o] d_out[n].
+//           One CTA per token: 16-byte loads, per-thread partial sums of the 20 coefficient
+//           gradients, a fixed-order block reduction.
+// pre-map   (upstream d_y, d_pre, d_post, d_comb; any may be absent)
+//   1. the projection is recomputed by the forward's own kernels (records of raw and ss);
+//   2. d_pre += sum_h d_y R_i (one CTA per token);
+//   3. per token (lane quad): rstd, logits, gates, the Sinkhorn states (recomputed round by round)
+//      and the reverse pass -> d_raw, d_ss, the gates, and the per-token terms of d_scale, d_base;
+//   4. d_scale, d_base: fixed-order sums over tokens;
+//   5. d_R = d_raw . hc_fn^T + 2 R d_ss + pre_i d_y (token x column tiles, hc_fn slice in shared
+//      memory, fp32 on CUDA cores);
+//   6. d_hc_fn = R_flat^T d_raw (a column slice of R per CTA, tokens summed in order).
+#include "mhc_device.cuh"
+#include "mhc_internal.h"
+
+namespace mhc {
+
+constexpr int kBwThreads = 256;
+
+// Warp sum of v (fixed xor tree) into red[slot * 8 + warp]; the caller adds the 8 warps in order
+// after a barrier.
+__device__ __forceinline__ void bw_warp_partial(float v, float* red, int slot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) red[slot * 8 + warp] = v;
+}
+
+// ------------------------------------------------------------------------------ post backward
+
+template <bool kVec>
+__global__ void __launch_bounds__(kBwThreads) post_bwd_kernel(
+    const uint16_t* __restrict__ dout, const uint16_t* __restrict__ x,
+    const uint16_t* __restrict__ R, const float* __restrict__ post,
+    const float* __restrict__ comb, uint16_t* __restrict__ dx, uint16_t* __restrict__ dR,
+    float* __restrict__ dpost, float* __restrict__ dcomb, int64_t H) {
+  __shared__ float red[20 * 8];
+  const int64_t t = blockIdx.x;
+  const int tid = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
+  float p[4], c[4][4];
+#pragma unroll
+  for (int n = 0; n < 4; ++n) p[n] = __ldg(post + t * 4 + n);
+#pragma unroll
+  for (int o = 0; o < 4; ++o)
+#pragma unroll
+    for (int n = 0; n < 4; ++n) c[o][n] = __ldg(comb + t * 16 + o * 4 + n);
+  float ap[4] = {0.f, 0.f, 0.f, 0.f}, ac[4][4];
+#pragma unroll
+  for (int o = 0; o < 4; ++o)
+#pragma unroll
+    for (int n = 0; n < 4; ++n) ac[o][n] = 0.f;
+  const uint16_t* dO = dout + t * 4 * H;
+  const uint16_t* Rt = R + t * 4 * H;
+  const uint16_t* xt = x + t * H;
+  if (kVec) {
+    for (int64_t v = tid; v < H / 8; v += kBwThreads) {
+      uint4 gv[4], rv[4];
+#pragma unroll
+      for (int n = 0; n < 4; ++n) gv[n] = ld_stream_ro(dO + n * H + v * 8);
+#pragma unroll
+      for (int o = 0; o < 4; ++o) rv[o] = ld_stream_ro(Rt + o * H + v * 8);
+      const uint4 xv = ld_stream_ro(xt + v * 8);
+      uint32_t ox[4], orr[4][4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float g[2][4], r[2][4], xx[2];
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+          const uint32_t w = (&gv[n].x)[q];
+          g[0][n] = bf16_lo(w);
+          g[1][n] = bf16_hi(w);
+        }
+#pragma unroll
+        for (int o = 0; o < 4; ++o) {
+          const uint32_t w = (&rv[o].x)[q];
+          r[0][o] = bf16_lo(w);
+          r[1][o] = bf16_hi(w);
+        }
+        xx[0] = bf16_lo((&xv.x)[q]);
+        xx[1] = bf16_hi((&xv.x)[q]);
+        float vx[2], vr[2][4];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float s = p[0] * g[e][0];
+#pragma unroll
+          for (int n = 1; n < 4; ++n) s = fmaf(p[n], g[e][n], s);
+          vx[e] = s;
+#pragma unroll
+          for (int o = 0; o < 4; ++o) {
+            float u = c[o][0] * g[e][0];
+#pragma unroll
+            for (int n = 1; n < 4; ++n) u = fmaf(c[o][n], g[e][n], u);
+            vr[e][o] = u;
+          }
+#pragma unroll
+          for (int n = 0; n < 4; ++n) {
+            ap[n] = fmaf(xx[e], g[e][n], ap[n]);
+#pragma unroll
+            for (int o = 0; o < 4; ++o) ac[o][n] = fmaf(r[e][o], g[e][n], ac[o][n]);
+          }
+        }
+        ox[q] = pack_bf16x2(vx[0], vx[1]);
+#pragma unroll
+        for (int o = 0; o < 4; ++o) orr[o][q] = pack_bf16x2(vr[0][o], vr[1][o]);
+      }
+      st_plain(dx + t * H + v * 8, make_uint4(ox[0], ox[1], ox[2], ox[3]));
+#pragma unroll
+      for (int o = 0; o < 4; ++o)
+        st_plain(dR + t * 4 * H + o * H + v * 8,
+                 make_uint4(orr[o][0], orr[o][1], orr[o][2], orr[o][3]));
+    }
+  } else {
+    for (int64_t h = tid; h < H; h += kBwThreads) {
+      float g[4], r[4];
+#pragma unroll
+      for (int n = 0; n < 4; ++n) g[n] = bf16_to_f32(dO[n * H + h]);
+#pragma unroll
+      for (int o = 0; o < 4; ++o) r[o] = bf16_to_f32(Rt[o * H + h]);
+      const float xx = bf16_to_f32(xt[h]);
+      float s = p[0] * g[0];
+#pragma unroll
+      for (int n = 1; n < 4; ++n) s = fmaf(p[n], g[n], s);
+      dx[t * H + h] = f32_to_bf16(s);
+#pragma unroll
+      for (int o = 0; o < 4; ++o) {
+        float u = c[o][0] * g[0];
+#pragma unroll
+        for (int n = 1; n < 4; ++n) u = fmaf(c[o][n], g[n], u);
+        dR[t * 4 * H + o * H + h] = f32_to_bf16(u);
+      }
+#pragma unroll
+      for (int n = 0; n < 4; ++n) {
+        ap[n] = fmaf(xx, g[n], ap[n]);
+#pragma unroll
+        for (int o = 0; o < 4; ++o) ac[o][n] = fmaf(r[o], g[n], ac[o][n]);
+      }
+    }
+  }
+  // Block sums of the 20 coefficient gradients, fixed order (xor tree in each warp, then warps).
+#pragma unroll
+  for (int n = 0; n < 4; ++n) bw_warp_partial(ap[n], red, n);
+#pragma unroll
+  for (int o = 0; o < 4; ++o)
+#pragma unroll
+    for (int n = 0; n < 4; ++n) bw_warp_partial(ac[o][n], red, 4 + o * 4 + n);
+  __syncthreads();
+  if (tid < 20) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) s += red[tid * 8 + w];
+    if (tid < 4)
+      dpost[t * 4 + tid] = s;
+    else
+      dcomb[t * 16 + (tid - 4)] = s;
+  }
+}
+
+int launch_post_backward(const uint16_t* dout, const uint16_t* x, const uint16_t* R,
+                         const float* post, const float* comb, uint16_t* dx, uint16_t* dR,
+                         float* dpost, float* dcomb, int64_t T, int64_t H, cudaStream_t s) {
+  if (T > 0x7fffffff) return -5;
+  const bool vec = H % 8 == 0 && aligned16(dout) && aligned16(x) && aligned16(R) &&
+                   aligned16(dx) && aligned16(dR);
+  const cudaError_t e =
+      vec ? launch_pdl(post_bwd_kernel<true>, dim3(static_cast<unsigned>(T)), dim3(kBwThreads), 0,
+                       s, dout, x, R, post, comb, dx, dR, dpost, dcomb, H)
+          : launch_pdl(post_bwd_kernel<false>, dim3(static_cast<unsigned>(T)), dim3(kBwThreads),
+                       0, s, dout, x, R, post, comb, dx, dR, dpost, dcomb, H);
+  if (e != cudaSuccess) return -4;
+  note_launches(1);
+  return 0;
+}
+
+
+// ------------------------------------------------------------------------------ pre backward
+
+constexpr int kBrec = 64;  // floats per token of the backward record (see pre_bwd_coef_kernel)
+
+// d_pre_tot[t][i] = d_pre[t][i] + sum_h d_y[t][h] R[t][i][h] (d_pre, d_y may be null).
+template <bool kVec>
+__global__ void __launch_bounds__(kBwThreads) pre_bwd_dpre_kernel(
+    const uint16_t* __restrict__ dy, const float* __restrict__ dpre,
+    const uint16_t* __restrict__ R, float* __restrict__ dpt, int64_t H) {
+  __shared__ float red[4 * 8];
+  const int64_t t = blockIdx.x;
+  const int tid = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
+  float a[4] = {0.f, 0.f, 0.f, 0.f};
+  if (dy) {
+    const uint16_t* Rt = R + t * 4 * H;
+    const uint16_t* gt = dy + t * H;
+    if (kVec) {
+      for (int64_t v = tid; v < H / 8; v += kBwThreads) {
+        const uint4 g = ld_stream_ro(gt + v * 8);
+        uint4 rv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) rv[i] = ld_stream_ro(Rt + i * H + v * 8);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float g0 = bf16_lo((&g.x)[q]), g1 = bf16_hi((&g.x)[q]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            a[i] = fmaf(g0, bf16_lo((&rv[i].x)[q]), a[i]);
+            a[i] = fmaf(g1, bf16_hi((&rv[i].x)[q]), a[i]);
+          }
+        }
+      }
+    } else {
+      for (int64_t h = tid; h < H; h += kBwThreads) {
+        const float g = bf16_to_f32(gt[h]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) a[i] = fmaf(g, bf16_to_f32(Rt[i * H + h]), a[i]);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) bw_warp_partial(a[i], red, i);
+  __syncthreads();
+  if (tid < 4) {
+    float s = dpre ? dpre[t * 4 + tid] : 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) s += red[tid * 8 + w];
+    dpt[t * 4 + tid] = s;
+  }
+}
+
+__device__ __forceinline__ float quad_sum(float v) {
+  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  return v + __shfl_xor_sync(0xffffffffu, v, 2);
+}
+
+// One Sinkhorn round on the quad's 4x4 (lane r holds row r): row normalisation then column
+// normalisation; returns B (after the row step), rs and cs (the normalisers) for the reverse pass.
+__device__ __forceinline__ void sk_round(float (&a)[4], float (&b)[4], float& rs, float (&cs)[4],
+                                         float eps) {
+  rs = ((a[0] + a[1]) + a[2]) + a[3] + eps;
+#pragma unroll
+  for (int n = 0; n < 4; ++n) b[n] = a[n] / rs;
+#pragma unroll
+  for (int n = 0; n < 4; ++n) {
+    cs[n] = quad_sum(b[n]) + eps;
+    a[n] = b[n] / cs[n];
+  }
+}
+
+// Per token, one lane quad (lane r: pre r, post r, comb row r). Writes the backward record
+// brec[t][64]: [0..23] d_raw, [24] d_ss, [25..28] pre gates, [29..31] the token's terms of
+// d_scale, [32..55] d_l (the token's term of d_base).
+__global__ void __launch_bounds__(256) pre_bwd_coef_kernel(
+    const float* __restrict__ part, int nrec, const float* __restrict__ dpt,
+    const float* __restrict__ dpost, const float* __restrict__ dcomb,
+    const float* __restrict__ scale, const float* __restrict__ base, float* __restrict__ brec,
+    int64_t T, int64_t K, FinishParams fp) {
+  const int lane = threadIdx.x & 31;
+  const int r = lane & 3;
+  const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 2;
+  const bool live = t < T;
+  const int64_t tt = live ? t : 0;
+  pdl_wait();
+  pdl_trigger();
+  float g0 = 0.f, g1 = 0.f, gc[4] = {0.f, 0.f, 0.f, 0.f}, ss = 0.f;
+  for (int s = 0; s < nrec; ++s) {
+    const float* rec = part + (static_cast<int64_t>(s) * T + tt) * 32;
+    g0 += __ldg(rec + r);
+    g1 += __ldg(rec + 4 + r);
+#pragma unroll
+    for (int n = 0; n < 4; ++n) gc[n] += __ldg(rec + 8 + 4 * r + n);
+    ss += __ldg(rec + 24);
+  }
+  const float rstd = 1.0f / sqrtf(ss / static_cast<float>(K) + fp.rms_eps);
+  const float s0 = __ldg(scale), s1 = __ldg(scale + 1), s2 = __ldg(scale + 2);
+  const float m0 = g0 * rstd, m1 = g1 * rstd;
+  float mc[4], lc[4];
+#pragma unroll
+  for (int n = 0; n < 4; ++n) {
+    mc[n] = gc[n] * rstd;
+    lc[n] = fmaf(mc[n], s2, __ldg(base + 8 + 4 * r + n));
+  }
+  const float sg0 = 1.0f / (1.0f + expf(-fmaf(m0, s0, __ldg(base + r))));
+  const float sg1 = 1.0f / (1.0f + expf(-fmaf(m1, s1, __ldg(base + 4 + r))));
+  const float dl0 = dpt[tt * 4 + r] * sg0 * (1.0f - sg0);
+  const float dl1 = (dpost ? dpost[tt * 4 + r] : 0.f) * fp.post_mult * sg1 * (1.0f - sg1);
+
+  // Sinkhorn reverse pass: the state entering round k is recomputed from A0 for each k.
+  float a0[4], dA[4];
+  const float mx = fmaxf(fmaxf(lc[0], lc[1]), fmaxf(lc[2], lc[3]));
+#pragma unroll
+  for (int n = 0; n < 4; ++n) {
+    a0[n] = expf(lc[n] - mx);
+    dA[n] = dcomb ? dcomb[tt * 16 + 4 * r + n] : 0.f;
+  }
+  for (int k = fp.iters - 1; k >= 0; --k) {
+    float a[4] = {a0[0], a0[1], a0[2], a0[3]}, b[4], rs, cs[4];
+    for (int j = 0; j < k; ++j) sk_round(a, b, rs, cs, fp.sinkhorn_eps);
+    sk_round(a, b, rs, cs, fp.sinkhorn_eps);  // round k: a is now C
+    float dB[4];
+#pragma unroll
+    for (int n = 0; n < 4; ++n) dB[n] = (dA[n] - quad_sum(dA[n] * a[n])) / cs[n];
+    const float rdot = ((dB[0] * b[0] + dB[1] * b[1]) + dB[2] * b[2]) + dB[3] * b[3];
+#pragma unroll
+    for (int n = 0; n < 4; ++n) dA[n] = (dB[n] - rdot) / rs;
+  }
+  float dlc[4], gsum = 0.f;
+  int am = 0;
+#pragma unroll
+  for (int n = 0; n < 4; ++n) {
+    dlc[n] = dA[n] * a0[n];
+    gsum += dlc[n];
+  }
+#pragma unroll
+  for (int n = 1; n < 4; ++n)
+    if (lc[n] > lc[am]) am = n;  // the first maximum takes the row-max shift's derivative
+#pragma unroll
+  for (int n = 0; n < 4; ++n)
+    if (n == am) dlc[n] -= gsum;
+
+  const float dm0 = dl0 * s0, dm1 = dl1 * s1;
+  float dmc[4];
+#pragma unroll
+  for (int n = 0; n < 4; ++n) dmc[n] = dlc[n] * s2;
+  float drs = fmaf(dm0, g0, dm1 * g1);
+#pragma unroll
+  for (int n = 0; n < 4; ++n) drs = fmaf(dmc[n], gc[n], drs);
+  const float d_rstd = quad_sum(drs);
+  const float d_ss = -0.5f * rstd * rstd * rstd / static_cast<float>(K) * d_rstd;
+  const float sc0 = quad_sum(dl0 * m0), sc1 = quad_sum(dl1 * m1);
+  float scc = 0.f;
+#pragma unroll
+  for (int n = 0; n < 4; ++n) scc = fmaf(dlc[n], mc[n], scc);
+  scc = quad_sum(scc);
+  if (live) {
+    float* o = brec + t * kBrec;
+    o[r] = dm0 * rstd;
+    o[4 + r] = dm1 * rstd;
+#pragma unroll
+    for (int n = 0; n < 4; ++n) o[8 + 4 * r + n] = dmc[n] * rstd;
+    o[25 + r] = sg0 + fp.pre_eps;
+    o[32 + r] = dl0;
+    o[36 + r] = dl1;
+#pragma unroll
+    for (int n = 0; n < 4; ++n) o[40 + 4 * r + n] = dlc[n];
+    if (r == 0) {
+      o[24] = d_ss;
+      o[29] = sc0;
+      o[30] = sc1;
+      o[31] = scc;
+    }
+  }
+}
+
+// d_scale[g] = sum_t brec[t][29 + g]; d_base[j] = sum_t brec[t][32 + j]: block b sums column b in a
+// fixed order (strided per thread, then a fixed tree).
+__global__ void __launch_bounds__(256) pre_bwd_param_kernel(const float* __restrict__ brec,
+                                                            float* __restrict__ dscale,
+                                                            float* __restrict__ dbase, int64_t T) {
+  __shared__ float red[8];
+  const int b = blockIdx.x;  // 0..26
+  const int col = b < 3 ? 29 + b : 32 + (b - 3);
+  pdl_wait();
+  pdl_trigger();
+  float v = 0.f;
+  for (int64_t t = threadIdx.x; t < T; t += blockDim.x) v += brec[t * kBrec + col];
+  bw_warp_partial(v, red, 0);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) s += red[w];
+    if (b < 3)
+      dscale[b] = s;
+    else
+      dbase[b - 3] = s;
+  }
+}
+
+constexpr int kDxCols = 256;  // columns of the flattened row per CTA
+constexpr int kDxTok = 32;    // tokens per sub-tile
+constexpr int kDxSub = 4;     // sub-tiles per CTA (the hc_fn slice is loaded once)
+
+// d_R = d_raw . hc_fn^T + 2 R d_ss + pre_i d_y, tile of kDxCols columns x kDxSub*kDxTok tokens.
+// Thread: 8-column chunk kc = tid % 32, tokens tk + 8 j (tk = tid / 32, j < 4) of a sub-tile.
+// Requires H % 8 == 0 and 16-byte aligned R, d_R, d_y.
+__global__ void __launch_bounds__(256) pre_bwd_dx_kernel(
+    const uint16_t* __restrict__ R, const uint16_t* __restrict__ dy,
+    const float* __restrict__ W, const float* __restrict__ brec, uint16_t* __restrict__ dR,
+    int64_t T, int64_t H) {
+  __shared__ __align__(16) float ws[kMix][kDxCols];   // hc_fn slice, transposed: [j][k]
+  __shared__ float tokv[kDxTok][32];                  // d_raw[24], d_ss, pre[4]
+  const int64_t K = 4 * H;
+  const int64_t k0 = static_cast<int64_t>(blockIdx.x) * kDxCols;
+  const int tid = threadIdx.x;
+  const int kc = tid & 31, tk = tid >> 5;
+  pdl_wait();
+  pdl_trigger();
+  for (int e = tid; e < kDxCols * kMix; e += 256) {
+    const int kk = e / kMix, j = e - kk * kMix;
+    ws[j][kk] = k0 + kk < K ? __ldg(W + (k0 + kk) * kMix + j) : 0.f;
+  }
+  const int64_t kb = k0 + kc * 8;  // this thread's 8 columns
+  const bool kvalid = kb < K;
+  const int64_t si = kvalid ? kb / H : 0;  // stream
+  const int64_t hh = kb - si * H;
+  for (int sub = 0; sub < kDxSub; ++sub) {
+    const int64_t t0 = (static_cast<int64_t>(blockIdx.y) * kDxSub + sub) * kDxTok;
+    if (t0 >= T) break;
+    __syncthreads();  // ws ready / previous sub-tile's tokv reads done
+    for (int e = tid; e < kDxTok * 29; e += 256) {
+      const int tl = e / 29, v = e - tl * 29;
+      tokv[tl][v] = t0 + tl < T ? brec[(t0 + tl) * kBrec + v] : 0.f;
+    }
+    __syncthreads();
+    float acc[4][8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
+#pragma unroll 4
+    for (int jj = 0; jj < kMix; ++jj) {
+      const float4 w0 = *reinterpret_cast<const float4*>(&ws[jj][kc * 8]);
+      const float4 w1 = *reinterpret_cast<const float4*>(&ws[jj][kc * 8 + 4]);
+      const float w8[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float d = tokv[tk + 8 * j][jj];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[j][e] = fmaf(d, w8[e], acc[j][e]);
+      }
+    }
+    if (!kvalid) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int tl = tk + 8 * j;
+      const int64_t t = t0 + tl;
+      if (t >= T) continue;
+      const uint4 xv = ld_stream_ro(R + t * K + kb);
+      const float dss2 = 2.0f * tokv[tl][24];
+      const float pi = tokv[tl][25 + si];
+      uint4 gv = make_uint4(0u, 0u, 0u, 0u);
+      if (dy) gv = ld_stream_ro(dy + t * H + hh);
+      uint32_t o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t xw = (&xv.x)[q], gw = (&gv.x)[q];
+        const float lo = fmaf(pi, bf16_lo(gw), fmaf(dss2, bf16_lo(xw), acc[j][2 * q]));
+        const float hi = fmaf(pi, bf16_hi(gw), fmaf(dss2, bf16_hi(xw), acc[j][2 * q + 1]));
+        o[q] = pack_bf16x2(lo, hi);
+      }
+      st_plain(dR + t * K + kb, make_uint4(o[0], o[1], o[2], o[3]));
+    }
+  }
+}
+
+// Any H / alignment: one thread per element of d_R.
+__global__ void __launch_bounds__(256) pre_bwd_dx_scalar_kernel(
+    const uint16_t* __restrict__ R, const uint16_t* __restrict__ dy,
+    const float* __restrict__ W, const float* __restrict__ brec, uint16_t* __restrict__ dR,
+    int64_t T, int64_t H) {
+  const int64_t K = 4 * H;
+  pdl_wait();
+  pdl_trigger();
+  for (int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u < T * K;
+       u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = u / K, k = u - t * K;
+    const float* o = brec + t * kBrec;
+    float acc = 0.f;
+#pragma unroll 4
+    for (int j = 0; j < kMix; ++j) acc = fmaf(o[j], __ldg(W + k * kMix + j), acc);
+    const int64_t i = k / H, h = k - i * H;
+    acc = fmaf(2.0f * o[24], bf16_to_f32(R[u]), acc);
+    if (dy) acc = fmaf(o[25 + i], bf16_to_f32(dy[t * H + h]), acc);
+    dR[u] = f32_to_bf16(acc);
+  }
+}
+
+constexpr int kDwCols = 64;   // columns of hc_fn per CTA
+constexpr int kDwTok = 32;    // tokens staged per step
+
+// Partial d_hc_fn over a token chunk: dwp[chunk][k][j] = sum_{t in chunk} R_flat[t][k] d_raw[t][j]
+// (tokens in increasing order). Thread: column kl = tid % 64, logits 6 g .. 6 g + 5 (g = tid / 64).
+__global__ void __launch_bounds__(256) pre_bwd_dw_kernel(const uint16_t* __restrict__ R,
+                                                         const float* __restrict__ brec,
+                                                         float* __restrict__ dwp, int64_t T,
+                                                         int64_t H, int64_t tchunk) {
+  __shared__ float xs[kDwTok][kDwCols];
+  __shared__ float ds[kDwTok][kMix];
+  const int64_t K = 4 * H;
+  const int64_t k0 = static_cast<int64_t>(blockIdx.x) * kDwCols;
+  const int64_t tb = static_cast<int64_t>(blockIdx.y) * tchunk;
+  const int64_t te = min(T, tb + tchunk);
+  const int tid = threadIdx.x;
+  const int kl = tid & 63, jg = tid >> 6;
+  pdl_wait();
+  pdl_trigger();
+  float acc[6] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int64_t t0 = tb; t0 < te; t0 += kDwTok) {
+    __syncthreads();
+    for (int e = tid; e < kDwTok * kDwCols; e += 256) {
+      const int tl = e / kDwCols, c = e - tl * kDwCols;
+      const int64_t t = t0 + tl, k = k0 + c;
+      xs[tl][c] = (t < te && k < K) ? bf16_to_f32(R[t * K + k]) : 0.f;
+    }
+    for (int e = tid; e < kDwTok * kMix; e += 256) {
+      const int tl = e / kMix, j = e - tl * kMix;
+      ds[tl][j] = t0 + tl < te ? brec[(t0 + tl) * kBrec + j] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int tl = 0; tl < kDwTok; ++tl) {
+      const float xv = xs[tl][kl];
+#pragma unroll
+      for (int j = 0; j < 6; ++j) acc[j] = fmaf(xv, ds[tl][6 * jg + j], acc[j]);
+    }
+  }
+  if (k0 + kl < K) {
+    float* o = dwp + (static_cast<int64_t>(blockIdx.y) * K + k0 + kl) * kMix + 6 * jg;
+#pragma unroll
+    for (int j = 0; j < 6; ++j) o[j] = acc[j];
+  }
+}
+
+// d_hc_fn[k][j] = sum over chunks (in order) of the partials.
+__global__ void __launch_bounds__(256) pre_bwd_dw_sum_kernel(const float* __restrict__ dwp,
+                                                             float* __restrict__ dw, int64_t KJ,
+                                                             int nchunk) {
+  pdl_wait();
+  pdl_trigger();
+  for (int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u < KJ;
+       u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float s = 0.f;
+    for (int c = 0; c < nchunk; ++c) s += dwp[c * KJ + u];
+    dw[u] = s;
+  }
+}
+
+struct BwPlan {
+  size_t proj, dpt, brec, dwp, total;
+  int64_t tchunk;
+  int nchunk;
+};
+
+static BwPlan bw_plan(int64_t T, int64_t H) {
+  BwPlan p;
+  auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+  size_t a = pre_tc_workspace_bytes(T, H), b = pre_cc_workspace_bytes(T, H);
+  p.proj = up(a > b ? a : b);
+  p.dpt = up(static_cast<size_t>(T) * 16);
+  p.brec = up(static_cast<size_t>(T) * kBrec * 4);
+  // Token chunks of d_hc_fn partials: enough CTAs (4H/64 x chunks) to fill the GPU twice.
+  const int64_t kcols = (4 * H + kDwCols - 1) / kDwCols;
+  int64_t nchunk = (2 * 148 * 4 + kcols - 1) / kcols;
+  if (nchunk < 1) nchunk = 1;
+  if (nchunk > (T + kDwTok - 1) / kDwTok) nchunk = (T + kDwTok - 1) / kDwTok;
+  if (nchunk < 1) nchunk = 1;
+  p.tchunk = ((T + nchunk - 1) / nchunk + kDwTok - 1) / kDwTok * kDwTok;
+  p.nchunk = static_cast<int>((T + p.tchunk - 1) / p.tchunk);
+  p.dwp = up(static_cast<size_t>(p.nchunk) * 4 * H * kMix * 4);
+  p.total = p.proj + p.dpt + p.brec + p.dwp;
+  return p;
+}
+
+size_t pre_backward_workspace_bytes(int64_t T, int64_t H) {
+  if (T <= 0 || H <= 0) return 0;
+  return bw_plan(T, H).total;
+}
+
+int launch_pre_backward(const PreBwdArgs& a, cudaStream_t s) {
+  const BwPlan plan = bw_plan(a.T, a.H);
+  uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+  float* dpt = reinterpret_cast<float*>(ws + plan.proj);
+  float* brec = reinterpret_cast<float*>(ws + plan.proj + plan.dpt);
+  float* dwp = reinterpret_cast<float*>(ws + plan.proj + plan.dpt + plan.brec);
+  const int64_t K = 4 * a.H;
+  if (a.T > 0x7fffffff) return -5;
+
+  // 1. The projection, by the forward's kernels (its records hold raw and ss).
+  PreArgs f{a.R, a.hc_fn, a.hc_scale, a.hc_base, nullptr, nullptr, nullptr, nullptr,
+            a.workspace, plan.proj, a.T, a.H, a.iters, a.sinkhorn_eps, a.rms_eps, a.pre_eps,
+            a.post_mult};
+  float* part = nullptr;
+  int nrec = 0;
+  const bool tc = pre_tc_supported(a.T, a.H) && aligned16(a.R) && aligned16(a.workspace) &&
+                  a.T >= 128;
+  int r = tc ? launch_tc_projection(f, s, &part, &nrec) : launch_cc_projection(f, s, &part, &nrec);
+  if (r != 0) return r;
+
+  const bool vec = a.H % 8 == 0 && aligned16(a.R) && aligned16(a.dR) &&
+                   (a.dy == nullptr || aligned16(a.dy));
+  const dim3 tok(static_cast<unsigned>(a.T));
+  cudaError_t e;
+  // 2. d_pre.
+  e = vec ? launch_pdl(pre_bwd_dpre_kernel<true>, tok, dim3(kBwThreads), 0, s, a.dy, a.dpre, a.R,
+                       dpt, a.H)
+          : launch_pdl(pre_bwd_dpre_kernel<false>, tok, dim3(kBwThreads), 0, s, a.dy, a.dpre, a.R,
+                       dpt, a.H);
+  if (e != cudaSuccess) return -4;
+  // 3. Coefficients' reverse pass.
+  const FinishParams fp{a.iters, a.sinkhorn_eps, a.rms_eps, a.pre_eps, a.post_mult};
+  e = launch_pdl(pre_bwd_coef_kernel, dim3(static_cast<unsigned>((4 * a.T + 255) / 256)),
+                 dim3(256), 0, s, static_cast<const float*>(part), nrec,
+                 static_cast<const float*>(dpt), a.dpost, a.dcomb, a.hc_scale, a.hc_base, brec,
+                 a.T, K, fp);
+  if (e != cudaSuccess) return -4;
+  // 4. d_scale, d_base.
+  e = launch_pdl(pre_bwd_param_kernel, dim3(3 + kMix), dim3(256), 0, s,
+                 static_cast<const float*>(brec), a.dscale, a.dbase, a.T);
+  if (e != cudaSuccess) return -4;
+  // 5. d_R.
+  if (vec) {
+    const dim3 g(static_cast<unsigned>((K + kDxCols - 1) / kDxCols),
+                 static_cast<unsigned>((a.T + kDxSub * kDxTok - 1) / (kDxSub * kDxTok)));
+    e = launch_pdl(pre_bwd_dx_kernel, g, dim3(256), 0, s, a.R, a.dy, a.hc_fn,
+                   static_cast<const float*>(brec), a.dR, a.T, a.H);
+  } else {
+    int64_t nb = (a.T * K + 255) / 256;
+    if (nb > 148 * 16) nb = 148 * 16;
+    e = launch_pdl(pre_bwd_dx_scalar_kernel, dim3(static_cast<unsigned>(nb)), dim3(256), 0, s,
+                   a.R, a.dy, a.hc_fn, static_cast<const float*>(brec), a.dR, a.T, a.H);
+  }
+  if (e != cudaSuccess) return -4;
+  // 6. d_hc_fn.
+  const dim3 gw(static_cast<unsigned>((K + kDwCols - 1) / kDwCols),
+                static_cast<unsigned>(plan.nchunk));
+  e = launch_pdl(pre_bwd_dw_kernel, gw, dim3(256), 0, s, a.R, static_cast<const float*>(brec),
+                 dwp, a.T, a.H, plan.tchunk);
+  if (e != cudaSuccess) return -4;
+  int64_t nb = (K * kMix + 255) / 256;
+  if (nb > 148 * 8) nb = 148 * 8;
+  e = launch_pdl(pre_bwd_dw_sum_kernel, dim3(static_cast<unsigned>(nb)), dim3(256), 0, s,
+                 static_cast<const float*>(dwp), a.dW, K * kMix, plan.nchunk);
+  if (e != cudaSuccess) return -4;
+  note_launches(7);
+  return 0;
+}
+
+}  // namespace mhc

@@ -75,6 +75,8 @@ struct PreArgs {
 // CUDA-core split-K path.
 size_t pre_cc_workspace_bytes(int64_t T, int64_t H);
 int launch_pre_cc(const PreArgs& a, cudaStream_t s);
+// Its projection step alone: records [nrec][T][32] (raw[24], ss) at the workspace start.
+int launch_cc_projection(const PreArgs& a, cudaStream_t s, float** part, int* nrec);
 
 // Tensor-core path: persistent fused kernel (launch returns 1 when the device cannot co-schedule
 // its grid; the caller then takes the split pair).
@@ -125,6 +127,35 @@ int post_project_splits(int64_t T, int64_t H);
 size_t post_project_workspace_bytes(int64_t T, int64_t H);
 int launch_post_project(const PostProjectArgs& a, cudaStream_t s);
 
+// Backward passes (mhc_backward.cu).
+int launch_post_backward(const uint16_t* dout, const uint16_t* x, const uint16_t* R,
+                         const float* post, const float* comb, uint16_t* dx, uint16_t* dR,
+                         float* dpost, float* dcomb, int64_t T, int64_t H, cudaStream_t s);
+struct PreBwdArgs {
+  const uint16_t* dy;   // [T][H] or null
+  const float* dpre;    // [T][4] or null
+  const float* dpost;   // [T][4] or null
+  const float* dcomb;   // [T][4][4] or null
+  const uint16_t* R;
+  const float* hc_fn;
+  const float* hc_scale;
+  const float* hc_base;
+  uint16_t* dR;
+  float* dW;            // [4H][24]
+  float* dscale;        // [3]
+  float* dbase;         // [24]
+  void* workspace;
+  int64_t T;
+  int64_t H;
+  int iters;
+  float sinkhorn_eps;
+  float rms_eps;
+  float pre_eps;
+  float post_mult;
+};
+size_t pre_backward_workspace_bytes(int64_t T, int64_t H);
+int launch_pre_backward(const PreBwdArgs& a, cudaStream_t s);
+
 // Model-boundary operations (mhc_boundary.cu).
 int launch_expand(const uint16_t* hidden, uint16_t* streams, int64_t T, int64_t H, cudaStream_t s);
 int launch_head_mean(const uint16_t* R, uint16_t* y, int64_t T, int64_t H, cudaStream_t s);
@@ -135,5 +166,7 @@ int launch_head_pad(const float* fn4, const float* scale1, const float* base4, f
 size_t pre_tc_workspace_bytes(int64_t T, int64_t H);
 bool pre_tc_supported(int64_t T, int64_t H);
 int launch_pre_tc(const PreArgs& a, cudaStream_t s);
+// The tensor path's split + projection alone: records [nrec][T][32] after the Bw operand.
+int launch_tc_projection(const PreArgs& a, cudaStream_t s, float** part, int* nrec);
 
 }  // namespace mhc

@@ -244,7 +244,8 @@ __global__ void __launch_bounds__(256) pre_cc_finish_kernel(
   aggregate_cols<kVec>(R, y, t, H, c0, c1, p);
 }
 
-int launch_pre_cc(const PreArgs& a, cudaStream_t s) {
+// Split-K projection partials: records [nsplit][T][32] (raw[24], ss) at the workspace start.
+int launch_cc_projection(const PreArgs& a, cudaStream_t s, float** part_out, int* nrec_out) {
   const CcPlan plan = cc_plan(a.T, a.H);
   const int64_t K = 4 * a.H;
   float* part = static_cast<float*>(a.workspace);
@@ -263,6 +264,17 @@ int launch_pre_cc(const PreArgs& a, cudaStream_t s) {
     pre_cc_partial_kernel<false, false><<<g1, 256, 0, s>>>(a.R, a.hc_fn, part, a.T, K, plan.KS);
   note_launches(1);
   if (cudaGetLastError() != cudaSuccess) return -4;
+  *part_out = part;
+  *nrec_out = static_cast<int>(plan.nsplit);
+  return 0;
+}
+
+int launch_pre_cc(const PreArgs& a, cudaStream_t s) {
+  const CcPlan plan = cc_plan(a.T, a.H);
+  float* part = nullptr;
+  int nrec = 0;
+  const int r = launch_cc_projection(a, s, &part, &nrec);
+  if (r != 0) return r;
 
   const int64_t nhb = (a.H + kAggCols - 1) / kAggCols;
   if (a.T > 0x7fffffff || 1 + nhb > 65535) return -5;

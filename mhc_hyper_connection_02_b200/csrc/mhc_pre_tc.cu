@@ -530,7 +530,9 @@ static bool make_map(CUtensorMap* m, const void* base, int64_t cols, int64_t row
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int launch_pre_tc(const PreArgs& a, cudaStream_t s) {
+// Split + projection: records [S][T][32] (raw[24], ss) in the workspace after Bw. Returns 0 or a
+// negative MHC_ERR_* code; *part_out / *nrec_out receive the records and their slot count.
+int launch_tc_projection(const PreArgs& a, cudaStream_t s, float** part_out, int* nrec_out) {
   const TcPlan plan = tc_plan(a.T, a.H);
   const int64_t K = 4 * a.H;
   uint8_t* ws = static_cast<uint8_t*>(a.workspace);
@@ -562,6 +564,17 @@ int launch_pre_tc(const PreArgs& a, cudaStream_t s) {
                  static_cast<int>(plan.kblocks), static_cast<int>(plan.S)) != cudaSuccess)
     return -4;
   note_launches(1);
+  *part_out = part;
+  *nrec_out = static_cast<int>(plan.S);
+  return 0;
+}
+
+int launch_pre_tc(const PreArgs& a, cudaStream_t s) {
+  const TcPlan plan = tc_plan(a.T, a.H);
+  float* part = nullptr;
+  int nrec = 0;
+  const int r = launch_tc_projection(a, s, &part, &nrec);
+  if (r != 0) return r;
 
   const FinishParams fp{a.iters, a.sinkhorn_eps, a.rms_eps, a.pre_eps, a.post_mult};
   const bool vec = aligned16(a.R) && aligned16(a.y) && aligned16(a.comb) && (a.H % 8 == 0);

@@ -33,10 +33,6 @@ import numpy as np
 from .c_oracle import bf16_bits_to_f64
 
 
-def _f64(a, bits):
-    return bf16_bits_to_f64(a) if bits else np.asarray(a, dtype=np.float64)
-
-
 def post_backward(d_out, x, R, post, comb):
     """d_out, R: uint16 bf16 bits [T,4,H]; x: bits [T,H]; post [T,4], comb [T,4,4] fp32.
     Returns fp64 d_x [T,H], d_R [T,4,H], d_post [T,4], d_comb [T,4,4]."""
@@ -86,10 +82,10 @@ def sinkhorn_vjp(lg, d_comb, iters, eps):
 
 
 def pre_backward(d_y, d_pre, d_post, d_comb, R, hc_fn, scale, base, rms_eps=1e-6, pre_eps=0.0,
-                 post_mult=2.0, iters=20, eps=1e-6):
+                 post_mult=2.0, iters=20, eps=1e-6, parts=False):
     """d_y: bits [T,H] (or None); d_pre, d_post [T,4], d_comb [T,4,4] fp32 (or None); R bits
     [T,4,H]; hc_fn [4H,24], scale [3], base [24] fp32. Returns fp64 d_R [T,4,H], d_hc_fn [4H,24],
-    d_scale [3], d_base [24]."""
+    d_scale [3], d_base [24] (and, with parts=True, a dict of per-token intermediates)."""
     T, _, H = R.shape
     K = 4 * H
     X = bf16_bits_to_f64(R).reshape(T, K)
@@ -124,4 +120,7 @@ def pre_backward(d_y, d_pre, d_post, d_comb, R, hc_fn, scale, base, rms_eps=1e-6
     dX = d_raw @ W.T + 2.0 * X * d_ss[:, None]
     dX = dX.reshape(T, 4, H) + pre[:, :, None] * dY[:, None, :]
     d_W = X.T @ d_raw
+    if parts:  # intermediate per-token quantities (used by tests to size error bounds)
+        return dX, d_W, d_scale, d_base, {"dl": dl, "m": m, "d_raw": d_raw, "d_ss": d_ss,
+                                          "pre": pre, "X": X}
     return dX, d_W, d_scale, d_base
