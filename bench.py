@@ -200,7 +200,9 @@ def time_extras(mhc, R, x, out, y, pre, post, comb, hc_fn, scale, base, params, 
     (4, external only) + pre/post/comb (96); expand: hidden (2H) + streams (8H); head_mean: R (8H)
     + y (2H); weighted head: R (8H) + y (2H) + weights (16), plus hc_fn (4H x 16) once; post with
     the next projection: the post-map's 18H + 80 plus S x 100 of partials; layer chain (that, then
-    the next pre-map from the partials): the post-map's bytes plus the pre-map's 10H + 96."""
+    the next pre-map from the partials): the post-map's bytes plus the pre-map's 10H + 96;
+    post-map backward: d_out (8H) + x (2H) + R (8H) + d_x (2H) + d_R (8H) + 160; pre-map backward:
+    R (8H) + d_y (2H) + d_R (8H) + 96 of coefficient gradients, plus hc_fn and d_hc_fn once."""
     import torch
     g = torch.Generator(device=dev).manual_seed(5)
     dot = torch.randn((1, T, 24), generator=g, device=dev) * 0.01
@@ -244,6 +246,19 @@ def time_extras(mhc, R, x, out, y, pre, post, comb, hc_fn, scale, base, params, 
 
         calls["post_project"] = (post_project, T * (18 * H + 80 + S * 100) + 4 * H * 96)
         calls["layer_chain"] = (layer_chain, T * (18 * H + 80) + T * (10 * H + 96) + 4 * H * 96)
+    # Backward passes on the step's tensors: d_out / d_y random bf16, upstream coefficient grads.
+    d_out = (torch.randn(R.shape, generator=g, device=dev) * 0.1).to(torch.bfloat16)
+    d_y = d_out[:, 0, :].contiguous()
+    d_c = torch.randn((T, 24), generator=g, device=dev) * 0.1
+    d_pre_u, d_post_u = d_c[:, 0:4].contiguous(), d_c[:, 4:8].contiguous()
+    d_comb_u = d_c[:, 8:24].contiguous()
+    bws = torch.empty(int(mhc.lib().mhc_pre_backward_workspace_bytes(T, H)), dtype=torch.uint8,
+                      device=dev)
+    calls["post_backward"] = (lambda: mhc.post_backward(d_out, x, R, post, comb, stream=stream),
+                              T * (28 * H + 160))
+    calls["pre_backward"] = (lambda: mhc.pre_backward(
+        R, hc_fn, scale, base, d_y=d_y, d_pre=d_pre_u, d_post=d_post_u, d_comb=d_comb_u,
+        params=params, workspace=bws, stream=stream), T * (18 * H + 96) + 4 * H * 96 * 2)
     res = {}
     for name, (fn, nbytes) in calls.items():
         for _ in range(3):

@@ -35,7 +35,7 @@ __device__ __forceinline__ void bw_warp_partial(float v, float* red, int slot) {
 // ------------------------------------------------------------------------------ post backward
 
 template <bool kVec>
-__global__ void __launch_bounds__(kBwThreads) post_bwd_kernel(
+__global__ void __launch_bounds__(kBwThreads, 2) post_bwd_kernel(
     const uint16_t* __restrict__ dout, const uint16_t* __restrict__ x,
     const uint16_t* __restrict__ R, const float* __restrict__ post,
     const float* __restrict__ comb, uint16_t* __restrict__ dx, uint16_t* __restrict__ dR,
@@ -418,6 +418,15 @@ __global__ void __launch_bounds__(256) pre_bwd_dx_kernel(
       tokv[tl][v] = t0 + tl < T ? brec[(t0 + tl) * kBrec + v] : 0.f;
     }
     __syncthreads();
+    // This thread's residual and d_y chunks first: their loads overlap the contraction below.
+    uint4 xr[4], gr[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t t = t0 + tk + 8 * j;
+      const bool ok = kvalid && t < T;
+      xr[j] = ok ? ld_stream_ro(R + t * K + kb) : make_uint4(0u, 0u, 0u, 0u);
+      gr[j] = (ok && dy) ? ld_stream_ro(dy + t * H + hh) : make_uint4(0u, 0u, 0u, 0u);
+    }
     float acc[4][8];
 #pragma unroll
     for (int j = 0; j < 4; ++j)
@@ -441,11 +450,9 @@ __global__ void __launch_bounds__(256) pre_bwd_dx_kernel(
       const int tl = tk + 8 * j;
       const int64_t t = t0 + tl;
       if (t >= T) continue;
-      const uint4 xv = ld_stream_ro(R + t * K + kb);
+      const uint4 xv = xr[j], gv = gr[j];
       const float dss2 = 2.0f * tokv[tl][24];
       const float pi = tokv[tl][25 + si];
-      uint4 gv = make_uint4(0u, 0u, 0u, 0u);
-      if (dy) gv = ld_stream_ro(dy + t * H + hh);
       uint32_t o[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -481,26 +488,32 @@ __global__ void __launch_bounds__(256) pre_bwd_dx_scalar_kernel(
   }
 }
 
-constexpr int kDwCols = 64;   // columns of hc_fn per CTA
+constexpr int kDwCols = 256;  // columns of hc_fn per CTA
 constexpr int kDwTok = 32;    // tokens staged per step
 
 // Partial d_hc_fn over a token chunk: dwp[chunk][k][j] = sum_{t in chunk} R_flat[t][k] d_raw[t][j]
-// (tokens in increasing order). Thread: column kl = tid % 64, logits 6 g .. 6 g + 5 (g = tid / 64).
+// (tokens in increasing order). Thread: columns 4 kq .. 4 kq + 3 (kq = tid % 64) x logits
+// 6 g .. 6 g + 5 (g = tid / 64): 24 accumulators, fed per token by one 16-byte and three 8-byte
+// shared-memory loads.
 __global__ void __launch_bounds__(256) pre_bwd_dw_kernel(const uint16_t* __restrict__ R,
                                                          const float* __restrict__ brec,
                                                          float* __restrict__ dwp, int64_t T,
                                                          int64_t H, int64_t tchunk) {
-  __shared__ float xs[kDwTok][kDwCols];
-  __shared__ float ds[kDwTok][kMix];
+  __shared__ __align__(16) float xs[kDwTok][kDwCols];
+  __shared__ __align__(16) float ds[kDwTok][kMix];
   const int64_t K = 4 * H;
   const int64_t k0 = static_cast<int64_t>(blockIdx.x) * kDwCols;
   const int64_t tb = static_cast<int64_t>(blockIdx.y) * tchunk;
   const int64_t te = min(T, tb + tchunk);
   const int tid = threadIdx.x;
-  const int kl = tid & 63, jg = tid >> 6;
+  const int kq = tid & 63, jg = tid >> 6;
   pdl_wait();
   pdl_trigger();
-  float acc[6] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float acc[4][6];
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+#pragma unroll
+    for (int j = 0; j < 6; ++j) acc[c][j] = 0.f;
   for (int64_t t0 = tb; t0 < te; t0 += kDwTok) {
     __syncthreads();
     for (int e = tid; e < kDwTok * kDwCols; e += 256) {
@@ -513,17 +526,28 @@ __global__ void __launch_bounds__(256) pre_bwd_dw_kernel(const uint16_t* __restr
       ds[tl][j] = t0 + tl < te ? brec[(t0 + tl) * kBrec + j] : 0.f;
     }
     __syncthreads();
-#pragma unroll 4
+#pragma unroll 2
     for (int tl = 0; tl < kDwTok; ++tl) {
-      const float xv = xs[tl][kl];
+      const float4 x4 = *reinterpret_cast<const float4*>(&xs[tl][4 * kq]);
+      const float2 d01 = *reinterpret_cast<const float2*>(&ds[tl][6 * jg]);
+      const float2 d23 = *reinterpret_cast<const float2*>(&ds[tl][6 * jg + 2]);
+      const float2 d45 = *reinterpret_cast<const float2*>(&ds[tl][6 * jg + 4]);
+      const float xv[4] = {x4.x, x4.y, x4.z, x4.w};
+      const float dv[6] = {d01.x, d01.y, d23.x, d23.y, d45.x, d45.y};
 #pragma unroll
-      for (int j = 0; j < 6; ++j) acc[j] = fmaf(xv, ds[tl][6 * jg + j], acc[j]);
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int j = 0; j < 6; ++j) acc[c][j] = fmaf(xv[c], dv[j], acc[c][j]);
     }
   }
-  if (k0 + kl < K) {
-    float* o = dwp + (static_cast<int64_t>(blockIdx.y) * K + k0 + kl) * kMix + 6 * jg;
 #pragma unroll
-    for (int j = 0; j < 6; ++j) o[j] = acc[j];
+  for (int c = 0; c < 4; ++c) {
+    const int64_t k = k0 + 4 * kq + c;
+    if (k < K) {
+      float* o = dwp + (static_cast<int64_t>(blockIdx.y) * K + k) * kMix + 6 * jg;
+#pragma unroll
+      for (int j = 0; j < 6; ++j) o[j] = acc[c][j];
+    }
   }
 }
 
@@ -554,9 +578,9 @@ static BwPlan bw_plan(int64_t T, int64_t H) {
   p.proj = up(a > b ? a : b);
   p.dpt = up(static_cast<size_t>(T) * 16);
   p.brec = up(static_cast<size_t>(T) * kBrec * 4);
-  // Token chunks of d_hc_fn partials: enough CTAs (4H/64 x chunks) to fill the GPU twice.
+  // Token chunks of d_hc_fn partials: enough CTAs (4H/256 x chunks) for about sixteen per SM.
   const int64_t kcols = (4 * H + kDwCols - 1) / kDwCols;
-  int64_t nchunk = (2 * 148 * 4 + kcols - 1) / kcols;
+  int64_t nchunk = (16 * 148 + kcols - 1) / kcols;
   if (nchunk < 1) nchunk = 1;
   if (nchunk > (T + kDwTok - 1) / kDwTok) nchunk = (T + kDwTok - 1) / kDwTok;
   if (nchunk < 1) nchunk = 1;
