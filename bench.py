@@ -176,11 +176,11 @@ def load_traffic():
         return {}
 
 
-# Source files that define each map's kernels; a recorded DRAM traffic figure is used only while
-# their digest matches the one it was recorded with.
+# Source files that define each map's kernels (device code and launch configuration); a recorded
+# DRAM traffic figure is used only while their digest matches the one it was recorded with.
 KERNEL_SOURCES = {
-    "post": ["mhc_post.cu", "mhc_device.cuh", "mhc_internal.h"],
-    "pre": ["mhc_pre_tc.cu", "mhc_pre_cc.cu", "mhc_device.cuh", "mhc_internal.h"],
+    "post": ["mhc_post.cu", "mhc_device.cuh"],
+    "pre": ["mhc_pre_tc.cu", "mhc_pre_cc.cu", "mhc_device.cuh"],
 }
 
 
