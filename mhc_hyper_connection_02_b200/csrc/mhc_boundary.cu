@@ -35,6 +35,8 @@ __global__ void __launch_bounds__(256) expand_vec8_kernel(const uint16_t* __rest
 __global__ void __launch_bounds__(256) expand_scalar_kernel(const uint16_t* __restrict__ hidden,
                                                             uint16_t* __restrict__ streams,
                                                             int64_t T, int64_t H) {
+  pdl_wait();  // launched as a programmatic dependent of the previous grid
+  pdl_trigger();
   const int64_t total = T * H;
   for (int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u < total;
        u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -78,6 +80,8 @@ __global__ void __launch_bounds__(256) head_mean_vec8_kernel(const uint16_t* __r
 __global__ void __launch_bounds__(256) head_mean_scalar_kernel(const uint16_t* __restrict__ R,
                                                                uint16_t* __restrict__ y, int64_t T,
                                                                int64_t H) {
+  pdl_wait();  // launched as a programmatic dependent of the previous grid
+  pdl_trigger();
   const int64_t total = T * H;
   for (int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u < total;
        u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -97,6 +101,8 @@ __global__ void __launch_bounds__(256) head_pad_kernel(const float* __restrict__
                                                        const float* __restrict__ base4,
                                                        float* __restrict__ fn24,
                                                        float* __restrict__ sb, int64_t K) {
+  pdl_wait();  // launched as a programmatic dependent of the previous grid
+  pdl_trigger();
   const int64_t total = K * kMix;
   for (int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u < total;
        u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -129,8 +135,8 @@ int launch_expand(const uint16_t* hidden, uint16_t* streams, int64_t T, int64_t 
     e = launch_pdl(expand_vec8_kernel, dim3(stream_grid(T * (H / 8))), dim3(256), 0, s, hidden,
                    streams, T, H / 8);
   } else {
-    expand_scalar_kernel<<<stream_grid(T * H), 256, 0, s>>>(hidden, streams, T, H);
-    e = cudaGetLastError();
+    e = launch_pdl(expand_scalar_kernel, dim3(stream_grid(T * H)), dim3(256), 0, s, hidden, streams,
+                   T, H);
   }
   note_launches(1);
   return e == cudaSuccess ? 0 : -4;
@@ -142,8 +148,7 @@ int launch_head_mean(const uint16_t* R, uint16_t* y, int64_t T, int64_t H, cudaS
     e = launch_pdl(head_mean_vec8_kernel, dim3(stream_grid(T * (H / 8))), dim3(256), 0, s, R, y,
                    T, H / 8);
   } else {
-    head_mean_scalar_kernel<<<stream_grid(T * H), 256, 0, s>>>(R, y, T, H);
-    e = cudaGetLastError();
+    e = launch_pdl(head_mean_scalar_kernel, dim3(stream_grid(T * H)), dim3(256), 0, s, R, y, T, H);
   }
   note_launches(1);
   return e == cudaSuccess ? 0 : -4;
@@ -152,9 +157,10 @@ int launch_head_mean(const uint16_t* R, uint16_t* y, int64_t T, int64_t H, cudaS
 int launch_head_pad(const float* fn4, const float* scale1, const float* base4, float* fn24,
                     float* sb, int64_t H, cudaStream_t s) {
   const int64_t K = 4 * H;
-  head_pad_kernel<<<stream_grid(K * kMix), 256, 0, s>>>(fn4, scale1, base4, fn24, sb, K);
+  const cudaError_t e = launch_pdl(head_pad_kernel, dim3(stream_grid(K * kMix)), dim3(256), 0, s,
+                                   fn4, scale1, base4, fn24, sb, K);
   note_launches(1);
-  return cudaGetLastError() == cudaSuccess ? 0 : -4;
+  return e == cudaSuccess ? 0 : -4;
 }
 
 }  // namespace mhc

@@ -85,6 +85,8 @@ __global__ void __launch_bounds__(256) post_vec8_kernel(const uint16_t* __restri
                                                         const float* __restrict__ post,
                                                         const float* __restrict__ comb,
                                                         uint16_t* out, int64_t T, int64_t H8) {
+  pdl_wait();  // launched as a programmatic dependent of the previous grid
+  pdl_trigger();
   const int64_t total = T * H8;
   const int64_t H = H8 * 8;
   for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < total;
@@ -111,6 +113,8 @@ template <bool kAlignedCoef>
 __global__ void __launch_bounds__(256) post_scalar_kernel(const uint16_t* x, const uint16_t* R,
                                                           const float* post, const float* comb,
                                                           uint16_t* out, int64_t T, int64_t H) {
+  pdl_wait();  // launched as a programmatic dependent of the previous grid
+  pdl_trigger();
   const int64_t total = T * H;
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
        e += (int64_t)gridDim.x * blockDim.x) {
@@ -247,12 +251,15 @@ int launch_post_vec8(const uint16_t* x, const uint16_t* R, const float* post, co
   const int64_t H8 = H / 8;
   const int threads = 256;
   const int blocks = grid_for(T * H8, threads, device_sm_count() * 64);
+  cudaError_t e;
   if (out == R)
-    post_vec8_kernel<true><<<blocks, threads, 0, s>>>(x, R, post, comb, out, T, H8);
+    e = launch_pdl(post_vec8_kernel<true>, dim3(blocks), dim3(threads), 0, s, x, R,
+                   post, comb, out, T, H8);
   else
-    post_vec8_kernel<false><<<blocks, threads, 0, s>>>(x, R, post, comb, out, T, H8);
+    e = launch_pdl(post_vec8_kernel<false>, dim3(blocks), dim3(threads), 0, s, x, R,
+                   post, comb, out, T, H8);
   note_launches(1);
-  return cudaGetLastError() == cudaSuccess ? 0 : -4;
+  return e == cudaSuccess ? 0 : -4;
 }
 
 int launch_post_scalar(const uint16_t* x, const uint16_t* R, const float* post, const float* comb,
@@ -260,12 +267,15 @@ int launch_post_scalar(const uint16_t* x, const uint16_t* R, const float* post, 
   const int threads = 256;
   const int blocks = grid_for(T * H, threads, device_sm_count() * 64);
   const bool aligned = aligned16(post) && aligned16(comb);
+  cudaError_t e;
   if (aligned)
-    post_scalar_kernel<true><<<blocks, threads, 0, s>>>(x, R, post, comb, out, T, H);
+    e = launch_pdl(post_scalar_kernel<true>, dim3(blocks), dim3(threads), 0, s, x, R,
+                   post, comb, out, T, H);
   else
-    post_scalar_kernel<false><<<blocks, threads, 0, s>>>(x, R, post, comb, out, T, H);
+    e = launch_pdl(post_scalar_kernel<false>, dim3(blocks), dim3(threads), 0, s, x, R,
+                   post, comb, out, T, H);
   note_launches(1);
-  return cudaGetLastError() == cudaSuccess ? 0 : -4;
+  return e == cudaSuccess ? 0 : -4;
 }
 
 int launch_post_persistent(const uint16_t* x, const uint16_t* R, const float* post,

@@ -76,6 +76,8 @@ __global__ void __launch_bounds__(256) pre_cc_partial_kernel(const uint16_t* __r
                                                              const float* __restrict__ W,
                                                              float* __restrict__ part, int64_t T,
                                                              int64_t K, int64_t KS) {
+  pdl_wait();  // launched as a programmatic dependent of the previous grid
+  pdl_trigger();
   __shared__ float red[kCcWarps][kCcTokens][25];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -215,6 +217,8 @@ __global__ void __launch_bounds__(256) pre_cc_finish_kernel(
     const float* __restrict__ scale, const float* __restrict__ base, uint16_t* __restrict__ y,
     float* __restrict__ pre, float* __restrict__ post, float* __restrict__ comb, int64_t T,
     int64_t H, FinishParams fp) {
+  pdl_wait();  // launched as a programmatic dependent of the previous grid
+  pdl_trigger();
   __shared__ float red[kCcWarps][25];
   __shared__ float pre_s[4];
   const int warp = threadIdx.x >> 5;
@@ -254,16 +258,21 @@ int launch_cc_projection(const PreArgs& a, cudaStream_t s, float** part_out, int
   const dim3 g1(static_cast<unsigned>(groups), static_cast<unsigned>(plan.nsplit));
   const bool vecR = aligned16(a.R) && (K % 8 == 0);
   const bool alignW = aligned16(a.hc_fn);
+  cudaError_t e;
   if (vecR && alignW)
-    pre_cc_partial_kernel<true, true><<<g1, 256, 0, s>>>(a.R, a.hc_fn, part, a.T, K, plan.KS);
+    e = launch_pdl(pre_cc_partial_kernel<true, true>, g1, dim3(256), 0, s, a.R,
+                   a.hc_fn, part, a.T, K, plan.KS);
   else if (vecR)
-    pre_cc_partial_kernel<true, false><<<g1, 256, 0, s>>>(a.R, a.hc_fn, part, a.T, K, plan.KS);
+    e = launch_pdl(pre_cc_partial_kernel<true, false>, g1, dim3(256), 0, s, a.R,
+                   a.hc_fn, part, a.T, K, plan.KS);
   else if (alignW)
-    pre_cc_partial_kernel<false, true><<<g1, 256, 0, s>>>(a.R, a.hc_fn, part, a.T, K, plan.KS);
+    e = launch_pdl(pre_cc_partial_kernel<false, true>, g1, dim3(256), 0, s, a.R,
+                   a.hc_fn, part, a.T, K, plan.KS);
   else
-    pre_cc_partial_kernel<false, false><<<g1, 256, 0, s>>>(a.R, a.hc_fn, part, a.T, K, plan.KS);
+    e = launch_pdl(pre_cc_partial_kernel<false, false>, g1, dim3(256), 0, s, a.R,
+                   a.hc_fn, part, a.T, K, plan.KS);
   note_launches(1);
-  if (cudaGetLastError() != cudaSuccess) return -4;
+  if (e != cudaSuccess) return -4;
   *part_out = part;
   *nrec_out = static_cast<int>(plan.nsplit);
   return 0;
@@ -281,14 +290,15 @@ int launch_pre_cc(const PreArgs& a, cudaStream_t s) {
   const dim3 g2(static_cast<unsigned>(a.T), static_cast<unsigned>(1 + nhb));
   const FinishParams fp{a.iters, a.sinkhorn_eps, a.rms_eps, a.pre_eps, a.post_mult};
   const bool vec = aligned16(a.R) && aligned16(a.y) && (a.H % 8 == 0);
+  cudaError_t e;
   if (vec)
-    pre_cc_finish_kernel<true><<<g2, 256, 0, s>>>(a.R, part, plan.nsplit, a.hc_scale, a.hc_base,
-                                                  a.y, a.pre, a.post, a.comb, a.T, a.H, fp);
+    e = launch_pdl(pre_cc_finish_kernel<true>, g2, dim3(256), 0, s, a.R, part, plan.nsplit,
+                   a.hc_scale, a.hc_base, a.y, a.pre, a.post, a.comb, a.T, a.H, fp);
   else
-    pre_cc_finish_kernel<false><<<g2, 256, 0, s>>>(a.R, part, plan.nsplit, a.hc_scale, a.hc_base,
-                                                   a.y, a.pre, a.post, a.comb, a.T, a.H, fp);
+    e = launch_pdl(pre_cc_finish_kernel<false>, g2, dim3(256), 0, s, a.R, part, plan.nsplit,
+                   a.hc_scale, a.hc_base, a.y, a.pre, a.post, a.comb, a.T, a.H, fp);
   note_launches(1);
-  return cudaGetLastError() == cudaSuccess ? 0 : -4;
+  return e == cudaSuccess ? 0 : -4;
 }
 
 }  // namespace mhc

@@ -597,8 +597,9 @@ int launch_pre_tc(const PreArgs& a, cudaStream_t s) {
     const int64_t nhb = (a.H + kAggCols - 1) / kAggCols;
     if (a.T > 0x7fffffff || 1 + nhb > 65535) return -5;
     const dim3 g2(static_cast<unsigned>(a.T), static_cast<unsigned>(1 + nhb));
-    pre_cc_finish_kernel<false><<<g2, 256, 0, s>>>(a.R, part, plan.S, a.hc_scale, a.hc_base,
-                                                   a.y, a.pre, a.post, a.comb, a.T, a.H, fp);
+    if (launch_pdl(pre_cc_finish_kernel<false>, g2, dim3(256), 0, s, a.R, part, plan.S,
+                   a.hc_scale, a.hc_base, a.y, a.pre, a.post, a.comb, a.T, a.H, fp) != cudaSuccess)
+      return -4;
   }
   note_launches(1);
   return cudaGetLastError() == cudaSuccess ? 0 : -4;

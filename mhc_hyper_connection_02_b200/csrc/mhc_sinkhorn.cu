@@ -12,6 +12,8 @@ namespace mhc {
 template <bool kAligned>
 __global__ void __launch_bounds__(256) sinkhorn_kernel(const float* logits, float* comb, int64_t T,
                                                        int iters, float eps) {
+  pdl_wait();  // launched as a programmatic dependent of the previous grid
+  pdl_trigger();
   const int64_t gid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   const int64_t t = gid >> 2;
   const int q = static_cast<int>(gid & 3);
@@ -44,12 +46,14 @@ int launch_sinkhorn(const float* logits, float* comb, int64_t T, int iters, floa
   const int threads = 256;
   const int64_t blocks = (4 * T + threads - 1) / threads;
   if (blocks > 0x7fffffff) return -1;
-  if (aligned16(logits) && aligned16(comb))
-    sinkhorn_kernel<true><<<static_cast<unsigned>(blocks), threads, 0, s>>>(logits, comb, T, iters, eps);
-  else
-    sinkhorn_kernel<false><<<static_cast<unsigned>(blocks), threads, 0, s>>>(logits, comb, T, iters, eps);
+  const dim3 grid(static_cast<unsigned>(blocks));
+  const cudaError_t e =
+      (aligned16(logits) && aligned16(comb))
+          ? launch_pdl(sinkhorn_kernel<true>, grid, dim3(threads), 0, s, logits, comb, T, iters, eps)
+          : launch_pdl(sinkhorn_kernel<false>, grid, dim3(threads), 0, s, logits, comb, T, iters,
+                       eps);
   note_launches(1);
-  return cudaGetLastError() == cudaSuccess ? 0 : -4;
+  return e == cudaSuccess ? 0 : -4;
 }
 
 }  // namespace mhc
