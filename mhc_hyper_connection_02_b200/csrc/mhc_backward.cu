@@ -382,87 +382,123 @@ __global__ void __launch_bounds__(256) pre_bwd_param_kernel(const float* __restr
   }
 }
 
-constexpr int kDxCols = 256;  // columns of the flattened row per CTA
-constexpr int kDxTok = 32;    // tokens per sub-tile
-constexpr int kDxSub = 4;     // sub-tiles per CTA (the hc_fn slice is loaded once)
+// 16-byte and 4-byte asynchronous copies global -> shared for the contraction kernels' staging.
+__device__ __forceinline__ void bw_cp16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void bw_cp_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void bw_cp_wait() {  // all but the N newest groups have landed
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
-// d_R = d_raw . hc_fn^T + 2 R d_ss + pre_i d_y, tile of kDxCols columns x kDxSub*kDxTok tokens.
-// Thread: 8-column chunk kc = tid % 32, tokens tk + 8 j (tk = tid / 32, j < 4) of a sub-tile.
-// Requires H % 8 == 0 and 16-byte aligned R, d_R, d_y.
-__global__ void __launch_bounds__(256) pre_bwd_dx_kernel(
+constexpr int kDxThreads = 128;
+constexpr int kDxCols = 4 * kDxThreads;  // columns of the flattened row per CTA
+constexpr int kDxTok = 16;               // tokens per staged step (two buffers)
+constexpr int kDxSmem = 2 * kDxTok * (2 * kDxCols * 2 + 32 * 4);  // R, d_y tiles + records
+constexpr int kDxSlotsPerSm = 3;  // resident CTAs per SM (shared memory) the chunking aims at
+
+// d_R = d_raw . hc_fn^T + 2 R d_ss + pre_i d_y over a slice of kDxCols columns and a chunk of
+// tokens. A thread holds hc_fn's 24 weights of its 4 columns in registers and runs through the
+// chunk's tokens; each step's R and d_y tiles [kDxTok][kDxCols] and the tokens' records (d_raw,
+// d_ss, pre) are staged in shared memory by asynchronous copies one step ahead. Per element the
+// arithmetic is acc = sum_j d_raw[j] w[j] in j order from 0, then fma(pre_i, dy, fma(2 d_ss, R,
+// acc)), rounded once. Requires H % 8 == 0 and 16-byte aligned R, d_R, d_y.
+__global__ void __launch_bounds__(kDxThreads) pre_bwd_dx_kernel(
     const uint16_t* __restrict__ R, const uint16_t* __restrict__ dy,
     const float* __restrict__ W, const float* __restrict__ brec, uint16_t* __restrict__ dR,
-    int64_t T, int64_t H) {
-  __shared__ __align__(16) float ws[kMix][kDxCols];   // hc_fn slice, transposed: [j][k]
-  __shared__ float tokv[kDxTok][32];                  // d_raw[24], d_ss, pre[4]
+    int64_t T, int64_t H, int64_t tchunk) {
+  extern __shared__ __align__(16) uint8_t dx_smem[];
+  uint16_t* xs = reinterpret_cast<uint16_t*>(dx_smem);      // [2][kDxTok][kDxCols]
+  uint16_t* gs = xs + 2 * kDxTok * kDxCols;                 // [2][kDxTok][kDxCols]
+  float* tv = reinterpret_cast<float*>(gs + 2 * kDxTok * kDxCols);  // [2][kDxTok][32]
   const int64_t K = 4 * H;
   const int64_t k0 = static_cast<int64_t>(blockIdx.x) * kDxCols;
   const int tid = threadIdx.x;
-  const int kc = tid & 31, tk = tid >> 5;
+  const int64_t kb = k0 + 4 * tid;  // this thread's 4 columns (K % 4 == 0)
+  const bool kvalid = kb < K;
+  const int64_t si = kvalid ? kb / H : 0;
+  const int64_t tb = static_cast<int64_t>(blockIdx.y) * tchunk;
+  const int64_t te = min(T, tb + tchunk);
   pdl_wait();
   pdl_trigger();
-  for (int e = tid; e < kDxCols * kMix; e += 256) {
-    const int kk = e / kMix, j = e - kk * kMix;
-    ws[j][kk] = k0 + kk < K ? __ldg(W + (k0 + kk) * kMix + j) : 0.f;
-  }
-  const int64_t kb = k0 + kc * 8;  // this thread's 8 columns
-  const bool kvalid = kb < K;
-  const int64_t si = kvalid ? kb / H : 0;  // stream
-  const int64_t hh = kb - si * H;
-  for (int sub = 0; sub < kDxSub; ++sub) {
-    const int64_t t0 = (static_cast<int64_t>(blockIdx.y) * kDxSub + sub) * kDxTok;
-    if (t0 >= T) break;
-    __syncthreads();  // ws ready / previous sub-tile's tokv reads done
-    for (int e = tid; e < kDxTok * 29; e += 256) {
-      const int tl = e / 29, v = e - tl * 29;
-      tokv[tl][v] = t0 + tl < T ? brec[(t0 + tl) * kBrec + v] : 0.f;
-    }
-    __syncthreads();
-    // This thread's residual and d_y chunks first: their loads overlap the contraction below.
-    uint4 xr[4], gr[4];
+  float w[4][kMix];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int64_t t = t0 + tk + 8 * j;
-      const bool ok = kvalid && t < T;
-      xr[j] = ok ? ld_stream_ro(R + t * K + kb) : make_uint4(0u, 0u, 0u, 0u);
-      gr[j] = (ok && dy) ? ld_stream_ro(dy + t * H + hh) : make_uint4(0u, 0u, 0u, 0u);
-    }
-    float acc[4][8];
+  for (int c = 0; c < 4; ++c)
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
-#pragma unroll 4
-    for (int jj = 0; jj < kMix; ++jj) {
-      const float4 w0 = *reinterpret_cast<const float4*>(&ws[jj][kc * 8]);
-      const float4 w1 = *reinterpret_cast<const float4*>(&ws[jj][kc * 8 + 4]);
-      const float w8[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float d = tokv[tk + 8 * j][jj];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[j][e] = fmaf(d, w8[e], acc[j][e]);
+    for (int j = 0; j < kMix; ++j) w[c][j] = kvalid ? __ldg(W + (kb + c) * kMix + j) : 0.f;
+
+  const int nsteps = static_cast<int>((te - tb + kDxTok - 1) / kDxTok);
+  auto stage = [&](int step, int b) {
+    const int64_t t0 = tb + static_cast<int64_t>(step) * kDxTok;
+    for (int e = tid; e < kDxTok * (kDxCols / 8); e += kDxThreads) {
+      const int tl = e / (kDxCols / 8), c8 = e - tl * (kDxCols / 8);
+      const int64_t t = t0 + tl, k = k0 + c8 * 8;
+      if (t < te && k < K) {
+        bw_cp16(xs + (b * kDxTok + tl) * kDxCols + c8 * 8, R + t * K + k);
+        if (dy) {
+          const int64_t i = k / H;
+          bw_cp16(gs + (b * kDxTok + tl) * kDxCols + c8 * 8, dy + t * H + (k - i * H));
+        }
       }
     }
-    if (!kvalid) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int tl = tk + 8 * j;
+    for (int e = tid; e < kDxTok * 8; e += kDxThreads) {  // record floats 0..31 of each token
+      const int tl = e >> 3, q = e & 7;
       const int64_t t = t0 + tl;
-      if (t >= T) continue;
-      const uint4 xv = xr[j], gv = gr[j];
-      const float dss2 = 2.0f * tokv[tl][24];
-      const float pi = tokv[tl][25 + si];
-      uint32_t o[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint32_t xw = (&xv.x)[q], gw = (&gv.x)[q];
-        const float lo = fmaf(pi, bf16_lo(gw), fmaf(dss2, bf16_lo(xw), acc[j][2 * q]));
-        const float hi = fmaf(pi, bf16_hi(gw), fmaf(dss2, bf16_hi(xw), acc[j][2 * q + 1]));
-        o[q] = pack_bf16x2(lo, hi);
-      }
-      st_plain(dR + t * K + kb, make_uint4(o[0], o[1], o[2], o[3]));
+      if (t < te) bw_cp16(tv + (b * kDxTok + tl) * 32 + q * 4, brec + t * kBrec + q * 4);
     }
+    bw_cp_commit();
+  };
+  if (nsteps > 0) stage(0, 0);
+  for (int step = 0; step < nsteps; ++step) {
+    const int b = step & 1;
+    if (step + 1 < nsteps) {
+      stage(step + 1, b ^ 1);
+      bw_cp_wait<1>();
+    } else {
+      bw_cp_wait<0>();
+    }
+    __syncthreads();  // step's tiles visible to every thread
+    const int64_t t0 = tb + static_cast<int64_t>(step) * kDxTok;
+    const int n = static_cast<int>(min(static_cast<int64_t>(kDxTok), te - t0));
+    if (kvalid) {
+      for (int tl = 0; tl < n; ++tl) {
+        const float* o = tv + (b * kDxTok + tl) * 32;
+        float d[kMix];
+#pragma unroll
+        for (int q = 0; q < kMix / 4; ++q) {
+          const float4 v = *reinterpret_cast<const float4*>(o + 4 * q);
+          d[4 * q] = v.x;
+          d[4 * q + 1] = v.y;
+          d[4 * q + 2] = v.z;
+          d[4 * q + 3] = v.w;
+        }
+        const float dss2 = 2.0f * o[24];
+        const float pi = o[25 + si];
+        const int off = (b * kDxTok + tl) * kDxCols + 4 * tid;
+        const uint2 xv = *reinterpret_cast<const uint2*>(xs + off);
+        const uint2 gv = dy ? *reinterpret_cast<const uint2*>(gs + off) : make_uint2(0u, 0u);
+        float acc[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          acc[c] = 0.f;
+#pragma unroll
+          for (int j = 0; j < kMix; ++j) acc[c] = fmaf(d[j], w[c][j], acc[c]);
+        }
+        const float x0 = bf16_lo(xv.x), x1 = bf16_hi(xv.x), x2 = bf16_lo(xv.y), x3 = bf16_hi(xv.y);
+        const float g0 = bf16_lo(gv.x), g1 = bf16_hi(gv.x), g2 = bf16_lo(gv.y), g3 = bf16_hi(gv.y);
+        const uint32_t o0 = pack_bf16x2(fmaf(pi, g0, fmaf(dss2, x0, acc[0])),
+                                        fmaf(pi, g1, fmaf(dss2, x1, acc[1])));
+        const uint32_t o1 = pack_bf16x2(fmaf(pi, g2, fmaf(dss2, x2, acc[2])),
+                                        fmaf(pi, g3, fmaf(dss2, x3, acc[3])));
+        *reinterpret_cast<uint2*>(dR + (t0 + tl) * K + kb) = make_uint2(o0, o1);
+      }
+    }
+    __syncthreads();  // buffer b is restaged two steps on
   }
 }
 
@@ -488,65 +524,98 @@ __global__ void __launch_bounds__(256) pre_bwd_dx_scalar_kernel(
   }
 }
 
-constexpr int kDwCols = 256;  // columns of hc_fn per CTA
-constexpr int kDwTok = 32;    // tokens staged per step
+constexpr int kDwThreads = 128;
+constexpr int kDwCols = 4 * kDwThreads;  // columns of hc_fn per CTA
+constexpr int kDwTok = 16;               // tokens per staged step (two buffers)
+constexpr int kDwSlotsPerSm = 4;         // resident CTAs per SM the chunking aims at
 
-// Partial d_hc_fn over a token chunk: dwp[chunk][k][j] = sum_{t in chunk} R_flat[t][k] d_raw[t][j]
-// (tokens in increasing order). Thread: columns 4 kq .. 4 kq + 3 (kq = tid % 64) x logits
-// 6 g .. 6 g + 5 (g = tid / 64): 24 accumulators, fed per token by one 16-byte and three 8-byte
-// shared-memory loads.
-__global__ void __launch_bounds__(256) pre_bwd_dw_kernel(const uint16_t* __restrict__ R,
-                                                         const float* __restrict__ brec,
-                                                         float* __restrict__ dwp, int64_t T,
-                                                         int64_t H, int64_t tchunk) {
-  __shared__ __align__(16) float xs[kDwTok][kDwCols];
-  __shared__ __align__(16) float ds[kDwTok][kMix];
+// Partial d_hc_fn over a token chunk: dwp[chunk][k][j] = sum_{t in chunk} R_flat[t][k] d_raw[t][j],
+// tokens in increasing order. A thread owns 4 columns x all 24 logits (96 accumulators); per
+// token it reads its 4 bf16 values and the token's d_raw (a broadcast) from shared memory, where
+// each step's R tile [kDwTok][kDwCols] (bf16, as stored) and d_raw rows are staged one step ahead
+// (asynchronous 16-byte copies when kVec: H % 8 == 0 and R 16-byte aligned).
+template <bool kVec>
+__global__ void __launch_bounds__(kDwThreads, kDwSlotsPerSm)
+    pre_bwd_dw_kernel(const uint16_t* __restrict__ R, const float* __restrict__ brec,
+                      float* __restrict__ dwp, int64_t T, int64_t H, int64_t tchunk) {
+  __shared__ __align__(16) uint16_t xs[2][kDwTok][kDwCols];
+  __shared__ __align__(16) float ds[2][kDwTok][kMix];
   const int64_t K = 4 * H;
   const int64_t k0 = static_cast<int64_t>(blockIdx.x) * kDwCols;
   const int64_t tb = static_cast<int64_t>(blockIdx.y) * tchunk;
   const int64_t te = min(T, tb + tchunk);
   const int tid = threadIdx.x;
-  const int kq = tid & 63, jg = tid >> 6;
+  const int64_t kb = k0 + 4 * tid;
   pdl_wait();
   pdl_trigger();
-  float acc[4][6];
+  float acc[4][kMix];
 #pragma unroll
   for (int c = 0; c < 4; ++c)
 #pragma unroll
-    for (int j = 0; j < 6; ++j) acc[c][j] = 0.f;
-  for (int64_t t0 = tb; t0 < te; t0 += kDwTok) {
+    for (int j = 0; j < kMix; ++j) acc[c][j] = 0.f;
+
+  const int nsteps = static_cast<int>((te - tb + kDwTok - 1) / kDwTok);
+  auto stage = [&](int step, int b) {
+    const int64_t t0 = tb + static_cast<int64_t>(step) * kDwTok;
+    if (kVec) {
+      for (int e = tid; e < kDwTok * (kDwCols / 8); e += kDwThreads) {
+        const int tl = e / (kDwCols / 8), c8 = e - tl * (kDwCols / 8);
+        const int64_t t = t0 + tl, k = k0 + c8 * 8;
+        if (t < te && k < K) bw_cp16(&xs[b][tl][c8 * 8], R + t * K + k);
+      }
+    } else {
+      for (int e = tid; e < kDwTok * kDwCols; e += kDwThreads) {
+        const int tl = e / kDwCols, c = e - tl * kDwCols;
+        const int64_t t = t0 + tl, k = k0 + c;
+        if (t < te && k < K) xs[b][tl][c] = R[t * K + k];
+      }
+    }
+    for (int e = tid; e < kDwTok * (kMix / 4); e += kDwThreads) {  // d_raw: 6 x 16 bytes a token
+      const int tl = e / (kMix / 4), q = e - tl * (kMix / 4);
+      const int64_t t = t0 + tl;
+      if (t < te) bw_cp16(&ds[b][tl][q * 4], brec + t * kBrec + q * 4);
+    }
+    bw_cp_commit();
+  };
+  if (nsteps > 0) stage(0, 0);
+  for (int step = 0; step < nsteps; ++step) {
+    const int b = step & 1;
+    if (step + 1 < nsteps) {
+      stage(step + 1, b ^ 1);
+      bw_cp_wait<1>();
+    } else {
+      bw_cp_wait<0>();
+    }
     __syncthreads();
-    for (int e = tid; e < kDwTok * kDwCols; e += 256) {
-      const int tl = e / kDwCols, c = e - tl * kDwCols;
-      const int64_t t = t0 + tl, k = k0 + c;
-      xs[tl][c] = (t < te && k < K) ? bf16_to_f32(R[t * K + k]) : 0.f;
-    }
-    for (int e = tid; e < kDwTok * kMix; e += 256) {
-      const int tl = e / kMix, j = e - tl * kMix;
-      ds[tl][j] = t0 + tl < te ? brec[(t0 + tl) * kBrec + j] : 0.f;
-    }
-    __syncthreads();
-#pragma unroll 2
-    for (int tl = 0; tl < kDwTok; ++tl) {
-      const float4 x4 = *reinterpret_cast<const float4*>(&xs[tl][4 * kq]);
-      const float2 d01 = *reinterpret_cast<const float2*>(&ds[tl][6 * jg]);
-      const float2 d23 = *reinterpret_cast<const float2*>(&ds[tl][6 * jg + 2]);
-      const float2 d45 = *reinterpret_cast<const float2*>(&ds[tl][6 * jg + 4]);
-      const float xv[4] = {x4.x, x4.y, x4.z, x4.w};
-      const float dv[6] = {d01.x, d01.y, d23.x, d23.y, d45.x, d45.y};
+    const int64_t t0 = tb + static_cast<int64_t>(step) * kDwTok;
+    const int n = static_cast<int>(min(static_cast<int64_t>(kDwTok), te - t0));
+    if (kb < K) {
+      for (int tl = 0; tl < n; ++tl) {
+        const uint2 xv = *reinterpret_cast<const uint2*>(&xs[b][tl][4 * tid]);
+        const float xf[4] = {bf16_lo(xv.x), bf16_hi(xv.x), bf16_lo(xv.y), bf16_hi(xv.y)};
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+        for (int q = 0; q < kMix / 4; ++q) {
+          const float4 d4 = *reinterpret_cast<const float4*>(&ds[b][tl][4 * q]);
 #pragma unroll
-        for (int j = 0; j < 6; ++j) acc[c][j] = fmaf(xv[c], dv[j], acc[c][j]);
+          for (int c = 0; c < 4; ++c) {
+            acc[c][4 * q] = fmaf(xf[c], d4.x, acc[c][4 * q]);
+            acc[c][4 * q + 1] = fmaf(xf[c], d4.y, acc[c][4 * q + 1]);
+            acc[c][4 * q + 2] = fmaf(xf[c], d4.z, acc[c][4 * q + 2]);
+            acc[c][4 * q + 3] = fmaf(xf[c], d4.w, acc[c][4 * q + 3]);
+          }
+        }
+      }
     }
+    __syncthreads();  // buffer b is restaged two steps on
   }
+  if (kb < K) {
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const int64_t k = k0 + 4 * kq + c;
-    if (k < K) {
-      float* o = dwp + (static_cast<int64_t>(blockIdx.y) * K + k) * kMix + 6 * jg;
+    for (int c = 0; c < 4; ++c) {
+      float4* o = reinterpret_cast<float4*>(dwp + (static_cast<int64_t>(blockIdx.y) * K + kb + c) *
+                                                      kMix);
 #pragma unroll
-      for (int j = 0; j < 6; ++j) o[j] = acc[c][j];
+      for (int q = 0; q < kMix / 4; ++q)
+        o[q] = make_float4(acc[c][4 * q], acc[c][4 * q + 1], acc[c][4 * q + 2], acc[c][4 * q + 3]);
     }
   }
 }
@@ -578,9 +647,10 @@ static BwPlan bw_plan(int64_t T, int64_t H) {
   p.proj = up(a > b ? a : b);
   p.dpt = up(static_cast<size_t>(T) * 16);
   p.brec = up(static_cast<size_t>(T) * kBrec * 4);
-  // Token chunks of d_hc_fn partials: enough CTAs (4H/256 x chunks) for about sixteen per SM.
+  // Token chunks of d_hc_fn partials: column slices x chunks fill the SMs' CTA slots in one
+  // wave (the same chunks serve d_R).
   const int64_t kcols = (4 * H + kDwCols - 1) / kDwCols;
-  int64_t nchunk = (16 * 148 + kcols - 1) / kcols;
+  int64_t nchunk = (kDwSlotsPerSm * 148) / kcols;
   if (nchunk < 1) nchunk = 1;
   if (nchunk > (T + kDwTok - 1) / kDwTok) nchunk = (T + kDwTok - 1) / kDwTok;
   if (nchunk < 1) nchunk = 1;
@@ -637,12 +707,26 @@ int launch_pre_backward(const PreBwdArgs& a, cudaStream_t s) {
   e = launch_pdl(pre_bwd_param_kernel, dim3(3 + kMix), dim3(256), 0, s,
                  static_cast<const float*>(brec), a.dscale, a.dbase, a.T);
   if (e != cudaSuccess) return -4;
-  // 5. d_R.
+  // 5. d_R: column slices x token chunks, one wave of kDxSlotsPerSm CTAs per SM.
   if (vec) {
-    const dim3 g(static_cast<unsigned>((K + kDxCols - 1) / kDxCols),
-                 static_cast<unsigned>((a.T + kDxSub * kDxTok - 1) / (kDxSub * kDxTok)));
-    e = launch_pdl(pre_bwd_dx_kernel, g, dim3(256), 0, s, a.R, a.dy, a.hc_fn,
-                   static_cast<const float*>(brec), a.dR, a.T, a.H);
+    static bool attr_set[64] = {};
+    const int dev = current_device();
+    if (dev < 0) return -4;
+    if (!attr_set[dev]) {
+      if (cudaFuncSetAttribute(pre_bwd_dx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kDxSmem) != cudaSuccess)
+        return -4;
+      attr_set[dev] = true;
+    }
+    const int64_t xcols = (K + kDxCols - 1) / kDxCols;
+    int64_t xch = (kDxSlotsPerSm * static_cast<int64_t>(device_sm_count())) / xcols;
+    if (xch < 1) xch = 1;
+    if (xch > (a.T + kDxTok - 1) / kDxTok) xch = (a.T + kDxTok - 1) / kDxTok;
+    const int64_t xtchunk = ((a.T + xch - 1) / xch + kDxTok - 1) / kDxTok * kDxTok;
+    const dim3 g(static_cast<unsigned>(xcols),
+                 static_cast<unsigned>((a.T + xtchunk - 1) / xtchunk));
+    e = launch_pdl(pre_bwd_dx_kernel, g, dim3(kDxThreads), static_cast<size_t>(kDxSmem), s, a.R,
+                   a.dy, a.hc_fn, static_cast<const float*>(brec), a.dR, a.T, a.H, xtchunk);
   } else {
     int64_t nb = (a.T * K + 255) / 256;
     if (nb > 148 * 16) nb = 148 * 16;
@@ -653,8 +737,11 @@ int launch_pre_backward(const PreBwdArgs& a, cudaStream_t s) {
   // 6. d_hc_fn.
   const dim3 gw(static_cast<unsigned>((K + kDwCols - 1) / kDwCols),
                 static_cast<unsigned>(plan.nchunk));
-  e = launch_pdl(pre_bwd_dw_kernel, gw, dim3(256), 0, s, a.R, static_cast<const float*>(brec),
-                 dwp, a.T, a.H, plan.tchunk);
+  const bool dwvec = a.H % 8 == 0 && aligned16(a.R);
+  e = dwvec ? launch_pdl(pre_bwd_dw_kernel<true>, gw, dim3(kDwThreads), 0, s, a.R,
+                         static_cast<const float*>(brec), dwp, a.T, a.H, plan.tchunk)
+            : launch_pdl(pre_bwd_dw_kernel<false>, gw, dim3(kDwThreads), 0, s, a.R,
+                         static_cast<const float*>(brec), dwp, a.T, a.H, plan.tchunk);
   if (e != cudaSuccess) return -4;
   int64_t nb = (K * kMix + 255) / 256;
   if (nb > 148 * 8) nb = 148 * 8;
