@@ -252,6 +252,8 @@ __device__ __forceinline__ void sk_round(float (&a)[4], float (&b)[4], float& rs
   }
 }
 
+constexpr int kSkCk = 16;  // Sinkhorn forward checkpoints kept by the reverse pass
+
 // Per token, one lane quad (lane r: pre r, post r, comb row r). Writes the backward record
 // brec[t][64]: [0..23] d_raw, [24] d_ss, [25..28] pre gates, [29..31] the token's terms of
 // d_scale, [32..55] d_l (the token's term of d_base).
@@ -290,7 +292,9 @@ __global__ void __launch_bounds__(256) pre_bwd_coef_kernel(
   const float dl0 = dpt[tt * 4 + r] * sg0 * (1.0f - sg0);
   const float dl1 = (dpost ? dpost[tt * 4 + r] : 0.f) * fp.post_mult * sg1 * (1.0f - sg1);
 
-  // Sinkhorn reverse pass: the state entering round k is recomputed from A0 for each k.
+  // Sinkhorn reverse pass. The forward states are checkpointed every G rounds (at most kSkCk
+  // checkpoints); the state entering round k is recomputed from the checkpoint at or before it,
+  // by the same operations as the forward, so it is the forward's state exactly.
   float a0[4], dA[4];
   const float mx = fmaxf(fmaxf(lc[0], lc[1]), fmaxf(lc[2], lc[3]));
 #pragma unroll
@@ -298,9 +302,22 @@ __global__ void __launch_bounds__(256) pre_bwd_coef_kernel(
     a0[n] = expf(lc[n] - mx);
     dA[n] = dcomb ? dcomb[tt * 16 + 4 * r + n] : 0.f;
   }
-  for (int k = fp.iters - 1; k >= 0; --k) {
+  const int G = (fp.iters + kSkCk - 1) / kSkCk;
+  float ck[kSkCk][4];
+  {
     float a[4] = {a0[0], a0[1], a0[2], a0[3]}, b[4], rs, cs[4];
-    for (int j = 0; j < k; ++j) sk_round(a, b, rs, cs, fp.sinkhorn_eps);
+    for (int k = 0; k < fp.iters; ++k) {
+      if (k % G == 0) {
+#pragma unroll
+        for (int n = 0; n < 4; ++n) ck[k / G][n] = a[n];
+      }
+      sk_round(a, b, rs, cs, fp.sinkhorn_eps);
+    }
+  }
+  for (int k = fp.iters - 1; k >= 0; --k) {
+    const int c = k / G;
+    float a[4] = {ck[c][0], ck[c][1], ck[c][2], ck[c][3]}, b[4], rs, cs[4];
+    for (int j = c * G; j < k; ++j) sk_round(a, b, rs, cs, fp.sinkhorn_eps);
     sk_round(a, b, rs, cs, fp.sinkhorn_eps);  // round k: a is now C
     float dB[4];
 #pragma unroll
