@@ -450,16 +450,24 @@ __global__ void __launch_bounds__(kDxThreads) pre_bwd_dx_kernel(
     for (int j = 0; j < kMix; ++j) w[c][j] = kvalid ? __ldg(W + (kb + c) * kMix + j) : 0.f;
 
   const int nsteps = static_cast<int>((te - tb + kDxTok - 1) / kDxTok);
+  // Staging: this thread always copies 8-column chunk sc of the slice, for tokens sr + 2 u.
+  static_assert(kDxThreads == 2 * (kDxCols / 8), "staging map");
+  const int sc = tid & (kDxCols / 8 - 1), sr = tid / (kDxCols / 8);
+  const int64_t sk = k0 + sc * 8;
+  const bool skv = sk < K;
+  const int64_t sh = skv ? sk - (sk / H) * H : 0;  // d_y column of the chunk
   auto stage = [&](int step, int b) {
     const int64_t t0 = tb + static_cast<int64_t>(step) * kDxTok;
-    for (int e = tid; e < kDxTok * (kDxCols / 8); e += kDxThreads) {
-      const int tl = e / (kDxCols / 8), c8 = e - tl * (kDxCols / 8);
-      const int64_t t = t0 + tl, k = k0 + c8 * 8;
-      if (t < te && k < K) {
-        bw_cp16(xs + (b * kDxTok + tl) * kDxCols + c8 * 8, R + t * K + k);
-        if (dy) {
-          const int64_t i = k / H;
-          bw_cp16(gs + (b * kDxTok + tl) * kDxCols + c8 * 8, dy + t * H + (k - i * H));
+    if (skv) {
+      const uint16_t* rp = R + (t0 + sr) * K + sk;
+      const uint16_t* gp = dy ? dy + (t0 + sr) * H + sh : nullptr;
+      uint16_t* xd = xs + (b * kDxTok + sr) * kDxCols + sc * 8;
+      uint16_t* gd = gs + (b * kDxTok + sr) * kDxCols + sc * 8;
+#pragma unroll
+      for (int u = 0; u < kDxTok / 2; ++u) {
+        if (t0 + sr + 2 * u < te) {
+          bw_cp16(xd + 2 * u * kDxCols, rp + 2 * u * K);
+          if (gp) bw_cp16(gd + 2 * u * kDxCols, gp + 2 * u * H);
         }
       }
     }
@@ -574,11 +582,14 @@ __global__ void __launch_bounds__(kDwThreads, kDwSlotsPerSm)
   const int nsteps = static_cast<int>((te - tb + kDwTok - 1) / kDwTok);
   auto stage = [&](int step, int b) {
     const int64_t t0 = tb + static_cast<int64_t>(step) * kDwTok;
-    if (kVec) {
-      for (int e = tid; e < kDwTok * (kDwCols / 8); e += kDwThreads) {
-        const int tl = e / (kDwCols / 8), c8 = e - tl * (kDwCols / 8);
-        const int64_t t = t0 + tl, k = k0 + c8 * 8;
-        if (t < te && k < K) bw_cp16(&xs[b][tl][c8 * 8], R + t * K + k);
+    if (kVec) {  // this thread copies 8-column chunk sc for tokens sr + 2 u
+      static_assert(kDwThreads == 2 * (kDwCols / 8), "staging map");
+      const int sc = tid & (kDwCols / 8 - 1), sr = tid / (kDwCols / 8);
+      if (k0 + sc * 8 < K) {
+        const uint16_t* rp = R + (t0 + sr) * K + k0 + sc * 8;
+#pragma unroll
+        for (int u = 0; u < kDwTok / 2; ++u)
+          if (t0 + sr + 2 * u < te) bw_cp16(&xs[b][sr + 2 * u][sc * 8], rp + 2 * u * K);
       }
     } else {
       for (int e = tid; e < kDwTok * kDwCols; e += kDwThreads) {
