@@ -415,9 +415,9 @@ __device__ __forceinline__ void bw_cp_wait() {  // all but the N newest groups h
 
 constexpr int kDxThreads = 128;
 constexpr int kDxCols = 4 * kDxThreads;  // columns of the flattened row per CTA
-constexpr int kDxTok = 16;               // tokens per staged step (two buffers)
+constexpr int kDxTok = 12;               // tokens per staged step (two buffers)
 constexpr int kDxSmem = 2 * kDxTok * (2 * kDxCols * 2 + 32 * 4);  // R, d_y tiles + records
-constexpr int kDxSlotsPerSm = 3;  // resident CTAs per SM (shared memory) the chunking aims at
+constexpr int kDxSlotsPerSm = 4;  // resident CTAs per SM (shared memory) the chunking aims at
 
 // d_R = d_raw . hc_fn^T + 2 R d_ss + pre_i d_y over a slice of kDxCols columns and a chunk of
 // tokens. A thread holds hc_fn's 24 weights of its 4 columns in registers and runs through the
@@ -425,7 +425,7 @@ constexpr int kDxSlotsPerSm = 3;  // resident CTAs per SM (shared memory) the ch
 // d_ss, pre) are staged in shared memory by asynchronous copies one step ahead. Per element the
 // arithmetic is acc = sum_j d_raw[j] w[j] in j order from 0, then fma(pre_i, dy, fma(2 d_ss, R,
 // acc)), rounded once. Requires H % 8 == 0 and 16-byte aligned R, d_R, d_y.
-__global__ void __launch_bounds__(kDxThreads) pre_bwd_dx_kernel(
+__global__ void __launch_bounds__(kDxThreads, kDxSlotsPerSm) pre_bwd_dx_kernel(
     const uint16_t* __restrict__ R, const uint16_t* __restrict__ dy,
     const float* __restrict__ W, const float* __restrict__ brec, uint16_t* __restrict__ dR,
     int64_t T, int64_t H, int64_t tchunk) {
