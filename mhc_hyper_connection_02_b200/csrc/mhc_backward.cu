@@ -10,12 +10,13 @@
 // pre-map   (upstream d_y, d_pre, d_post, d_comb; any may be absent)
 //   1. the projection is recomputed by the forward's own kernels (records of raw and ss);
 //   2. d_pre += sum_h d_y R_i (one CTA per token);
-//   3. per token (lane quad): rstd, logits, gates, the Sinkhorn states (recomputed round by round)
+//   3. per token (lane quad): rstd, logits, gates, the Sinkhorn forward (states checkpointed)
 //      and the reverse pass -> d_raw, d_ss, the gates, and the per-token terms of d_scale, d_base;
 //   4. d_scale, d_base: fixed-order sums over tokens;
-//   5. d_R = d_raw . hc_fn^T + 2 R d_ss + pre_i d_y (token x column tiles, hc_fn slice in shared
-//      memory, fp32 on CUDA cores);
-//   6. d_hc_fn = R_flat^T d_raw (a column slice of R per CTA, tokens summed in order).
+//   5. d_R = d_raw . hc_fn^T + 2 R d_ss + pre_i d_y (column slice x token chunk per CTA, a
+//      thread's hc_fn weights in registers, fp32 on CUDA cores);
+//   6. d_hc_fn = R_flat^T d_raw (column slice x token chunk per CTA, tokens summed in order, then
+//      the chunks in order).
 #include "mhc_device.cuh"
 #include "mhc_internal.h"
 
