@@ -141,3 +141,92 @@ def test_backward_errors():
         mhc.pre_backward(R, dev_f32(w.hc_fn), dev_f32(w.hc_scale), dev_f32(w.hc_base),
                          workspace=small)
     assert e.value.status == mhc.MHC_ERR_WORKSPACE_TOO_SMALL
+
+
+def _sample_rows(T, seed):
+    rng = np.random.default_rng(seed)
+    return np.unique(np.concatenate([rng.choice(T, 24, replace=False), [0, 127, 128, T - 1]]))
+
+
+@pytest.mark.slow
+def test_post_backward_large_sampled():
+    """Full size (T=8192, H=7168), the launch bench.py times; every output is per token, so
+    sampled tokens are checked against the oracle run on those tokens alone."""
+    w = inputs.large()
+    post, comb = post_coefficients(w)
+    g = np.random.default_rng(101)
+    d_out = _bits(g.standard_normal((w.T, 4, w.H), dtype=np.float32))
+    dx, dR, dp, dc = mhc.post_backward(dev_bf16(d_out), dev_bf16(w.x), dev_bf16(w.R),
+                                       dev_f32(post), dev_f32(comb))
+    torch.cuda.synchronize()
+    rows = _sample_rows(w.T, 5)
+    rx, rR, rp, rc = backward.post_backward(d_out[rows], w.x[rows], w.R[rows], post[rows],
+                                            comb[rows])
+    G = np.abs(bf16_bits_to_f64(d_out[rows]))
+    bx = 5 * U32 * np.einsum("tn,tnh->th", np.abs(post[rows].astype(np.float64)), G)
+    bR = 5 * U32 * np.einsum("ton,tnh->toh", np.abs(comb[rows].astype(np.float64)), G)
+    sel = torch.as_tensor(rows, device="cuda")
+    f1 = check_bf16(host_bits(dx[sel]), rx, oracle.round_bf16(rx), bx)
+    f2 = check_bf16(host_bits(dR[sel]), rR, oracle.round_bf16(rR), bR)
+    print(f"[post_backward large sampled] d_x fail={f1[0]} d_R fail={f2[0]}")
+    assert f1[0] == 0 and f2[0] == 0
+    X = np.abs(bf16_bits_to_f64(w.x[rows]))
+    Rb = np.abs(bf16_bits_to_f64(w.R[rows]))
+    _check_sum(dp[sel].cpu().numpy(), rp, np.einsum("th,tnh->tn", X, G), 1e-5, "d_post")
+    _check_sum(dc[sel].cpu().numpy(), rc, np.einsum("toh,tnh->ton", Rb, G), 1e-5, "d_comb")
+
+
+@pytest.mark.slow
+def test_pre_backward_large_sampled():
+    """Full size (T=8192, H=7168), the launch bench.py times. d_R is per token: sampled tokens
+    against the oracle on those tokens. d_hc_fn, d_scale and d_base are sums over all tokens: the
+    oracle runs on chunks of 1024 tokens and its fp64 chunk sums are added."""
+    w = inputs.large()
+    g = np.random.default_rng(202)
+    d_y = _bits(g.standard_normal((w.T, w.H), dtype=np.float32))
+    d_pre = g.standard_normal((w.T, 4)).astype(np.float32)
+    d_post = g.standard_normal((w.T, 4)).astype(np.float32)
+    d_comb = g.standard_normal((w.T, 4, 4)).astype(np.float32)
+    prm = mhc.make_params(iters=w.iters, eps=w.eps, rms_eps=w.rms_eps, pre_eps=w.pre_eps,
+                          post_mult=w.post_mult)
+    dR, dW, ds, db = mhc.pre_backward(
+        dev_bf16(w.R), dev_f32(w.hc_fn), dev_f32(w.hc_scale), dev_f32(w.hc_base),
+        d_y=dev_bf16(d_y), d_pre=dev_f32(d_pre), d_post=dev_f32(d_post), d_comb=dev_f32(d_comb),
+        params=prm)
+    torch.cuda.synchronize()
+    assert mhc.device_status() == 0
+    kw = dict(rms_eps=w.rms_eps, pre_eps=w.pre_eps, post_mult=w.post_mult, iters=w.iters,
+              eps=w.eps, parts=True)
+    Wa = np.abs(w.hc_fn.astype(np.float64))
+    grp = np.array([0] * 4 + [1] * 4 + [2] * 16)
+    rW = np.zeros((4 * w.H, 24))
+    tW = np.zeros((4 * w.H, 24))
+    rs = np.zeros(3)
+    ts = np.zeros(3)
+    rb = np.zeros(24)
+    tb = np.zeros(24)
+    for c0 in range(0, w.T, 1024):
+        sl = slice(c0, min(w.T, c0 + 1024))
+        _, cW, cs, cb, pt = backward.pre_backward(d_y[sl], d_pre[sl], d_post[sl], d_comb[sl],
+                                                  w.R[sl], w.hc_fn, w.hc_scale, w.hc_base, **kw)
+        rW += cW
+        rs += cs
+        rb += cb
+        tW += np.abs(pt["X"]).T @ np.abs(pt["d_raw"])
+        ts += np.array([(np.abs(pt["dl"][:, grp == k] * pt["m"][:, grp == k])).sum()
+                        for k in range(3)])
+        tb += np.abs(pt["dl"]).sum(0)
+    _check_sum(dW.cpu().numpy(), rW, tW, 1e-4, "d_hc_fn")
+    _check_sum(ds.cpu().numpy(), rs, ts, 1e-4, "d_scale")
+    _check_sum(db.cpu().numpy(), rb, tb, 1e-4, "d_base")
+    rows = _sample_rows(w.T, 6)
+    rR, _, _, _, pt = backward.pre_backward(d_y[rows], d_pre[rows], d_post[rows], d_comb[rows],
+                                            w.R[rows], w.hc_fn, w.hc_scale, w.hc_base, **kw)
+    n = len(rows)
+    X = np.abs(pt["X"])
+    terms = (np.abs(pt["d_raw"]) @ Wa.T + 2 * X * np.abs(pt["d_ss"])[:, None]).reshape(n, 4, w.H)
+    terms = terms + np.abs(pt["pre"])[:, :, None] * np.abs(bf16_bits_to_f64(d_y[rows]))[:, None, :]
+    sel = torch.as_tensor(rows, device="cuda")
+    f = check_bf16(host_bits(dR[sel]), rR, oracle.round_bf16(rR), (1e-4 + 30 * U32) * terms)
+    print(f"[pre_backward large sampled] d_R fail={f[0]} derived-bound={f[1]} worst/tol={f[2]:.3f}")
+    assert f[0] == 0
