@@ -120,13 +120,19 @@ def oracle_sample(w, n_tokens):
     return n_tokens / dt, dt, oracle.threads()
 
 
-def cpu_baseline(w, budget_s=12.0):
-    """Bounded sample: calibrate on a few tokens, then time about budget_s seconds of oracle work."""
+def cpu_baseline(w, budget_s=12.0, max_passes=50):
+    """Bounded sample: calibrate on a few tokens, then time about budget_s seconds of oracle work
+    (the first n tokens, n <= T; when one pass over them takes less than budget_s, repeated
+    passes until budget_s has elapsed)."""
     rate, _, _ = oracle_sample(w, 16)
     n = int(max(16, min(w.T, rate * budget_s)))
-    rate, dt, cores = oracle_sample(w, n)
-    return {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"first {n} of {w.T} tokens (pre+post), {dt:.1f} s"}
+    tot, passes, cores = 0.0, 0, 1
+    while passes < max_passes and (passes == 0 or tot < budget_s):
+        _, dt, cores = oracle_sample(w, n)
+        tot += dt
+        passes += 1
+    return {"value": n * passes / tot, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"first {n} of {w.T} tokens (pre+post), {passes} pass(es), {tot:.1f} s"}
 
 
 def dist_env():
