@@ -18,10 +18,11 @@
  *       §2.3 empty input returns without a launch; §3.1-3.2 pre-map parameters and defaults
  *       (rms_eps, sinkhorn eps, sinkhorn_repeat >= 1, eps > 0); §3.4 kernel phases (sum of
  *       squares, rstd, sigmoid gates, softmax with row-max shift, row -> column Sinkhorn rounds,
- *       vec8 aggregate); §4 RMS denominator 4*H; §5.2 test reference math.
- *   rwkv-ops 0.6.1 "rwkv_ops/mhc_kernel/jax_kernel/mhu_jax.py": docstrings of sinkhorn_knopp
- *       (eps guards the division), stream_aggregate (fp32 accumulate, cast back), mhc_pre_op
- *       (H_pre = sigmoid, H_post = 2 * sigmoid).
+ *       vec8 aggregate); §4 RMS denominator 4*H; §5.2 test reference math (the Sinkhorn starts
+ *       from the row softmax plus eps and divides by plain row and column sums).
+ *   rwkv-ops 0.6.1 "rwkv_ops/mhc_kernel/jax_kernel/mhu_jax.py": docstrings of
+ *       stream_aggregate (fp32 accumulate, cast back) and mhc_pre_op (H_pre = sigmoid,
+ *       H_post = 2 * sigmoid).
  *   "metrale_model_layers/layers/ops/hyper_connection_dispatch.rs": hc_pre_site / hc_post_site
  *       argument lists (device pointers, token count, hidden size, stream; out may alias residual).
  *   "metrale_model_arch/glm5next_mhc.rs": glm_hc_pre (refuse to launch past the scratch
@@ -81,7 +82,7 @@ enum mhc_status {
  * H_post = 2 * sigmoid; FlashInfer's defaults 1e-6 and 1.0 are reachable by setting them). */
 typedef struct {
     int sinkhorn_iters; /* >= 1: rounds of (row normalise, column normalise) */
-    float sinkhorn_eps; /* > 0: added to every row / column sum before dividing by it */
+    float sinkhorn_eps; /* > 0: added to every entry of the row softmax before the rounds */
     float rms_eps;      /* > 0: rstd = 1 / sqrt(sum(R^2) / (4H) + rms_eps) */
     float pre_eps;      /* >= 0: added to each pre gate */
     float post_mult;    /* finite: post = post_mult * sigmoid(l[4:8]) */
@@ -139,11 +140,12 @@ MHC_API int mhc_post(const uint16_t* x, const uint16_t* R, const float* post, co
 
 /*
  * mhc_sinkhorn -- the Sinkhorn step on its own. "FlashInfer mHC module deep dive" §3.4 (softmax
- * with row-max shift, then row -> column rounds) and §5.2; rwkv-ops sinkhorn_knopp.
+ * with row-max shift, then row -> column rounds) and §5.2 (its test reference: softmax + eps,
+ * then plain row -> column rounds).
  *
  *   logits [T][4][4] fp32   pre-exp logits, [old][new]
- *   comb   [T][4][4] fp32   out: A = exp(l - rowmax); `iters` times { rows /= (rowsum + eps);
- *                           columns /= (colsum + eps) }; may be equal to logits (in place)
+ *   comb   [T][4][4] fp32   out: A = softmax(l, each row) + eps; `iters` times { rows /= rowsum;
+ *                           columns /= colsum }; may be equal to logits (in place)
  *   H_unused               ignored (kept so every entry takes T and H)
  *
  * Errors: MHC_ERR_INVALID_ARG (null array, T < 0, iters < 1, eps <= 0 or not finite);
@@ -296,8 +298,8 @@ MHC_API int mhc_post_project(const uint16_t* x, const uint16_t* R, const float* 
  *   forward's inputs R, hc_fn, hc_scale, hc_base with the same params p:
  *     d_R [T][4][H] bf16, d_hc_fn [4H][24] fp32, d_scale [3] fp32, d_base [24] fp32.
  *   The projection is recomputed; gradients flow through the gates (sigmoid), the Sinkhorn rounds
- *   (each normalisation Y = Z / (sum + eps) has dZ = (dY - sum(dY * Y)) / (sum + eps); the
- *   row-max shift sends the row's sum of dA0 * A0, negated, to its first maximum), the logit
+ *   (each normalisation Y = Z / sum has dZ = (dY - sum(dY * Y)) / sum; the starting softmax P
+ *   has d_l = P (dA0 - sum_n dA0 P) along the row), the logit
  *   affine, rstd (d_ss = -rstd^3 / (8H) d_rstd) and the aggregate. Token sums are fixed-order.
  *   workspace: mhc_pre_backward_workspace_bytes(T, H) bytes, 256-byte aligned.
  *   Errors: MHC_ERR_INVALID_ARG, MHC_ERR_WORKSPACE_TOO_SMALL, MHC_ERR_ALIAS.

@@ -240,15 +240,15 @@ __device__ __forceinline__ float quad_sum(float v) {
 }
 
 // One Sinkhorn round on the quad's 4x4 (lane r holds row r): row normalisation then column
-// normalisation; returns B (after the row step), rs and cs (the normalisers) for the reverse pass.
-__device__ __forceinline__ void sk_round(float (&a)[4], float (&b)[4], float& rs, float (&cs)[4],
-                                         float eps) {
-  rs = ((a[0] + a[1]) + a[2]) + a[3] + eps;
+// normalisation by plain sums; returns B (after the row step), rs and cs (the normalisers) for the
+// reverse pass.
+__device__ __forceinline__ void sk_round(float (&a)[4], float (&b)[4], float& rs, float (&cs)[4]) {
+  rs = ((a[0] + a[1]) + a[2]) + a[3];
 #pragma unroll
   for (int n = 0; n < 4; ++n) b[n] = a[n] / rs;
 #pragma unroll
   for (int n = 0; n < 4; ++n) {
-    cs[n] = quad_sum(b[n]) + eps;
+    cs[n] = quad_sum(b[n]);
     a[n] = b[n] / cs[n];
   }
 }
@@ -293,33 +293,41 @@ __global__ void __launch_bounds__(256) pre_bwd_coef_kernel(
   const float dl0 = dpt[tt * 4 + r] * sg0 * (1.0f - sg0);
   const float dl1 = (dpost ? dpost[tt * 4 + r] : 0.f) * fp.post_mult * sg1 * (1.0f - sg1);
 
-  // Sinkhorn reverse pass. The forward states are checkpointed every G rounds (at most kSkCk
-  // checkpoints); the state entering round k is recomputed from the checkpoint at or before it,
-  // by the same operations as the forward, so it is the forward's state exactly.
-  float a0[4], dA[4];
-  const float mx = fmaxf(fmaxf(lc[0], lc[1]), fmaxf(lc[2], lc[3]));
+  // Sinkhorn reverse pass. The forward starts from P = softmax(row) and A0 = P + eps; its states
+  // are checkpointed every G rounds (at most kSkCk checkpoints); the state entering round k is
+  // recomputed from the checkpoint at or before it, by the same operations as the forward, so it
+  // is the forward's state exactly.
+  float p[4], dA[4];
+  {
+    const float mx = fmaxf(fmaxf(lc[0], lc[1]), fmaxf(lc[2], lc[3]));
 #pragma unroll
-  for (int n = 0; n < 4; ++n) {
-    a0[n] = expf(lc[n] - mx);
-    dA[n] = dcomb ? dcomb[tt * 16 + 4 * r + n] : 0.f;
+    for (int n = 0; n < 4; ++n) p[n] = expf(lc[n] - mx);
+    const float es = ((p[0] + p[1]) + p[2]) + p[3];
+#pragma unroll
+    for (int n = 0; n < 4; ++n) {
+      p[n] = p[n] / es;
+      dA[n] = dcomb ? dcomb[tt * 16 + 4 * r + n] : 0.f;
+    }
   }
   const int G = (fp.iters + kSkCk - 1) / kSkCk;
   float ck[kSkCk][4];
   {
-    float a[4] = {a0[0], a0[1], a0[2], a0[3]}, b[4], rs, cs[4];
+    float a[4] = {p[0] + fp.sinkhorn_eps, p[1] + fp.sinkhorn_eps, p[2] + fp.sinkhorn_eps,
+                  p[3] + fp.sinkhorn_eps},
+          b[4], rs, cs[4];
     for (int k = 0; k < fp.iters; ++k) {
       if (k % G == 0) {
 #pragma unroll
         for (int n = 0; n < 4; ++n) ck[k / G][n] = a[n];
       }
-      sk_round(a, b, rs, cs, fp.sinkhorn_eps);
+      sk_round(a, b, rs, cs);
     }
   }
   for (int k = fp.iters - 1; k >= 0; --k) {
     const int c = k / G;
     float a[4] = {ck[c][0], ck[c][1], ck[c][2], ck[c][3]}, b[4], rs, cs[4];
-    for (int j = c * G; j < k; ++j) sk_round(a, b, rs, cs, fp.sinkhorn_eps);
-    sk_round(a, b, rs, cs, fp.sinkhorn_eps);  // round k: a is now C
+    for (int j = c * G; j < k; ++j) sk_round(a, b, rs, cs);
+    sk_round(a, b, rs, cs);  // round k: a is now C
     float dB[4];
 #pragma unroll
     for (int n = 0; n < 4; ++n) dB[n] = (dA[n] - quad_sum(dA[n] * a[n])) / cs[n];
@@ -327,19 +335,13 @@ __global__ void __launch_bounds__(256) pre_bwd_coef_kernel(
 #pragma unroll
     for (int n = 0; n < 4; ++n) dA[n] = (dB[n] - rdot) / rs;
   }
-  float dlc[4], gsum = 0.f;
-  int am = 0;
+  // Softmax: d_l = P (dA0 - sum_n dA0 P) along the row.
+  float dlc[4];
+  {
+    const float pd = ((dA[0] * p[0] + dA[1] * p[1]) + dA[2] * p[2]) + dA[3] * p[3];
 #pragma unroll
-  for (int n = 0; n < 4; ++n) {
-    dlc[n] = dA[n] * a0[n];
-    gsum += dlc[n];
+    for (int n = 0; n < 4; ++n) dlc[n] = p[n] * (dA[n] - pd);
   }
-#pragma unroll
-  for (int n = 1; n < 4; ++n)
-    if (lc[n] > lc[am]) am = n;  // the first maximum takes the row-max shift's derivative
-#pragma unroll
-  for (int n = 0; n < 4; ++n)
-    if (n == am) dlc[n] -= gsum;
 
   const float dm0 = dl0 * s0, dm1 = dl1 * s1;
   float dmc[4];

@@ -169,23 +169,27 @@ __device__ __forceinline__ float recip_nr(float s) {
 }
 
 // Sinkhorn on one 4x4 block held as 4 rows by 4 cooperating lanes: lane q (= lane & 3 within its
-// quad) owns row q. Row max shift and exp, then `iters` rounds of (row /= rowsum + eps,
-// column /= colsum + eps), each division done as a multiplication by recip_nr of the sum.
-// Column sums reduce across the quad with xor shuffles. All 32 lanes of the warp must call it
-// (inactive quads pass any finite values).
+// quad) owns row q. The row goes through a softmax (row maximum subtracted first) and eps is added
+// to every entry; then `iters` rounds of (row /= rowsum, column /= colsum) with plain sums
+// ("FlashInfer mHC module deep dive" §5.2 test reference, §3.4 phase 2). Every division is a
+// multiplication by recip_nr of the sum. Column sums reduce across the quad with xor shuffles.
+// All 32 lanes of the warp must call it (inactive quads pass any finite values).
 __device__ __forceinline__ void sinkhorn_quad(float (&a)[4], int iters, float eps) {
-  float m = fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3]));
+  const float m = fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3]));
 #pragma unroll
   for (int n = 0; n < 4; ++n) a[n] = expf(a[n] - m);
+  const float rs0 = recip_nr(((a[0] + a[1]) + a[2]) + a[3]);
+#pragma unroll
+  for (int n = 0; n < 4; ++n) a[n] = fmaf(a[n], rs0, eps);
   for (int it = 0; it < iters; ++it) {
-    const float rr = recip_nr(((a[0] + a[1]) + a[2]) + a[3] + eps);
+    const float rr = recip_nr(((a[0] + a[1]) + a[2]) + a[3]);
 #pragma unroll
     for (int n = 0; n < 4; ++n) a[n] *= rr;
 #pragma unroll
     for (int n = 0; n < 4; ++n) {
       float c = a[n] + __shfl_xor_sync(0xffffffffu, a[n], 1);
       c = c + __shfl_xor_sync(0xffffffffu, c, 2);
-      a[n] *= recip_nr(c + eps);
+      a[n] *= recip_nr(c);
     }
   }
 }

@@ -1,6 +1,6 @@
-// Standalone Sinkhorn normalisation of [T][4][4] logits ("FlashInfer mHC module deep dive" §3.4:
-// softmax with row-max shift, then rounds of row and column normalisation; rwkv-ops
-// sinkhorn_knopp: eps guards each division).
+// Standalone Sinkhorn normalisation of [T][4][4] logits ("FlashInfer mHC module deep dive" §3.4,
+// §5.2: row softmax with row-max shift, eps added to every entry, then rounds of row and column
+// normalisation by plain sums).
 //
 // Four lanes per token, lane q owning row q (16 bytes in, 16 bytes out): rows normalise in
 // registers, column sums reduce across the quad with xor shuffles.

@@ -19,7 +19,7 @@ from .c_oracle import (  # noqa: F401
     norm_project,
     sinkhorn,
     sinkhorn_converge,
-    sinkhorn_entry_eps,
+    sinkhorn_variant,
     coefficients,
     aggregate,
     pre,

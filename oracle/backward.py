@@ -19,11 +19,10 @@ pre-map   X = R_flat; ss = sum X^2; rstd = (ss/K + rms_eps)^(-1/2); raw = X . hc
     d_raw = d_m rstd;  d_rstd = sum_j d_m_j raw_j;  d_ss = -rstd^3 / (2K) d_rstd;
     d_X = d_y-part (pre_i d_y[h]) + d_raw . hc_fn^T + 2 X d_ss;  d_hc_fn = X^T d_raw.
 
-Sinkhorn VJP: the forward is A0 = exp(l - rowmax(l)), then per round B = A / (rowsum(A) + eps),
-C = B / (colsum(B) + eps). A normalisation Y = Z / (s + eps), s the sum of the row (or column) of
-Z, has dZ = (dY - sum(dY * Y) over that row or column) / (s + eps). The row-max shift is part of
-the function: its (almost-everywhere) derivative sends minus the row's sum of dA0 * A0 to the
-argmax entry.
+Sinkhorn VJP: the forward is P = softmax(l) over each row, A0 = P + eps, then per round
+B = A / rowsum(A), C = B / colsum(B). A normalisation Y = Z / s, s the sum of the row (or column)
+of Z, has dZ = (dY - sum(dY * Y) over that row or column) / s. The softmax has
+dl = P * (dA0 - sum_n dA0 * P) per row (the row-max shift cancels out of it).
 """
 
 from __future__ import annotations
@@ -49,36 +48,32 @@ def post_backward(d_out, x, R, post, comb):
 
 
 def _sinkhorn_forward_states(lg, iters, eps):
-    """lg [4,4] fp64 logits. Returns A0 and per round (B, rowsum+eps, C, colsum+eps)."""
-    A0 = np.exp(lg - lg.max(axis=1, keepdims=True))
-    A = A0
+    """lg [4,4] fp64 logits. Returns the row softmax P and per round (B, rowsum, C, colsum)."""
+    ex = np.exp(lg - lg.max(axis=1, keepdims=True))
+    P = ex / ex.sum(axis=1, keepdims=True)
+    A = P + eps
     states = []
     for _ in range(iters):
-        rs = A.sum(axis=1, keepdims=True) + eps
+        rs = A.sum(axis=1, keepdims=True)
         B = A / rs
-        cs = B.sum(axis=0, keepdims=True) + eps
+        cs = B.sum(axis=0, keepdims=True)
         C = B / cs
         states.append((B, rs, C, cs))
         A = C
-    return A0, states
+    return P, states
 
 
 def sinkhorn_vjp(lg, d_comb, iters, eps):
     """Gradient of Sinkhorn(lg) (fixed rounds) with respect to the logits lg [4,4]."""
-    A0, states = _sinkhorn_forward_states(lg, iters, eps)
+    P, states = _sinkhorn_forward_states(lg, iters, eps)
     dA = np.array(d_comb, dtype=np.float64)
     for B, rs, C, cs in reversed(states):
         # C = B / cs (column normalisation)
         dB = (dA - (dA * C).sum(axis=0, keepdims=True)) / cs
         # B = A / rs (row normalisation)
         dA = (dB - (dB * B).sum(axis=1, keepdims=True)) / rs
-    # A0 = exp(lg - rowmax)
-    g = dA * A0
-    dl = g.copy()
-    am = lg.argmax(axis=1)
-    for o in range(4):
-        dl[o, am[o]] -= g[o].sum()
-    return dl
+    # A0 = P + eps, P = softmax(lg) per row
+    return P * (dA - (dA * P).sum(axis=1, keepdims=True))
 
 
 def pre_backward(d_y, d_pre, d_post, d_comb, R, hc_fn, scale, base, rms_eps=1e-6, pre_eps=0.0,

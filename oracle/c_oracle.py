@@ -52,7 +52,8 @@ def _load():
     lib.mhc_oracle_sinkhorn_converge.argtypes = [_D, _I64, ctypes.c_double, ctypes.c_double,
                                                  ctypes.c_int, _D]
     lib.mhc_oracle_sinkhorn_converge.restype = ctypes.c_int
-    lib.mhc_oracle_sinkhorn_entry_eps.argtypes = [_D, _I64, ctypes.c_int, ctypes.c_double, _D]
+    lib.mhc_oracle_sinkhorn_variant.argtypes = [_D, _I64, ctypes.c_int, ctypes.c_double,
+                                                ctypes.c_int, _D]
     lib.mhc_oracle_coefficients.argtypes = [_D, _D, _F, _F, _I64, ctypes.c_double,
                                             ctypes.c_double, ctypes.c_int, ctypes.c_double,
                                             _D, _D, _D, _D]
@@ -104,7 +105,8 @@ def norm_project(R, hc_fn, rms_eps=1e-6):
 
 
 def sinkhorn(logits, iters=20, eps=1e-6):
-    """Step a4/a7 on logits [T,4,4] (or [T,16]); returns comb [T,4,4] ([old][new])."""
+    """Step a4/a7 on logits [T,4,4] (or [T,16]); returns comb [T,4,4] ([old][new]): softmax of
+    each row plus eps, then `iters` (row, column) normalisation rounds."""
     lg, pl = _c(logits, np.float64, _D)
     T = lg.size // 16
     out = np.empty((T, 4, 4))
@@ -121,11 +123,15 @@ def sinkhorn_converge(logits, eps=1e-6, tol=1e-12, max_iters=10000):
     return out, used
 
 
-def sinkhorn_entry_eps(logits, iters=20, eps=1e-6):
+def sinkhorn_variant(logits, iters=20, eps=1e-6, variant=1):
+    """Another reading of the Sinkhorn step, for the reading-gap report only (see mhc_oracle.h):
+    variant 1 = eps in the row/column sums, none on the entries; variant 2 = an extra column
+    normalisation straight after the softmax."""
     lg, pl = _c(logits, np.float64, _D)
     T = lg.size // 16
     out = np.empty((T, 4, 4))
-    _load().mhc_oracle_sinkhorn_entry_eps(pl, T, int(iters), float(eps), out.ctypes.data_as(_D))
+    _load().mhc_oracle_sinkhorn_variant(pl, T, int(iters), float(eps), int(variant),
+                                        out.ctypes.data_as(_D))
     return out
 
 

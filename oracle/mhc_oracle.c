@@ -72,26 +72,40 @@ void mhc_oracle_norm_project(const uint16_t* R, const float* hc_fn, int64_t T, i
     }
 }
 
-/* One token: A = exp(l - rowmax); then rounds of row and column normalisation. */
-static void sinkhorn_one(const double* l, int iters, double eps, double* A) {
+/* Start of the Sinkhorn step for one token ([FI] §5.2 test reference, §3.4 kernel phase 2): a
+ * softmax over each row of the 4x4 logits, computed with the row maximum subtracted first, and eps
+ * added to every entry of the result. */
+static void softmax_plus_eps(const double* l, double eps, double* A) {
     for (int o = 0; o < HC; ++o) {
         double m = l[o * HC];
         for (int n = 1; n < HC; ++n)
             if (l[o * HC + n] > m) m = l[o * HC + n];
-        for (int n = 0; n < HC; ++n) A[o * HC + n] = exp(l[o * HC + n] - m);
-    }
-    for (int it = 0; it < iters; ++it) {
-        for (int o = 0; o < HC; ++o) {
-            double s = 0.0;
-            for (int n = 0; n < HC; ++n) s += A[o * HC + n];
-            for (int n = 0; n < HC; ++n) A[o * HC + n] /= (s + eps);
-        }
+        double e[HC], s = 0.0;
         for (int n = 0; n < HC; ++n) {
-            double s = 0.0;
-            for (int o = 0; o < HC; ++o) s += A[o * HC + n];
-            for (int o = 0; o < HC; ++o) A[o * HC + n] /= (s + eps);
+            e[n] = exp(l[o * HC + n] - m);
+            s += e[n];
         }
+        for (int n = 0; n < HC; ++n) A[o * HC + n] = e[n] / s + eps;
     }
+}
+
+/* One Sinkhorn round ([FI] §5.2): every row divided by its sum, then every column by its sum. */
+static void row_then_column(double* A) {
+    for (int o = 0; o < HC; ++o) {
+        double s = 0.0;
+        for (int n = 0; n < HC; ++n) s += A[o * HC + n];
+        for (int n = 0; n < HC; ++n) A[o * HC + n] /= s;
+    }
+    for (int n = 0; n < HC; ++n) {
+        double s = 0.0;
+        for (int o = 0; o < HC; ++o) s += A[o * HC + n];
+        for (int o = 0; o < HC; ++o) A[o * HC + n] /= s;
+    }
+}
+
+static void sinkhorn_one(const double* l, int iters, double eps, double* A) {
+    softmax_plus_eps(l, eps, A);
+    for (int it = 0; it < iters; ++it) row_then_column(A);
 }
 
 void mhc_oracle_sinkhorn(const double* logits, int64_t T, int iters, double eps, double* comb) {
@@ -104,20 +118,11 @@ int mhc_oracle_sinkhorn_converge(const double* logits, int64_t T, double eps, do
     int used = 0;
     for (int64_t t = 0; t < T; ++t) {
         double A[16], prev[16];
-        sinkhorn_one(logits + t * 16, 0, eps, A);
+        softmax_plus_eps(logits + t * 16, eps, A);
         int it = 0;
         for (; it < max_iters; ++it) {
             memcpy(prev, A, sizeof A);
-            for (int o = 0; o < HC; ++o) {
-                double s = 0.0;
-                for (int n = 0; n < HC; ++n) s += A[o * HC + n];
-                for (int n = 0; n < HC; ++n) A[o * HC + n] /= (s + eps);
-            }
-            for (int n = 0; n < HC; ++n) {
-                double s = 0.0;
-                for (int o = 0; o < HC; ++o) s += A[o * HC + n];
-                for (int o = 0; o < HC; ++o) A[o * HC + n] /= (s + eps);
-            }
+            row_then_column(A);
             double d = 0.0;
             for (int i = 0; i < 16; ++i) d = fmax(d, fabs(A[i] - prev[i]));
             if (d < tol) {
@@ -131,30 +136,44 @@ int mhc_oracle_sinkhorn_converge(const double* logits, int64_t T, double eps, do
     return used;
 }
 
-void mhc_oracle_sinkhorn_entry_eps(const double* logits, int64_t T, int iters, double eps,
-                                   double* comb) {
+/* Other readings of the Sinkhorn step, kept only so that a test can report how far each sits from
+ * mhc_oracle_sinkhorn:
+ *   variant 1 (rwkv-ops sinkhorn_knopp, whose eps guards the divisions): A = exp(l - rowmax),
+ *             nothing added to the entries, eps added to every row and column sum instead;
+ *   variant 2 ([FI] §3.4 read as three phases): softmax + eps, one column normalisation, then
+ *             `iters` full (row, column) rounds. */
+void mhc_oracle_sinkhorn_variant(const double* logits, int64_t T, int iters, double eps,
+                                 int variant, double* comb) {
     for (int64_t t = 0; t < T; ++t) {
         const double* l = logits + t * 16;
         double* A = comb + t * 16;
-        for (int o = 0; o < HC; ++o) {
-            double m = l[o * HC];
-            for (int n = 1; n < HC; ++n)
-                if (l[o * HC + n] > m) m = l[o * HC + n];
-            double s = 0.0;
-            for (int n = 0; n < HC; ++n) s += exp(l[o * HC + n] - m);
-            for (int n = 0; n < HC; ++n) A[o * HC + n] = exp(l[o * HC + n] - m) / s + eps;
-        }
-        for (int it = 0; it < iters; ++it) {
+        if (variant == 1) {
             for (int o = 0; o < HC; ++o) {
-                double s = 0.0;
-                for (int n = 0; n < HC; ++n) s += A[o * HC + n];
-                for (int n = 0; n < HC; ++n) A[o * HC + n] /= s;
+                double m = l[o * HC];
+                for (int n = 1; n < HC; ++n)
+                    if (l[o * HC + n] > m) m = l[o * HC + n];
+                for (int n = 0; n < HC; ++n) A[o * HC + n] = exp(l[o * HC + n] - m);
             }
+            for (int it = 0; it < iters; ++it) {
+                for (int o = 0; o < HC; ++o) {
+                    double s = 0.0;
+                    for (int n = 0; n < HC; ++n) s += A[o * HC + n];
+                    for (int n = 0; n < HC; ++n) A[o * HC + n] /= (s + eps);
+                }
+                for (int n = 0; n < HC; ++n) {
+                    double s = 0.0;
+                    for (int o = 0; o < HC; ++o) s += A[o * HC + n];
+                    for (int o = 0; o < HC; ++o) A[o * HC + n] /= (s + eps);
+                }
+            }
+        } else {
+            softmax_plus_eps(l, eps, A);
             for (int n = 0; n < HC; ++n) {
                 double s = 0.0;
                 for (int o = 0; o < HC; ++o) s += A[o * HC + n];
                 for (int o = 0; o < HC; ++o) A[o * HC + n] /= s;
             }
+            for (int it = 0; it < iters; ++it) row_then_column(A);
         }
     }
 }

@@ -45,8 +45,10 @@ void mhc_oracle_round_bf16(const double* in, int64_t n, double* out);
 void mhc_oracle_norm_project(const uint16_t* R, const float* hc_fn, int64_t T, int64_t H,
                              double rms_eps, double* ss, double* rstd, double* raw);
 
-/* Step a4 on already-formed logits: A = exp(l - rowmax(l)), then `iters` rounds of
- * (rows /= rowsum + eps; columns /= colsum + eps). logits and comb are [T][16], [old][new]. */
+/* Step a4 on already-formed logits, as [FI] §5.2's test reference states it: each row of the 4x4
+ * goes through a softmax (row maximum subtracted first, [FI] §3.4), eps is added to every entry,
+ * then `iters` rounds of (every row divided by its sum; every column divided by its sum), the sums
+ * taken plainly. logits and comb are [T][16], [old][new]. */
 void mhc_oracle_sinkhorn(const double* logits, int64_t T, int iters, double eps, double* comb);
 
 /* The same normalisation run until the largest change in a round drops below tol or max_iters
@@ -54,11 +56,12 @@ void mhc_oracle_sinkhorn(const double* logits, int64_t T, int iters, double eps,
 int mhc_oracle_sinkhorn_converge(const double* logits, int64_t T, double eps, double tol,
                                  int max_iters, double* comb);
 
-/* The variant [FI] §5.2 describes for its test reference: softmax over each row, eps added to
- * every entry, then `iters` rounds of (row normalise, column normalise) with plain sums. Kept only
- * so a test can report how far it sits from mhc_oracle_sinkhorn. */
-void mhc_oracle_sinkhorn_entry_eps(const double* logits, int64_t T, int iters, double eps,
-                                   double* comb);
+/* Other readings of the pages' Sinkhorn, kept only so a test can report how far each sits from
+ * mhc_oracle_sinkhorn: variant 1 = rwkv-ops sinkhorn_knopp's (exp after the row-max shift, eps
+ * added to each row and column sum, nothing added to the entries); variant 2 = [FI] §3.4 read as
+ * three phases (softmax + eps, one column normalisation, then `iters` full rounds). */
+void mhc_oracle_sinkhorn_variant(const double* logits, int64_t T, int iters, double eps,
+                                 int variant, double* comb);
 
 /* Step a3 + a4: logits l = raw*rstd*scale[g(j)] + base[j] (g = 0,1,2 for pre, post, comb),
  * pre = sigmoid(l[0:4]) + pre_eps, post = post_mult*sigmoid(l[4:8]), comb = Sinkhorn(l[8:24]). */

@@ -17,12 +17,14 @@ def widen_bf16(bits) -> np.ndarray:
 
 
 def sinkhorn(logits, iters, eps):
-    """logits [T,4,4] -> doubly-stochastic estimate after `iters` (row, column) rounds."""
+    """logits [T,4,4] -> doubly-stochastic estimate: row softmax plus eps on every entry, then
+    `iters` rounds of (rows / row sums, columns / column sums)."""
     lg = np.asarray(logits, dtype=np.float64).reshape(-1, 4, 4)
-    A = np.exp(lg - lg.max(axis=2, keepdims=True))
+    ex = np.exp(lg - lg.max(axis=2, keepdims=True))
+    A = ex / ex.sum(axis=2, keepdims=True) + eps
     for _ in range(iters):
-        A = A / (A.sum(axis=2, keepdims=True) + eps)
-        A = A / (A.sum(axis=1, keepdims=True) + eps)
+        A = A / A.sum(axis=2, keepdims=True)
+        A = A / A.sum(axis=1, keepdims=True)
     return A
 
 

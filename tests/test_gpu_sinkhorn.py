@@ -1,6 +1,6 @@
 """GPU parity of the standalone Sinkhorn entry (mhc_sinkhorn) against the fp64 oracle:
-A = exp(l - rowmax), then `iters` rounds of (rows /= rowsum + eps, columns /= colsum + eps)
-("FlashInfer mHC module deep dive" §3.4; rwkv-ops sinkhorn_knopp). Coefficient bar: 1e-5."""
+A = softmax(l, each row) + eps, then `iters` rounds of (rows /= rowsum, columns /= colsum)
+("FlashInfer mHC module deep dive" §3.4, §5.2). Coefficient bar: 1e-5."""
 
 import numpy as np
 import pytest

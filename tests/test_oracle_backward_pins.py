@@ -1,6 +1,6 @@
 """Pins of the backward oracle (oracle/backward.py) against torch autograd on an independent float64
 restatement of the forward maps ("FlashInfer mHC module deep dive" §2.1 post-map, §3.4 / §5.2
-pre-map: RMS over 4H, projection, scale groups, sigmoid gates, row-max-shifted Sinkhorn rounds,
+pre-map: RMS over 4H, projection, scale groups, sigmoid gates, softmax + eps then Sinkhorn rounds,
 aggregate). Autograd derives the derivatives itself, so a dropped term, wrong sign or transposed
 operand in the oracle's hand-written reverse pass fails here. Also pins the Sinkhorn forward states
 the VJP replays against the C oracle's Sinkhorn."""
@@ -37,10 +37,10 @@ def torch_pre(R, W, sc, bs, rms_eps, pre_eps, post_mult, iters, eps):
     pre = torch.sigmoid(lg[:, :4]) + pre_eps
     post = post_mult * torch.sigmoid(lg[:, 4:8])
     c = lg[:, 8:].reshape(T, 4, 4)
-    A = torch.exp(c - c.max(dim=2, keepdim=True).values)
+    A = torch.softmax(c, dim=2) + eps
     for _ in range(iters):
-        A = A / (A.sum(dim=2, keepdim=True) + eps)
-        A = A / (A.sum(dim=1, keepdim=True) + eps)
+        A = A / A.sum(dim=2, keepdim=True)
+        A = A / A.sum(dim=1, keepdim=True)
     y = (pre[:, :, None] * R).sum(1)
     return y, pre, post, A
 
@@ -97,7 +97,7 @@ def test_sinkhorn_states_match_c_oracle():
 
 
 def test_sinkhorn_vjp_finite_differences():
-    """Central differences of the C oracle's Sinkhorn against the VJP (away from row-max ties)."""
+    """Central differences of the C oracle's Sinkhorn against the VJP."""
     lg = RNG.standard_normal((4, 4))
     dc = RNG.standard_normal((4, 4))
     dl = backward.sinkhorn_vjp(lg, dc, 20, 1e-6)

@@ -4,9 +4,9 @@ restatement). Each test names the step and the passage it pins:
 
 * [FI]  "FlashInfer mHC module deep dive": §2.1 post formula, §3.2 parameters, §3.4 kernel phases
         (sigmoid gates, softmax with row-max shift, Sinkhorn row->column rounds), §4 (RMS over 4*H),
-        §5.2 test reference math.
+        §5.2 test reference math (softmax, eps added to the entries, `iters` row -> column rounds).
 * [RW]  rwkv-ops ``mhu_jax.py``: ``mhc_pre_op`` docstring (H_pre = sigmoid, H_post = 2*sigmoid,
-        x_layer_in = sum(H_pre * x_expanded)), ``sinkhorn_knopp`` (eps guards a division).
+        x_layer_in = sum(H_pre * x_expanded)).
 * [GLM] ``glm5next_mhc.rs``: ``glm_hc_post`` (out[j] = post[j]*block_out + sum_i comb[i][j]*residual[i]).
 
 A plausible mistake (dropped term, wrong sign, swapped index, transposed operand, eps in the wrong
@@ -52,35 +52,33 @@ def test_sinkhorn_converges_to_doubly_stochastic():
 
 def test_sinkhorn_scaling_invariance_at_convergence():
     """Sinkhorn's limit is unique: adding a constant per row and per column of the logits
-    (D1 A D2 after exp) leaves the converged matrix unchanged."""
+    (D1 A D2 after exp) leaves the converged matrix unchanged. eps = 0 here: the eps added to the
+    entries is not a row or column scaling, so the invariant holds for the eps-free iteration."""
     logits = RNG.standard_normal((200, 4, 4))
     a = RNG.standard_normal((200, 4, 1)) * 3.0
     b = RNG.standard_normal((200, 1, 4)) * 3.0
-    c1, _ = oracle.sinkhorn_converge(logits, eps=1e-14, tol=1e-15, max_iters=20000)
-    c2, _ = oracle.sinkhorn_converge(logits + a + b, eps=1e-14, tol=1e-15, max_iters=20000)
+    c1, _ = oracle.sinkhorn_converge(logits, eps=0.0, tol=1e-15, max_iters=20000)
+    c2, _ = oracle.sinkhorn_converge(logits + a + b, eps=0.0, tol=1e-15, max_iters=20000)
     assert np.max(np.abs(c1 - c2)) < 1e-9
 
 
-@pytest.mark.parametrize("iters", [1, 2, 3, 20])
 @pytest.mark.parametrize("eps", [1e-6, 0.25])
-def test_sinkhorn_rank_one_closed_form(iters, eps):
-    """Logits l[o][n] = a_o + b_n: after the row-max shift every row is the same vector
-    e_n = exp(b_n - max b), so each round reduces to two scalar maps on one vector:
-    v <- v / (sum(v) + eps) (row step), then v <- v / (4 v + eps) (column step: 4 equal rows).
-    Pins the eps placement (denominator, not entries) and the row-then-column order."""
+def test_sinkhorn_rank_one_closed_form(eps):
+    """Logits l[o][n] = a_o + b_n: every row's softmax is the same vector p_n = exp(b_n)/sum exp(b)
+    (the row constant a_o cancels), so before any round every entry is p_n + eps ([FI] §5.2: eps is
+    added to the softmax output). A row step keeps the four rows equal, and a column step then
+    divides four equal entries by their sum: after one round or more, every entry is exactly 1/4.
+    Pins eps on the entries (zero rounds) and plain, eps-free row and column sums (an eps added
+    to the sums would leave v / (4 v + eps) instead of 1/4)."""
     a = RNG.standard_normal(4) * 2.0
     b = RNG.standard_normal(4)
     logits = a[:, None] + b[None, :]
-    v = [math.exp(bn - max(b)) for bn in b]
-    for _ in range(iters):
-        s = sum(v)
-        v = [vn / (s + eps) for vn in v]
-        v = [vn / (4.0 * vn + eps) for vn in v]
-    expect = np.tile(np.array(v), (4, 1))
-    got = oracle.sinkhorn(logits[None], iters=iters, eps=eps)[0]
-    np.testing.assert_allclose(got, expect, rtol=1e-14, atol=0)
-    if eps == 1e-6:
-        np.testing.assert_allclose(got, 0.25, atol=1e-5)  # uniform limit
+    p = np.exp(b) / np.exp(b).sum()
+    got0 = oracle.sinkhorn(logits[None], iters=0, eps=eps)[0]
+    np.testing.assert_allclose(got0, np.tile(p + eps, (4, 1)), rtol=1e-14, atol=0)
+    for iters in (1, 2, 3, 20):
+        got = oracle.sinkhorn(logits[None], iters=iters, eps=eps)[0]
+        np.testing.assert_allclose(got, 0.25, rtol=1e-14, atol=0)
 
 
 def test_sinkhorn_permutation_equivariance_brute_force():
@@ -107,34 +105,72 @@ def test_sinkhorn_permutation_dominant_stays_near_permutation():
         assert np.max(np.abs(comb[0] - P)) < 1e-4
 
 
+M_HAND = np.array([[1, 2, 3, 4], [4, 3, 2, 1], [1, 1, 1, 1], [1, 2, 2, 5]], dtype=np.float64)
+
+
 def test_sinkhorn_single_round_hand_example():
-    """A 4x4 example worked by hand, eps = 0: logits log(M), M = [[1,2,3,4],[4,3,2,1],[1,1,1,1],
-    [1,2,2,5]]. The row step gives rows (1,2,3,4)/10, (4,3,2,1)/10, (1,1,1,1)/4, (1,2,2,5)/10; the
-    column sums are then (0.85, 0.95, 0.95, 1.25) and the column step divides by them."""
-    M = np.array([[1, 2, 3, 4], [4, 3, 2, 1], [1, 1, 1, 1], [1, 2, 2, 5]], dtype=np.float64)
-    rows = np.array([[.1, .2, .3, .4], [.4, .3, .2, .1], [.25, .25, .25, .25], [.1, .2, .2, .5]])
-    cols = np.array([0.85, 0.95, 0.95, 1.25])
-    got = oracle.sinkhorn(np.log(M)[None], iters=1, eps=0.0)[0]
-    np.testing.assert_allclose(got, rows / cols[None, :], rtol=1e-14)
+    """Worked by hand, eps = 0.05, one round, logits log(M) with M = [[1,2,3,4],[4,3,2,1],[1,1,1,1],
+    [1,2,2,5]]. The row softmax gives M / rowsum: (.1,.2,.3,.4), (.4,.3,.2,.1), (.25,.25,.25,.25),
+    (.1,.2,.2,.5); eps makes them (.15,.25,.35,.45), (.45,.35,.25,.15), (.3,.3,.3,.3),
+    (.15,.25,.25,.55). Every row now sums to 1.2, so the row step divides everything by 1.2, and the
+    column step divides by the column sums (1.05, 1.15, 1.15, 1.45) / 1.2. Result: entry / column
+    sum of the eps-shifted matrix. Without eps on the entries the columns would be divided by
+    (.85, .95, .95, 1.25) instead."""
+    shifted = np.array([[.15, .25, .35, .45], [.45, .35, .25, .15], [.3, .3, .3, .3],
+                        [.15, .25, .25, .55]])
+    cols = np.array([1.05, 1.15, 1.15, 1.45])
+    got = oracle.sinkhorn(np.log(M_HAND)[None], iters=1, eps=0.05)[0]
+    np.testing.assert_allclose(got, shifted / cols[None, :], rtol=1e-14)
 
 
-def test_sinkhorn_entry_eps_reading_gap_report(capsys):
-    """Not a pin: a report of how far the chosen reading (eps only in the row/column denominators)
-    sits from the other one the FlashInfer page's §5.2 suggests (softmax, eps added to every entry,
-    then plain row/column rounds). On N(0,1) logits with 20 rounds the two agree to ~2e-5; on the
-    near-permutation 3*N(0,1) logits with 50 rounds they differ by up to ~3e-2, because the
-    fixed-round output has not converged and eps-sized entries still move it. The readings are not
-    interchangeable at the 1e-5 tolerance; the library follows the denominator reading."""
+def test_sinkhorn_two_round_hand_example():
+    """Pins the round count (`iters` counts full row -> column rounds). eps = 0, M as above, in
+    exact rational arithmetic. Round 1: rows of M / rowsum already sum to 1; the column sums are
+    (17/20, 19/20, 19/20, 5/4), giving C1 = [[2/17, 4/19, 6/19, 8/25], [8/17, 6/19, 4/19, 2/25],
+    [5/17, 5/19, 5/19, 1/5], [2/17, 4/19, 4/19, 2/5]]. Round 2: C1's row sums are
+    (7784/8075, 8696/8075, 1648/1615, 1516/1615); dividing the rows by them and then the columns by
+    their new sums gives the fractions below. One round fewer or more (e.g. an extra column step
+    straight after the softmax) misses them."""
+    num = [[848664380, 1697328760, 2545993140, 678931504],
+           [3038640080, 2278980060, 1519320040, 151932004],
+           [2004248645, 2004248645, 2004248645, 400849729],
+           [871504424, 1743008848, 1743008848, 871504424]]
+    den = [6763057529, 7723566313, 7812570673, 2103217661]
+    expect = np.array([[num[o][n] / den[n] for n in range(4)] for o in range(4)])
+    got = oracle.sinkhorn(np.log(M_HAND)[None], iters=2, eps=0.0)[0]
+    np.testing.assert_allclose(got, expect, rtol=1e-14)
+    np.testing.assert_allclose(got.sum(axis=0), 1.0, rtol=1e-14)  # the last step is a column step
+
+
+def test_sinkhorn_columns_sum_to_one_after_every_round():
+    """The last operation of each round is a column normalisation, so every column sums to 1 (to
+    rounding) after any number of rounds, while the rows only approach 1."""
+    logits = RNG.standard_normal((500, 4, 4)) * 2.0
+    for iters in (1, 3, 20):
+        comb = oracle.sinkhorn(logits, iters=iters, eps=1e-6)
+        assert np.max(np.abs(comb.sum(axis=1) - 1.0)) < 1e-14
+    assert np.max(np.abs(oracle.sinkhorn(logits, iters=1, eps=1e-6).sum(axis=2) - 1.0)) > 1e-3
+
+
+def test_sinkhorn_reading_gap_report(capsys):
+    """Not a pin: a report of how far the other readings of the pages' Sinkhorn sit from the one the
+    oracle follows ([FI] §5.2: softmax, eps added to every entry, then `iters` plain row -> column
+    rounds). Variant 1 is rwkv-ops' (eps in the row and column sums, none on the entries); variant
+    2 reads [FI] §3.4 as an extra column step straight after the softmax. On N(0,1) logits with 20
+    rounds they agree to ~1e-5; on the near-permutation 3*N(0,1) logits with 50 rounds the fixed-
+    round output has not converged and eps-sized entries still move it, so they differ by up to
+    ~3e-2. The readings are not interchangeable at the 1e-5 coefficient tolerance."""
     gaps = {}
     for std, iters in ((1.0, 20), (3.0, 50)):
         logits = RNG.standard_normal((4000, 4, 4)) * std
         a = oracle.sinkhorn(logits, iters=iters, eps=1e-6)
-        b = oracle.sinkhorn_entry_eps(logits, iters=iters, eps=1e-6)
-        gaps[(std, iters)] = float(np.max(np.abs(a - b)))
+        for v in (1, 2):
+            b = oracle.sinkhorn_variant(logits, iters=iters, eps=1e-6, variant=v)
+            gaps[(std, iters, v)] = float(np.max(np.abs(a - b)))
     with capsys.disabled():
-        print(f"\n[sinkhorn reading gap] max|denominator-eps - entry-eps| = {gaps}")
-    assert gaps[(1.0, 20)] < 1e-4
-    assert gaps[(3.0, 50)] < 1e-1
+        print(f"\n[sinkhorn reading gap] max|oracle - variant| by (std, iters, variant) = {gaps}")
+    assert gaps[(1.0, 20, 1)] < 1e-4
+    assert gaps[(3.0, 50, 1)] < 1e-1
 
 
 # ----------------------------------------------------------------------------- norm + projection
