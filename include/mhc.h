@@ -33,7 +33,8 @@
  *   - All array pointers are DEVICE pointers into the current CUDA context's memory, dense and
  *     row-major; bf16 arrays are passed as their 16-bit patterns (uint16_t). The caller owns and
  *     allocates every buffer, including the pre-map workspace; the library allocates no device
- *     memory and keeps no state between calls.
+ *     memory and keeps no state between calls. The one exception is mhc_pre_noalloc, whose fixed
+ *     scratch array lives in the library's device image (see its comment).
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy default stream) and the call
  *     returns without synchronising. Results are ready when the stream reaches that point.
  *   - Arguments are validated on the host BEFORE anything is launched; on an error nothing is
@@ -186,6 +187,15 @@ MHC_API int mhc_post_with_path(const uint16_t* x, const uint16_t* R, const float
  * they give up (MHC_OK or MHC_ERR_TIMEOUT). Synchronises `stream` first. Kernels never trap. */
 MHC_API int mhc_device_status(mhc_stream_t stream);
 
+/* mhc_selftest_wait_timeout -- health check of the bounded device waits (no counterpart on the
+ * pages). Enqueues one kernel whose single thread waits on an mbarrier that nothing arrives at,
+ * through the same wait routine every pipeline uses, but with limit_ns (1 us .. 1 s) instead of the
+ * library-wide 2 s. The wait runs out, the kernel records MHC_ERR_TIMEOUT in the device status word
+ * and returns; no copy is in flight, so the context stays usable. A following mhc_device_status()
+ * returns MHC_ERR_TIMEOUT (and clears the word). Errors: MHC_ERR_INVALID_ARG (limit out of range),
+ * MHC_ERR_UNSUPPORTED (current device not sm_100), MHC_ERR_CUDA (launch failed). */
+MHC_API int mhc_selftest_wait_timeout(int64_t limit_ns, mhc_stream_t stream);
+
 /*
  * mhc_pre_noalloc -- mhc_pre for callers that cannot allocate device memory. No counterpart on the
  * pages: it is an addition of this library.
@@ -199,11 +209,14 @@ MHC_API int mhc_device_status(mhc_stream_t stream);
  * caller workspace. The caller still passes every input and output.
  *
  *   - Sizes whose scratch would exceed MHC_NOALLOC_SCRATCH_BYTES return MHC_ERR_SCRATCH_LIMIT
- *     before anything is launched (every T up to 16384 tokens fits for H up to 16392; other
- *     arguments and errors are those of mhc_pre). It calls no cudaMalloc, cudaFree or allocating library routine.
+ *     before anything is launched (every T up to 32768 tokens fits, whatever H; other arguments
+ *     and errors are those of mhc_pre). It calls no cudaMalloc, cudaFree or allocating library
+ *     routine.
  *   - The array exists on every GPU that loads the library and is held until the process exits.
- *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
- *     that device current) and caches it; make that first call before any stream capture.
+ *   - Every call looks up the array's device address (cudaGetSymbolAddress, with the device that
+ *     owns R current), so a reset device or a recreated context never leaves a stale address
+ *     behind. The first lookup on a device can load the library's module there: make the first
+ *     call on each device before any stream capture.
  *   - All calls on a device share the one array, which keeps the last call's contents; every record
  *     a call reads is written earlier in the same call, so nothing needs clearing. Calls whose
  *     kernels can overlap on the GPU (different streams without ordering between them) race on the

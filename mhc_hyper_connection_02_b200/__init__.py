@@ -44,7 +44,7 @@ EXPORTED_SYMBOLS = (
     "mhc_pre_big_fuse_with_prenorm", "mhc_expand", "mhc_head_mean", "mhc_head",
     "mhc_head_workspace_bytes", "mhc_post_project", "mhc_post_project_splits",
     "mhc_post_project_workspace_bytes", "mhc_post_backward", "mhc_pre_backward",
-    "mhc_pre_backward_workspace_bytes",
+    "mhc_pre_backward_workspace_bytes", "mhc_selftest_wait_timeout",
 )
 
 
@@ -93,6 +93,8 @@ def lib() -> ctypes.CDLL:
     L.mhc_sinkhorn.argtypes = [_P, _P, _I64, _I64, ctypes.c_int, ctypes.c_float, _P]
     L.mhc_device_status.restype = ctypes.c_int
     L.mhc_device_status.argtypes = [_P]
+    L.mhc_selftest_wait_timeout.restype = ctypes.c_int
+    L.mhc_selftest_wait_timeout.argtypes = [_I64, _P]
     L.mhc_status_string.restype = ctypes.c_char_p
     L.mhc_status_string.argtypes = [ctypes.c_int]
     L.mhc_version.restype = ctypes.c_int
@@ -482,6 +484,14 @@ def sinkhorn(logits, *, comb=None, iters: int = 20, eps: float = 1e-6, stream=No
 def device_status(stream=None) -> int:
     """Reads and clears the library's device-side status word (0, or MHC_ERR_TIMEOUT)."""
     return int(lib().mhc_device_status(_stream(stream)))
+
+
+def selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    """Enqueues the bounded-wait health check: a kernel whose wait nothing ends gives up after
+    limit_ns and records MHC_ERR_TIMEOUT in the device status word (read it with device_status)."""
+    st = lib().mhc_selftest_wait_timeout(int(limit_ns), _stream(stream))
+    if st != MHC_OK:
+        raise MhcError(st, "mhc_selftest_wait_timeout")
 
 
 def launch_count() -> int:

@@ -31,7 +31,48 @@ void query_device(int dev) {
 }
 }  // namespace
 
+namespace {
+struct SmemLimit {
+  const void* kernel;
+  int device;
+  int bytes;
+};
+constexpr int kMaxSmemLimits = 256;
+SmemLimit g_smem_limits[kMaxSmemLimits];
+int g_n_smem_limits = 0;
+std::mutex g_smem_mu;
+}  // namespace
+
+bool ensure_smem_limit(const void* kernel, int bytes) {
+  const int dev = current_device();
+  if (dev < 0) return false;
+  std::lock_guard<std::mutex> lock(g_smem_mu);
+  for (int i = 0; i < g_n_smem_limits; ++i)
+    if (g_smem_limits[i].kernel == kernel && g_smem_limits[i].device == dev &&
+        g_smem_limits[i].bytes >= bytes)
+      return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (g_n_smem_limits < kMaxSmemLimits) g_smem_limits[g_n_smem_limits++] = {kernel, dev, bytes};
+  return true;
+}
+
 static std::atomic<uint64_t> g_launches{0};
+
+// Health check of the bounded waits: one thread waits on an mbarrier that nothing arrives at, with
+// the caller's limit instead of the library-wide one, through the same wait routine the pipelines
+// use. No copy or MMA is in flight, so giving up leaves nothing behind.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbarrier_init();
+    mbar_wait_for(&bar, 0, 99, limit_ns);
+  }
+}
 void note_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
 
 int current_device() {
@@ -228,8 +269,9 @@ int mhc_pre_with_path(const uint16_t* R, const float* hc_fn, const float* hc_sca
             prm.sinkhorn_iters, prm.sinkhorn_eps, prm.rms_eps, prm.pre_eps, prm.post_mult};
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (path == MHC_PRE_PATH_TENSOR_FUSED) {
+    // 1: the grid cannot be co-scheduled on this device right now; nothing was launched.
     const int r = launch_pre_fused(a, s);
-    if (r <= 0) return r;  // 1: grid cannot be co-scheduled here, take the split pair
+    return r == 1 ? MHC_ERR_UNSUPPORTED : r;
   }
   if (path != MHC_PRE_PATH_CUDA_CORE) return launch_pre_tc(a, s);
   return launch_pre_cc(a, s);
@@ -502,6 +544,17 @@ int mhc_head(const uint16_t* R, const float* hc_fn, const float* hc_scale, const
   float* pre_out = weights ? weights : coef;
   return mhc_pre_with_path(R, fn24, sb, sb + 3, y, pre_out, coef + 4 * T, coef + 8 * T,
                            ws + l.pre_ws, l.pre_ws_bytes, T, H, &p, MHC_PATH_AUTO, stream);
+}
+
+int mhc_selftest_wait_timeout(int64_t limit_ns, mhc_stream_t stream) {
+  if (limit_ns < 1000 || limit_ns > 1000000000) return MHC_ERR_INVALID_ARG;
+  const int dev = current_device();
+  if (dev < 0) return MHC_ERR_CUDA;
+  if (device_cc() / 10 != 10) return MHC_ERR_UNSUPPORTED;
+  selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<unsigned long long>(limit_ns));
+  note_launches(1);
+  return cudaGetLastError() == cudaSuccess ? MHC_OK : MHC_ERR_CUDA;
 }
 
 int mhc_device_status(mhc_stream_t stream) {

@@ -740,15 +740,7 @@ int launch_pre_backward(const PreBwdArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return -4;
   // 5. d_R: column slices x token chunks, one wave of kDxSlotsPerSm CTAs per SM.
   if (vec) {
-    static bool attr_set[64] = {};
-    const int dev = current_device();
-    if (dev < 0) return -4;
-    if (!attr_set[dev]) {
-      if (cudaFuncSetAttribute(pre_bwd_dx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               kDxSmem) != cudaSuccess)
-        return -4;
-      attr_set[dev] = true;
-    }
+    if (!ensure_smem_limit(reinterpret_cast<const void*>(pre_bwd_dx_kernel), kDxSmem)) return -4;
     const int64_t xcols = (K + kDxCols - 1) / kDxCols;
     int64_t xch = (kDxSlotsPerSm * static_cast<int64_t>(device_sm_count())) / xcols;
     if (xch < 1) xch = 1;

@@ -126,20 +126,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Wait for the phase with the given parity to complete. Returns false (and records a timeout) if
-// it has not completed within kWaitLimitNs; the caller then stops using the pipeline.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int where) {
+// it has not completed within limit_ns; the caller then stops using the pipeline. Also returns
+// false once another wait has recorded a timeout.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, int where,
+                                              unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 255u) == 0) {
       if (*reinterpret_cast<volatile int*>(&g_device_status) != 0) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         report_timeout(where);
         return false;
       }
     }
   }
+}
+// The kernels' waits use the library-wide limit.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int where) {
+  return mbar_wait_for(bar, parity, where, kWaitLimitNs);
 }
 
 // 1-D bulk copy global -> shared (TMA engine), completion counted on `bar` in bytes. Both
@@ -151,6 +157,20 @@ __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, u
           smem_u32(smem_dst)),
       "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Named barrier over `nthreads` threads that also ORs a predicate: every participant gets the same
+// answer, so a decision taken on it (such as stopping after a timeout) keeps the barrier sequence
+// matched.
+__device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 
 // ------------------------------------------------------------------------------ coefficient math

@@ -38,6 +38,10 @@ int device_cc();
 // Counts kernel launches enqueued through the library (mhc_launch_count).
 void note_launches(int n);
 
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` on the current device, once per
+// (kernel, device); safe to call from several host threads. Returns false if the runtime refuses.
+bool ensure_smem_limit(const void* kernel, int bytes);
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Launchers return 0 or a negative MHC_ERR_* code.

@@ -281,15 +281,7 @@ int launch_post_scalar(const uint16_t* x, const uint16_t* R, const float* post, 
 int launch_post_persistent(const uint16_t* x, const uint16_t* R, const float* post,
                            const float* comb, uint16_t* out, int64_t T, int64_t H,
                            cudaStream_t s) {
-  static bool attr_set[64] = {};
-  const int dev = current_device();
-  if (dev < 0) return -4;
-  if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(post_persistent_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kPostSmem) != cudaSuccess)
-      return -4;
-    attr_set[dev] = true;
-  }
+  if (!ensure_smem_limit(reinterpret_cast<const void*>(post_persistent_kernel), kPostSmem)) return -4;
   const int64_t tiles = T * ((H + kPostChunk - 1) / kPostChunk);
   int64_t blocks = static_cast<int64_t>(device_sm_count()) * 3;  // 3 x 61 KB of stages per SM
   if (blocks > tiles) blocks = tiles;

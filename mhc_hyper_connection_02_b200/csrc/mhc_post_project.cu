@@ -434,15 +434,7 @@ int launch_post_project(const PostProjectArgs& a, cudaStream_t s) {
   uint16_t* Bw = static_cast<uint16_t*>(a.workspace);
   CUtensorMap mB;
   if (!make_map(&mB, Bw, K, 80, 80)) return -4;
-  static bool attr_set[64] = {};
-  const int dev = current_device();
-  if (dev < 0) return -4;
-  if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(post_project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kPpSmem) != cudaSuccess)
-      return -4;
-    attr_set[dev] = true;
-  }
+  if (!ensure_smem_limit(reinterpret_cast<const void*>(post_project_kernel), kPpSmem)) return -4;
   const int64_t sb = (K + 255) / 256;
   if (launch_pdl(pre_tc_split_kernel, dim3(static_cast<unsigned>(sb < 4096 ? sb : 4096)),
                  dim3(256), 0, s, a.hc_fn, Bw, K) != cudaSuccess)

@@ -25,7 +25,8 @@ namespace mhc {
 constexpr int kCcWarps = 8;
 constexpr int kCcTokens = 32;
 constexpr int kCcRec = 32;            // floats per (split, token) record: raw[24], ss, padding
-constexpr int64_t kCcPlanCtas = 592;  // target CTAs for the split plan (device independent)
+constexpr int64_t kCcPlanCtas = 148;  // target CTAs for the split plan (device independent)
+constexpr int kCcLoadBatch = 19;      // records a finish warp loads before adding (148 / 8 rounded up)
 constexpr int kAggCols = 2048;        // columns per aggregate block (256 threads x 8)
 
 struct CcPlan {
@@ -226,9 +227,19 @@ __global__ void __launch_bounds__(256) pre_cc_finish_kernel(
   const int64_t t = blockIdx.x;
   float v = 0.f;
   if (lane < 25) {
-    // Loads of 8 records in flight per step; the additions keep split order.
-#pragma unroll 8
-    for (int64_t s = warp; s < nsplit; s += kCcWarps) v += part[(s * T + t) * kCcRec + lane];
+    // Warp w adds the records of splits w, w + 8, w + 16, ... in that order. A batch of up to
+    // kCcLoadBatch of them is loaded before any is added, so one batch (all of them for the split
+    // counts the plan produces) costs one round trip to L2.
+    for (int64_t s0 = warp; s0 < nsplit; s0 += static_cast<int64_t>(kCcWarps) * kCcLoadBatch) {
+      float r[kCcLoadBatch];
+#pragma unroll
+      for (int i = 0; i < kCcLoadBatch; ++i) {
+        const int64_t s = s0 + static_cast<int64_t>(i) * kCcWarps;
+        r[i] = s < nsplit ? part[(s * T + t) * kCcRec + lane] : 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < kCcLoadBatch; ++i) v += r[i];
+    }
   }
   if (lane < 25) red[warp][lane] = v;
   __syncthreads();

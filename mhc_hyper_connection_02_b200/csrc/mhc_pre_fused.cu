@@ -1,161 +1,211 @@
-// mHC pre-map as one persistent kernel: projection on tcgen05, sum of squares, cross-CTA
-// reduction, coefficients (gates, Sinkhorn) and aggregate. Streaming R from HBM never waits for
-// the reduction.
+// mHC pre-map in one pass over R: a persistent kernel that projects each token tile on tcgen05
+// tensor cores, reduces the split partials across the CTAs of a group, forms the coefficients and
+// aggregates y while the tile is still in L2.
 //
-// Work split. The hidden dimension is cut into 64-column slices; CTA c of a group owns q
-// consecutive slices (all four streams of them: 4q blocks of the flattened K = 4H, so it can also
-// form y on those columns) and keeps that part of the split hc_fn operand (Bw, bf16 x3, see
-// mhc_pre_tc.cu) resident in shared memory. A group of NSG CTAs covers all of H; G groups take
-// token tiles of 128 round robin. Per tile, inside each CTA:
+// Work layout. R is the flattened [T][4H] matrix (k = i*H + h) cut into 64-wide K blocks. The
+// launch is NG groups of G CTAs (NG * G <= SM count, one CTA per SM, cooperative launch so that all
+// of them are resident together). CTA j of a group owns a fixed, contiguous range of K blocks (the
+// ranges of a group cover K once) and keeps that slice of hc_fn resident in shared memory for the
+// whole call as the MMA B operand: each weight split exactly into three bf16 terms hi + mid + lo
+// (B rows [hi 24 | mid 24 | lo 24 | 8 zero], 128-byte swizzle, as in mhc_pre_tc.cu). Group g takes
+// the token tiles (128 tokens) g, g + NG, g + 2 NG, ... in that order, and every CTA of the group
+// projects its K range of each of them. Per tile n of a group, inside a CTA:
 //
-//   warp 0      TMA, projection ring: R block [128 tokens x 64 columns] of one stream per 16 KB
-//               stage (128-byte swizzle, the MMA operand layout).
-//   warp 1      tcgen05.mma M=128 N=80 K=16 into one of two TMEM accumulators.
-//   warps 2-5   sum of squares of each token row from the projection stage; after the tile the
-//               accumulator (tcgen05.ld) becomes the split record [group][tile ring][token][c][32]
-//               = raw[24], ss; release-increment count[tile].
-//   warps 6-8   one tile in three each: once count[tile] == NSG, sum the NSG records of this
-//               CTA's tokens (t = c, c + NSG, ...) in a fixed order, write the pre gates and
-//               release-increment ready[tile]; then post and comb (Sinkhorn), off the critical path.
-//   warp 9      releases count[tile] once the record warps have written (one gpu-scope fence per
-//               tile, so the record warps never stall on it).
-//   warps 10-15 once ready[tile] == NSG: y = sum_i pre_i * R_i on this CTA's columns, re-reading
-//               the tile with ordinary 16-byte loads. It was streamed a few microseconds earlier, so
-//               these hit L2, and they use the SM's load path rather than the TMA engine, whose
-//               per-SM rate the projection stream already uses up.
+//   warp 0      TMA: one [128 x 64] R block per stage of a ring (128-byte swizzle). Before tile n
+//               it waits until this CTA's coefficients of tile n - D are done: that bounds how far
+//               the stream runs ahead of the aggregate, and so how much of R must stay in L2.
+//   warp 1      tcgen05.mma M=128 N=80 K=16 over the K range into one of two TMEM accumulators.
+//   warps 2-5   sum of squares of each token row from the same stages; after the tile, the
+//               accumulator (tcgen05.ld) gives the partial record rec[token][j] = raw[24], ss, and
+//               one thread release-increments the tile's counter.
+//   warps 6-7   (alternate tiles) once the counter reaches G: for the tokens this CTA owns in the
+//               tile (token l with (l + 128 n) mod G == j), sum the G partial records in a fixed
+//               order, form rstd, the logits, the gates and the Sinkhorn comb, write pre, post and
+//               comb, and hand pre to the aggregate warps through shared memory.
+//   warps 8-15  y = bf16_rn(sum_i pre_i R_i) for the owned tokens, re-reading their rows with
+//               16-byte loads. The tile came from HBM a few microseconds earlier and is still in
+//               L2, so HBM sees R once.
 //
-// Counters are zeroed by a kernel launched just before. All CTAs are co-resident (cooperative
-// launch, one CTA per SM) and every wait is bounded by time: on expiry the kernel records
-// MHC_ERR_TIMEOUT in the status word and winds down instead of waiting forever.
+// The tile counters are zeroed by a one-block kernel launched just before (programmatic dependent
+// launch). Every wait is bounded by time: on expiry the kernel records MHC_ERR_TIMEOUT in the device
+// status word and winds down (copies in flight are drained, TMEM is released after the last MMA).
 //
-// "FlashInfer mHC module deep dive" §3.4 (per-token phases: sum of squares and rstd, gates,
-// softmax and Sinkhorn rounds, vec8 aggregate) and §3.3 (split reduction of dot_mix / sqrsum);
-// glm5next_mhc.rs glm_hc_pre (mix then finish).
+// "FlashInfer mHC module deep dive" §3.3 (split reduction of dot_mix / sqrsum), §3.4 (per-token
+// phases: sum of squares and rstd, gates, softmax and Sinkhorn rounds, vec8 aggregate), §5.2;
+// glm5next_mhc.rs glm_hc_pre (mix, then finish).
 #include <cuda.h>
+
+#include <mutex>
 
 #include "mhc_device.cuh"
 #include "mhc_internal.h"
 
 namespace mhc {
 
-constexpr int kFuM = 128;
-constexpr int kFuN = 80;
-constexpr int kFuHS = 64;                        // columns per slice
-constexpr int kFuPBytes = kFuM * kFuHS * 2;      // 16384: projection stage
-constexpr int kFuBBytes = kFuN * kFuHS * 2;      // 10240: one Bw block
-constexpr int kFuMaxQ = 2;
-constexpr int kFuRing = 8;                       // tiles of split records in flight
-constexpr int kFuRec = 32;                       // floats per record
-constexpr int kFuCoefWarps = 3;                  // warps 6..8
-constexpr int kFuRelWarp = 9;
-constexpr int kFuAggWarp0 = 10;                  // warps 10..15
-constexpr int kFuAggThreads = 6 * 32;
-constexpr int kFuThreads = 512;
-constexpr int kFuTmemCols = 256;                 // two accumulators at columns 0 and 128
-constexpr int kFuSmsPlan = 148;                  // SM count the workspace plan assumes (B200)
-// Slices per CTA are chosen so that a group has at most this many CTAs: two tile groups then run
-// side by side on 148 SMs, a token's records are fewer, and each CTA has twice the time per tile.
-constexpr int kFuGroupCtas = 74;
-constexpr int kFuTot = 28;                       // floats per token total in shared memory
-constexpr int kFuBarBytes = 512;                // mbarriers and the TMEM address word
-constexpr int kFuMisc = kFuBarBytes + kFuCoefWarps * 8 * kFuTot * 4;  // + coefficient scratch
+constexpr int kFsM = 128;                    // tokens per tile (MMA M)
+constexpr int kFsN = 80;                     // 3 x 24 split columns + 8 zero rows
+constexpr int kFsKB = 64;                    // K per block: one 128-byte swizzled row
+constexpr int kFsABytes = kFsM * kFsKB * 2;  // 16384: one R block
+constexpr int kFsBBytes = kFsN * kFsKB * 2;  // 10240: one resident hc_fn block
+constexpr int kFsMaxNb = 13;                 // most resident K blocks per CTA
+constexpr int kFsMinG = 4;                   // fewest CTAs per group
+constexpr int kFsMaxOwn = kFsM / kFsMinG;    // most tokens a CTA owns in one tile
+constexpr int kFsMaxStages = 8;
+constexpr int kFsRec = 28;                   // floats per partial record (raw[24], ss, 3 zero)
+constexpr int kFsRing = 6;                   // tiles of records per group (>= 2 D)
+constexpr int kFsSlots = 4;                  // coefficient -> aggregate hand-over slots
+constexpr int kFsCoefWarps = 2;
+constexpr int kFsCoefWarp0 = 6;
+constexpr int kFsAggWarp0 = 8;
+constexpr int kFsAggWarps = 8;
+constexpr int kFsThreads = 512;
+constexpr int kFsTmemCols = 256;             // accumulators at columns 0 and 128
+constexpr int kFsMaxCtas = 148;              // most CTAs a plan uses (workspace sizing)
+constexpr int kFsSmemLimit = 227 * 1024;
+constexpr int kFsDefaultLag = 2;             // D
 
-// Ring depths by slices per CTA (shared memory: 1 KB alignment slack + rings + Bw + misc).
-__host__ __device__ constexpr int fu_pstages(int q) { return q == 1 ? 11 : 8; }
+// Shared-memory scratch after the rings: barriers, TMEM address, coefficient sums, hand-over.
+constexpr int kFsOffBars = 0;      // full[8] empty[8] afull[2] aempty[2] cfull[4] cempty[4] done
+constexpr int kFsOffTmem = 240;
+constexpr int kFsOffCsum = 256;    // float [kFsCoefWarps][8][kFsRec]
+constexpr int kFsOffPre = kFsOffCsum + kFsCoefWarps * 8 * kFsRec * 4;  // float [slots][own][4]
+constexpr int kFsOffTok = kFsOffPre + kFsSlots * kFsMaxOwn * 16;       // int [slots][own]
+constexpr int kFsOffNown = kFsOffTok + kFsSlots * kFsMaxOwn * 4;       // int [slots]
+constexpr int kFsMisc = (kFsOffNown + kFsSlots * 4 + 127) / 128 * 128;
 
-struct FuPlan {
-  int64_t ns;     // 64-column slices
-  int64_t q;      // slices per CTA
-  int64_t nsg;    // CTAs per group
-  int64_t ntiles;
-  int64_t gmax;   // most tile groups a launch may use (each has its own record ring)
-  size_t bw_bytes, cnt_off, part_off, total;
+struct FsPlan {
+  bool ok;
+  int64_t KB;      // K blocks
+  int64_t ntiles;  // token tiles
+  int G, NG;       // CTAs per group, groups
+  int nbmax;       // most K blocks of a CTA
+  int stages;      // R ring depth
+  int smem;        // dynamic shared memory bytes
+  size_t cnt_off, rec_off, total;
 };
 
-static FuPlan fu_plan(int64_t T, int64_t H) {
-  FuPlan p;
-  p.ns = (H + kFuHS - 1) / kFuHS;
-  p.q = (p.ns + kFuGroupCtas - 1) / kFuGroupCtas;
-  if (p.q > kFuMaxQ) p.q = (p.ns + kFuSmsPlan - 1) / kFuSmsPlan;  // wide H: one group
-  p.nsg = (p.ns + p.q - 1) / p.q;
-  p.ntiles = (T + kFuM - 1) / kFuM;
-  p.gmax = kFuSmsPlan / p.nsg;
-  if (p.gmax > p.ntiles) p.gmax = p.ntiles;
-  if (p.gmax < 1) p.gmax = 1;
-  p.bw_bytes = (static_cast<size_t>(kFuN) * 4 * H * 2 + 1023) / 1024 * 1024;
-  p.cnt_off = p.bw_bytes;
-  p.part_off = p.cnt_off + (static_cast<size_t>(2 * p.ntiles) * 4 + 255) / 256 * 256;
-  p.total = p.part_off + static_cast<size_t>(p.gmax) * kFuRing * kFuM * p.nsg * kFuRec * 4;
+static FsPlan fs_plan(int64_t T, int64_t H, int sms) {
+  FsPlan p{};
+  p.ok = false;
+  if (T < 1 || H < 8 || H % 8 != 0 || sms < kFsMinG) return p;
+  if (sms > kFsMaxCtas) sms = kFsMaxCtas;
+  const int64_t K = 4 * H;
+  p.KB = (K + kFsKB - 1) / kFsKB;
+  p.ntiles = (T + kFsM - 1) / kFsM;
+  if (p.ntiles > (int64_t(1) << 30)) return p;
+  int64_t G = (p.KB + kFsMaxNb - 1) / kFsMaxNb;
+  if (G < kFsMinG) G = kFsMinG;
+  if (G > sms || G > p.KB) return p;
+  int64_t NG = sms / G;
+  if (NG > p.ntiles) NG = p.ntiles;
+  G = sms / NG;  // spread the groups over every SM
+  if (G > p.KB) G = p.KB;
+  p.G = static_cast<int>(G);
+  p.NG = static_cast<int>(NG);
+  p.nbmax = static_cast<int>((p.KB + G - 1) / G);
+  if (p.nbmax > kFsMaxNb) return p;
+  const int fixed = 1024 + p.nbmax * kFsBBytes + kFsMisc;
+  int st = (kFsSmemLimit - fixed) / kFsABytes;
+  if (st > kFsMaxStages) st = kFsMaxStages;
+  if (st < 2) return p;
+  p.stages = st;
+  p.smem = fixed + st * kFsABytes;
+  p.cnt_off = 0;
+  p.rec_off = (static_cast<size_t>(p.ntiles) * 4 + 255) / 256 * 256;
+  p.total = p.rec_off + static_cast<size_t>(p.NG) * kFsRing * kFsM * p.G * kFsRec * 4;
+  p.ok = true;
   return p;
 }
 
-static int fu_smem_bytes(int q) {
-  return 1024 + fu_pstages(q) * kFuPBytes + 4 * q * kFuBBytes + kFuMisc;
-}
-
-bool pre_fused_supported(int64_t T, int64_t H) {
-  if (T < 1 || H < 8 || H % 8 != 0) return false;
-  const FuPlan p = fu_plan(T, H);
-  // At least 8 CTAs per group keeps a CTA's tokens per tile within two batches of 8.
-  return p.q <= kFuMaxQ && p.nsg >= 8 && p.ntiles <= (int64_t(1) << 30);
-}
+bool pre_fused_supported(int64_t T, int64_t H) { return fs_plan(T, H, kFsMaxCtas).ok; }
 
 size_t pre_fused_workspace_bytes(int64_t T, int64_t H) {
-  if (!pre_fused_supported(T, H)) return 0;
-  return fu_plan(T, H).total;
+  // The largest plan: records for every CTA of a full-size launch. Plans on devices with fewer SMs
+  // need no more.
+  const FsPlan p = fs_plan(T, H, kFsMaxCtas);
+  if (!p.ok) return 0;
+  return p.rec_off + static_cast<size_t>(kFsMaxCtas) * kFsRing * kFsM * kFsRec * 4;
 }
 
 // ------------------------------------------------------------------------------ device helpers
 
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
-                                            uint64_t* bar) {
+__device__ __forceinline__ void fs_tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                               uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
 }
 
-__device__ __forceinline__ int ld_acquire(const int* p) {
+__device__ __forceinline__ void fs_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fs_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t fs_desc(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
+         (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+         (static_cast<uint64_t>(2) << 61);
+}
+
+// Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major, M = 128, N = 80.
+constexpr uint32_t kFsIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                              (static_cast<uint32_t>(kFsN >> 3) << 17) |
+                              (static_cast<uint32_t>(kFsM >> 4) << 24);
+
+__device__ __forceinline__ void fs_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(kFsIdesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void fs_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void fs_tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ int fs_ld_acquire(const int* p) {
   int v;
   asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
-__device__ __forceinline__ void named_bar(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-// Named barrier that also ORs a predicate over the participating threads (every thread gets the
-// same answer, so decisions taken on it are uniform and barrier sequences stay matched).
-__device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
-      : "memory");
-  return r != 0;
-}
-// Release increment: everything this thread has observed (including, through CTA-scope
-// synchronisation, other threads' stores) is visible at gpu scope before the add.
-__device__ __forceinline__ void red_release_add(int* p, int v) {
+
+// Everything this thread has observed (including, through the CTA-scope barrier before it, the
+// other epilogue threads' record stores) is visible at gpu scope before the add.
+__device__ __forceinline__ void fs_red_release_add(int* p, int v) {
   asm volatile("fence.acq_rel.gpu;\n\tred.relaxed.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v)
                : "memory");
 }
-__device__ __forceinline__ bool status_set() {
-  return *reinterpret_cast<volatile int*>(&g_device_status) != 0;
-}
 
-// Waits until *p >= target; false on timeout (or once another wait has timed out).
-__device__ __noinline__ bool wait_count(const int* p, int target, int where) {
-  if (ld_acquire(p) >= target) return true;
-  if (status_set()) return false;
+// Waits until *p >= target (acquire); false on timeout or once another wait has timed out.
+__device__ __noinline__ bool fs_wait_count(const int* p, int target, int where) {
+  if (fs_ld_acquire(p) >= target) return true;
   const unsigned long long t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
-    __nanosleep(20);
-    if (ld_acquire(p) >= target) return true;
+    __nanosleep(32);
+    if (fs_ld_acquire(p) >= target) return true;
     if ((i & 63u) == 0) {
-      if (status_set()) return false;
+      if (*reinterpret_cast<volatile int*>(&g_device_status) != 0) return false;
       if (global_timer_ns() - t0 > kWaitLimitNs) {
         report_timeout(where);
         return false;
@@ -164,466 +214,510 @@ __device__ __noinline__ bool wait_count(const int* p, int target, int where) {
   }
 }
 
-struct FuArgs {
+// Streaming read of data this kernel does not write; L1 not allocated.
+__device__ __forceinline__ uint4 fs_ld_ro(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+struct FsArgs {
   const uint16_t* R;
+  const float* hc_fn;
   const float* scale;
   const float* base;
   uint16_t* y;
   float* pre;
   float* post;
   float* comb;
-  int* cnt;      // [ntiles]
-  int* ready;    // [ntiles]
-  float* part;   // [groups][kFuRing][128][nsg][32]
-  int64_t T, H;
-  int ntiles, nsg, q, groups;
+  int* cnt;    // [ntiles]
+  float* rec;  // [NG][kFsRing][128][G][kFsRec]
+  int64_t T, H, K;
+  int KB, ntiles, G, NG, nbmax, stages, lag;
   FinishParams fp;
 };
 
-// Sums the NSG records of one token into tot (28 floats in shared memory). The token's records
-// are contiguous (NSG x 128 bytes); lane l adds float4 number l, l+32, ...: component group l % 8
-// of records l/8, l/8 + 4, ... in increasing order, then a fixed xor tree joins the four lanes of
-// each group. The order is fixed, so every run gives the same sums.
-__device__ __forceinline__ void fu_reduce_token(const float* recs_f, int nsg, float* tot) {
-  const int lane = threadIdx.x & 31;
-  const float4* recs = reinterpret_cast<const float4*>(recs_f);
-  const int nf4 = nsg * (kFuRec / 4);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  constexpr int kU = 14;  // loads in flight per lane
-  for (int m0 = lane; m0 < nf4; m0 += 32 * kU) {
-    float4 v[kU];
-#pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int m = m0 + 32 * u;
-      v[u] = m < nf4 ? __ldcg(recs + m) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      acc.x += v[u].x;
-      acc.y += v[u].y;
-      acc.z += v[u].z;
-      acc.w += v[u].w;
-    }
-  }
-#pragma unroll
-  for (int sh = 8; sh <= 16; sh <<= 1) {
-    acc.x += __shfl_xor_sync(0xffffffffu, acc.x, sh);
-    acc.y += __shfl_xor_sync(0xffffffffu, acc.y, sh);
-    acc.z += __shfl_xor_sync(0xffffffffu, acc.z, sh);
-    acc.w += __shfl_xor_sync(0xffffffffu, acc.w, sh);
-  }
-  if (lane < kFuTot / 4) reinterpret_cast<float4*>(tot)[lane] = acc;
-}
-
-__global__ void __launch_bounds__(kFuThreads, 1) pre_fused_kernel(
-    const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmB,
-    const FuArgs a) {
+__global__ void __launch_bounds__(kFsThreads, 1)
+    pre_fused_kernel(const __grid_constant__ CUtensorMap tmR, const FsArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
-  const int nP = fu_pstages(a.q);
-  const int nkb = 4 * a.q;  // projection blocks (and aggregate stages) per tile
-  uint8_t* pring = smem;
-  uint8_t* bres = pring + nP * kFuPBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(bres + nkb * kFuBBytes);
-  uint64_t* pfull = bars;             // [11]
-  uint64_t* pempty = bars + 11;       // [11]
-  uint64_t* bfull = bars + 22;
-  uint64_t* dfull = bars + 23;        // [2]
-  uint64_t* dempty = bars + 25;       // [2]
-  uint64_t* mma_done = bars + 27;
-  uint64_t* recdone = bars + 28;      // [2] record warps -> warp 15
-  uint64_t* recfree = bars + 30;      // [2] warp 15 -> record warps
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 32);
-  float* coef_smem = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + kFuBarBytes);
-  static_assert(33 * 8 <= kFuBarBytes, "barrier area");
+  uint8_t* Bres = smem;                                       // nbmax resident hc_fn blocks
+  uint8_t* Aring = smem + a.nbmax * kFsBBytes;                // R ring
+  uint8_t* misc = Aring + a.stages * kFsABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(misc + kFsOffBars);
+  uint64_t* empty = full + kFsMaxStages;
+  uint64_t* afull = empty + kFsMaxStages;
+  uint64_t* aempty = afull + 2;
+  uint64_t* cfull = aempty + 2;
+  uint64_t* cempty = cfull + kFsSlots;
+  uint64_t* done = cempty + kFsSlots;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + kFsOffTmem);
+  float* csum = reinterpret_cast<float*>(misc + kFsOffCsum);
+  float* slot_pre = reinterpret_cast<float*>(misc + kFsOffPre);
+  int* slot_tok = reinterpret_cast<int*>(misc + kFsOffTok);
+  int* slot_nown = reinterpret_cast<int*>(misc + kFsOffNown);
+  static_assert((2 * kFsMaxStages + 4 + 2 * kFsSlots + 1) * 8 <= kFsOffTmem, "barrier area");
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int c = blockIdx.x % a.nsg;  // slice group within the tile group
-  const int g = blockIdx.x / a.nsg;  // tile group
-  const int h0 = c * a.q * kFuHS;    // first column of this CTA
-  const int64_t K = 4 * a.H;
+  const int G = a.G, NG = a.NG, ST = a.stages;
+  const int g = blockIdx.x / G;
+  const int j = blockIdx.x - g * G;
+  const int kb0 = static_cast<int>(static_cast<int64_t>(j) * a.KB / G);
+  const int nb = static_cast<int>(static_cast<int64_t>(j + 1) * a.KB / G) - kb0;
+  const int ntg = (a.ntiles - g + NG - 1) / NG;  // tiles of this group
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < nP; ++s) {
-      mbar_init(&pfull[s], 1);
-      mbar_init(&pempty[s], 1 + 4);  // MMA commit + one arrival per sum-of-squares warp
+    for (int s = 0; s < kFsMaxStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1 + 4);  // MMA commit + one arrival per sum-of-squares warp
     }
-    mbar_init(bfull, 1);
-    for (int d = 0; d < 2; ++d) {
-      mbar_init(&dfull[d], 1);
-      mbar_init(&dempty[d], 4);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&afull[b], 1);
+      mbar_init(&aempty[b], 4);
     }
-    mbar_init(mma_done, 1);
-    for (int d = 0; d < 2; ++d) {
-      mbar_init(&recdone[d], 4);
-      mbar_init(&recfree[d], 1);
+    for (int s = 0; s < kFsSlots; ++s) {
+      mbar_init(&cfull[s], 1);
+      mbar_init(&cempty[s], kFsAggWarps);
     }
+    mbar_init(done, 1);
     fence_mbarrier_init();
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
-                 "r"(kFuTmemCols)
+                 "r"(kFsTmemCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  tc_fence_before();
+  pdl_wait();  // the counters were zeroed by the grid launched just before
+  pdl_trigger();
+
+  // Resident B operand: hc_fn rows [kb0 * 64, (kb0 + nb) * 64) split into three exact bf16 terms.
+  // Tile b holds rows r = 0..79 of 128 bytes; the 16-byte chunk c (k = 8c .. 8c + 7) of row r sits
+  // at chunk position c ^ (r & 7) (the 128-byte swizzle the MMA descriptor names).
+  {
+    const int items = nb * 8 * kMix;
+    for (int i = threadIdx.x; i < items; i += kFsThreads) {
+      const int col = i % kMix;
+      const int rest = i / kMix;
+      const int c = rest & 7;
+      const int b = rest >> 3;
+      const int64_t k0 = static_cast<int64_t>(kb0 + b) * kFsKB + c * 8;
+      uint32_t hi[4], mid[4], lo[4];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        uint16_t h2[2], m2[2], l2[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int64_t k = k0 + e + u;
+          const float w = k < a.K ? __ldg(a.hc_fn + k * kMix + col) : 0.f;
+          h2[u] = f32_to_bf16(w);
+          const float r1 = w - bf16_to_f32(h2[u]);
+          m2[u] = f32_to_bf16(r1);
+          const float r2 = r1 - bf16_to_f32(m2[u]);
+          l2[u] = f32_to_bf16(r2);
+        }
+        hi[e / 2] = static_cast<uint32_t>(h2[0]) | (static_cast<uint32_t>(h2[1]) << 16);
+        mid[e / 2] = static_cast<uint32_t>(m2[0]) | (static_cast<uint32_t>(m2[1]) << 16);
+        lo[e / 2] = static_cast<uint32_t>(l2[0]) | (static_cast<uint32_t>(l2[1]) << 16);
+      }
+      uint8_t* tile = Bres + b * kFsBBytes;
+      const int r0 = col, r1 = kMix + col, r2 = 2 * kMix + col;
+      *reinterpret_cast<uint4*>(tile + r0 * 128 + ((c ^ (r0 & 7)) << 4)) =
+          make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(tile + r1 * 128 + ((c ^ (r1 & 7)) << 4)) =
+          make_uint4(mid[0], mid[1], mid[2], mid[3]);
+      *reinterpret_cast<uint4*>(tile + r2 * 128 + ((c ^ (r2 & 7)) << 4)) =
+          make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+    for (int i = threadIdx.x; i < nb * 8 * 8; i += kFsThreads) {  // rows 72..79: zero
+      const int b = i >> 6;
+      const int r = 3 * kMix + ((i >> 3) & 7);
+      *reinterpret_cast<uint4*>(Bres + b * kFsBBytes + r * 128 + ((i & 7) << 4)) =
+          make_uint4(0u, 0u, 0u, 0u);
+    }
+    // Generic-proxy writes become visible to the tensor cores' (async proxy) reads.
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  fs_fence_before();
   __syncthreads();
-  tc_fence_after();
+  fs_fence_after();
   const uint32_t tmem = *tmem_slot;
+  float* const rec_g = a.rec + static_cast<size_t>(g) * kFsRing * kFsM * G * kFsRec;
 
   if (warp == 0) {
-    // ---------------------------------------------------------------- projection TMA
+    // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      mbar_arrive_expect_tx(bfull, nkb * kFuBBytes);
-      for (int kb = 0; kb < nkb; ++kb)
-        tma_load_3d(bres + kb * kFuBBytes, &tmB, h0 + (kb >> 2) * kFuHS, kb & 3, 0, bfull);
-      int64_t n = 0;
+      int64_t it = 0;
       bool ok = true;
-      for (int j = g; j < a.ntiles && ok; j += a.groups) {
-        for (int kb = 0; kb < nkb; ++kb, ++n) {
-          const int s = static_cast<int>(n % nP);
-          const uint32_t ph = static_cast<uint32_t>(n / nP) & 1u;
-          if (n >= nP && !mbar_wait(&pempty[s], ph ^ 1u, 20)) {
+      for (int n = 0; n < ntg && ok; ++n) {
+        if (n >= a.lag) {
+          const int m = n - a.lag;
+          if (!mbar_wait(&cfull[m % kFsSlots], static_cast<uint32_t>(m / kFsSlots) & 1u, 40)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&pfull[s], kFuPBytes);
-          tma_load_3d(pring + s * kFuPBytes, &tmR, h0 + (kb >> 2) * kFuHS, kb & 3, j * kFuM,
-                      &pfull[s]);
+        }
+        const int X = g + n * NG;
+        for (int b = 0; b < nb; ++b, ++it) {
+          const int s = static_cast<int>(it % ST);
+          const uint32_t ph = static_cast<uint32_t>(it / ST) & 1u;
+          if (it >= ST && !mbar_wait(&empty[s], ph ^ 1u, 41)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], kFsABytes);
+          fs_tma_load_2d(Aring + s * kFsABytes, &tmR, (kb0 + b) * kFsKB, X * kFsM, &full[s]);
         }
       }
-      // Never leave with copies into shared memory in flight.
-      mbar_wait(bfull, 0, 21);
-      for (int64_t i = n - nP; i < n; ++i)
-        if (i >= 0) mbar_wait(&pfull[i % nP], static_cast<uint32_t>(i / nP) & 1u, 22);
+      if (!ok) {  // do not leave while copies into shared memory are in flight
+        for (int64_t i = it - ST; i < it; ++i)
+          if (i >= 0) mbar_wait(&full[i % ST], static_cast<uint32_t>(i / ST) & 1u, 42);
+      }
     }
   } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
+    // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      bool ok = mbar_wait(bfull, 0, 23);
-      int64_t n = 0;
-      int it = 0;
-      for (int j = g; j < a.ntiles && ok; j += a.groups, ++it) {
-        const int d = it & 1;
-        if (it >= 2 && !mbar_wait(&dempty[d], static_cast<uint32_t>((it >> 1) - 1) & 1u, 24)) {
+      int64_t it = 0;
+      bool ok = true;
+      for (int n = 0; n < ntg && ok; ++n) {
+        const int b = n & 1;
+        if (n >= 2 && !mbar_wait(&aempty[b], static_cast<uint32_t>((n >> 1) - 1) & 1u, 43)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        const uint32_t dtm = tmem + static_cast<uint32_t>(d * 128);
-        for (int kb = 0; kb < nkb; ++kb, ++n) {
-          const int s = static_cast<int>(n % nP);
-          const uint32_t ph = static_cast<uint32_t>(n / nP) & 1u;
-          if (!mbar_wait(&pfull[s], ph, 25)) {
+        fs_fence_after();
+        const uint32_t dt = tmem + static_cast<uint32_t>(b * 128);
+        for (int kb = 0; kb < nb; ++kb, ++it) {
+          const int s = static_cast<int>(it % ST);
+          const uint32_t ph = static_cast<uint32_t>(it / ST) & 1u;
+          if (!mbar_wait(&full[s], ph, 44)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint64_t adesc = sw128_desc(smem_u32(pring + s * kFuPBytes));
-          const uint64_t bdesc = sw128_desc(smem_u32(bres + kb * kFuBBytes));
+          fs_fence_after();
+          const uint64_t adesc = fs_desc(smem_u32(Aring + s * kFsABytes));
+          const uint64_t bdesc = fs_desc(smem_u32(Bres + kb * kFsBBytes));
 #pragma unroll
-          for (int k = 0; k < kFuHS / 16; ++k)
-            umma_bf16(dtm, adesc + 2 * k, bdesc + 2 * k, (kb > 0 || k > 0) ? 1u : 0u);
-          umma_commit(&pempty[s]);
+          for (int k = 0; k < kFsKB / 16; ++k)  // +32 bytes along the swizzled row per K=16 step
+            fs_mma(dt, adesc + 2 * k, bdesc + 2 * k, (kb > 0 || k > 0) ? 1u : 0u);
+          fs_commit(&empty[s]);
         }
-        umma_commit(&dfull[d]);
+        if (!ok) break;
+        fs_commit(&afull[b]);
       }
       // Every issued MMA has finished before TMEM is released.
-      umma_commit(mma_done);
-      mbar_wait(mma_done, 0, 31);
+      fs_commit(done);
+      mbar_wait(done, 0, 45);
     }
-  } else if (warp < 6) {
-    // ---------------------------------------------------------------- sum of squares + records
-    // Loops never leave early: after a failed wait a thread only skips work, so the four warps
-    // always meet the same named barriers; the barrier's OR makes a failure uniform.
-    const int qd = warp & 3;
-    const int row = qd * 32 + lane;
-    int64_t n = 0;
-    int it = 0;
-    bool dead = false;
-    for (int j = g; j < a.ntiles; j += a.groups, ++it) {
+  } else if (warp < kFsCoefWarp0) {
+    // ------------------------------------------------------------------ sum of squares + records
+    // TMEM lane quarter q = warp % 4 holds accumulator rows 32q .. 32q + 31.
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    int64_t it = 0;
+    for (int n = 0; n < ntg; ++n) {
+      const int X = g + n * NG;
+      bool ok = true;
       float ss0 = 0.f, ss1 = 0.f;
-      for (int kb = 0; kb < nkb; ++kb, ++n) {
-        const int s = static_cast<int>(n % nP);
-        const uint32_t ph = static_cast<uint32_t>(n / nP) & 1u;
-        if (!dead) dead = !__all_sync(0xffffffffu, mbar_wait(&pfull[s], ph, 26));
-        if (dead) continue;
+      for (int kb = 0; kb < nb; ++kb, ++it) {
+        const int s = static_cast<int>(it % ST);
+        const uint32_t ph = static_cast<uint32_t>(it / ST) & 1u;
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, 46))) {
+          ok = false;
+          break;
+        }
         // Row `row` of the swizzled block is its own 128 contiguous bytes (chunks permuted within
-        // it), and a sum does not depend on element order. Each lane starts at a different 16-byte
-        // chunk, so the 8 lanes of a load phase hit 8 different bank groups.
-        const uint4* rp = reinterpret_cast<const uint4*>(pring + s * kFuPBytes + row * 128);
+        // it); a sum does not depend on the order. Lanes start at different chunks.
+        const uint4* rp = reinterpret_cast<const uint4*>(Aring + s * kFsABytes + row * 128);
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc) {
-          const uint4 v = rp[cc ^ (lane & 7)];
-          const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+          const uint4 w = rp[cc ^ (lane & 7)];
+          const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float x0 = bf16_lo(u[e]), x1 = bf16_hi(u[e]);
+            const float x0 = bf16_lo(w4[e]), x1 = bf16_hi(w4[e]);
             ss0 = fmaf(x0, x0, ss0);
             ss1 = fmaf(x1, x1, ss1);
           }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&pempty[s]);
+        if (lane == 0) mbar_arrive(&empty[s]);
       }
-      const int d = it & 1;
-      if (!dead)
-        dead = !__all_sync(0xffffffffu,
-                           mbar_wait(&dfull[d], static_cast<uint32_t>(it >> 1) & 1u, 27));
-      uint32_t dr[5][16];
-      if (!dead) {
-        tc_fence_after();
-        const uint32_t tb =
-            tmem + static_cast<uint32_t>(d * 128) + (static_cast<uint32_t>(qd * 32) << 16);
+      const int b = n & 1;
+      if (ok && !__all_sync(0xffffffffu,
+                            mbar_wait(&afull[b], static_cast<uint32_t>(n >> 1) & 1u, 47)))
+        ok = false;
+      if (ok) {
+        fs_fence_after();
+        uint32_t d[5][16];
+        const uint32_t tbase = tmem + static_cast<uint32_t>(b * 128) +
+                               (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll
-        for (int cc = 0; cc < 5; ++cc) tmem_ld16(tb + cc * 16, dr[cc]);
-        tmem_wait_ld();
-        tc_fence_before();
+        for (int cc = 0; cc < 5; ++cc) fs_tmem_ld16(tbase + cc * 16, d[cc]);
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        const int64_t t = static_cast<int64_t>(X) * kFsM + row;
+        if (t < a.T) {
+          float raw[kMix];
+#pragma unroll
+          for (int c = 0; c < kMix; ++c) {
+            const float hi3 = __uint_as_float(d[c / 16][c % 16]);
+            const float mid = __uint_as_float(d[(kMix + c) / 16][(kMix + c) % 16]);
+            const float lo3 = __uint_as_float(d[(2 * kMix + c) / 16][(2 * kMix + c) % 16]);
+            raw[c] = (lo3 + mid) + hi3;
+          }
+          float4* r4 = reinterpret_cast<float4*>(
+              rec_g + ((static_cast<size_t>(n % kFsRing) * kFsM + row) * G + j) * kFsRec);
+#pragma unroll
+          for (int w = 0; w < 6; ++w)
+            r4[w] = make_float4(raw[4 * w], raw[4 * w + 1], raw[4 * w + 2], raw[4 * w + 3]);
+          r4[6] = make_float4(ss0 + ss1, 0.f, 0.f, 0.f);
+        }
+        fs_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&dempty[d]);
+        if (lane == 0) mbar_arrive(&aempty[b]);
       }
-      // Ring slot reuse: the records of tile j - kFuRing*groups must have been consumed.
-      bool w = true;
-      if (it >= kFuRing && threadIdx.x == 64 && !dead)
-        w = wait_count(&a.ready[j - kFuRing * a.groups], a.nsg, 28);
-      dead = named_bar_or(1, 128, dead || !w);
-      const int64_t t = static_cast<int64_t>(j) * kFuM + row;
-      if (!dead && t < a.T) {
-        const int64_t slot = static_cast<int64_t>(g) * kFuRing + it % kFuRing;
-        float* rec = a.part + ((slot * kFuM + row) * a.nsg + c) * kFuRec;
-        float raw[kMix];
-#pragma unroll
-        for (int jj = 0; jj < kMix; ++jj) {
-          const float hi = __uint_as_float(dr[jj / 16][jj % 16]);
-          const float mi = __uint_as_float(dr[(kMix + jj) / 16][(kMix + jj) % 16]);
-          const float lo = __uint_as_float(dr[(2 * kMix + jj) / 16][(2 * kMix + jj) % 16]);
-          raw[jj] = (lo + mi) + hi;
-        }
-        float4* r4 = reinterpret_cast<float4*>(rec);
-#pragma unroll
-        for (int v = 0; v < 6; ++v)
-          r4[v] = make_float4(raw[4 * v], raw[4 * v + 1], raw[4 * v + 2], raw[4 * v + 3]);
-        r4[6] = make_float4(ss0 + ss1, 0.f, 0.f, 0.f);
-      }
-      // Hand the tile to warp 15, which releases count[tile]. Its 2-slot ring is guarded by
-      // recfree so that a slot's phase is consumed before it is armed again.
-      const int rs = it & 1;
-      if (it >= 2 && !dead)
-        dead = !__all_sync(0xffffffffu,
-                           mbar_wait(&recfree[rs], static_cast<uint32_t>((it >> 1) - 1) & 1u, 36));
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&recdone[rs]);
+      // The four warps agree on going on (a matched barrier sequence even after a timeout), and
+      // their records are published with one release-increment of the tile's counter.
+      if (named_bar_or(1, 128, !ok)) break;
+      if (warp == 2 && lane == 0) fs_red_release_add(a.cnt + X, 1);
     }
-  } else if (warp < 6 + kFuCoefWarps) {
-    // ---------------------------------------------------------------- coefficients
-    // Warp cw takes every kFuCoefWarps-th tile of this CTA; no barrier ties the coefficient warps
-    // together. For a tile: sum the records of this CTA's tokens (at most 16: NSG >= 8), write the
-    // pre gates, signal ready (the aggregate needs only those), then post and comb. Lane quad k
-    // handles token k of a batch of 8; lane r of the quad owns row r of comb.
-    const int cw = warp - 6;
-    float* tot_s = coef_smem + cw * 8 * kFuTot;
-    int it = 0;
-    bool dead = false;
-    for (int j = g; j < a.ntiles; j += a.groups, ++it) {
-      if (it % kFuCoefWarps != cw) continue;
-      bool w = true;
-      if (lane == 0 && !dead) w = wait_count(&a.cnt[j], a.nsg, 29);
-      dead = dead || !__all_sync(0xffffffffu, w);
-      const int64_t slot = static_cast<int64_t>(g) * kFuRing + it % kFuRing;
-      int ntok = 0;  // this CTA's tokens in the tile: tl = c + k*NSG
-      for (int tl = c; tl < kFuM && static_cast<int64_t>(j) * kFuM + tl < a.T; tl += a.nsg) ++ntok;
-      const int nbatch = (ntok + 7) / 8;
-      for (int pass = 0; pass < 2 && !dead; ++pass) {
-        for (int b = 0; b < nbatch; ++b) {
-          const int nk = min(8, ntok - 8 * b);
-          // A single batch keeps its sums from the first pass.
-          if (pass == 0 || nbatch > 1) {
-            for (int k = 0; k < nk; ++k) {
-              const int tl = c + (8 * b + k) * a.nsg;
-              fu_reduce_token(a.part + (slot * kFuM + tl) * a.nsg * kFuRec, a.nsg,
-                              tot_s + k * kFuTot);
+  } else if (warp < kFsAggWarp0) {
+    // ------------------------------------------------------------------ coefficients
+    const int cw = warp - kFsCoefWarp0;
+    float* cs = csum + cw * 8 * kFsRec;
+    const int quad = lane >> 2;
+    const int r = lane & 3;
+    for (int n = cw; n < ntg; n += kFsCoefWarps) {
+      const int X = g + n * NG;
+      const int slot = n % kFsSlots;
+      if (n >= kFsSlots &&
+          !__all_sync(0xffffffffu, mbar_wait(&cempty[slot],
+                                             static_cast<uint32_t>(n / kFsSlots - 1) & 1u, 48)))
+        break;
+      if (!__all_sync(0xffffffffu, fs_wait_count(a.cnt + X, G, 49))) break;
+      const float* recs = rec_g + static_cast<size_t>(n % kFsRing) * kFsM * G * kFsRec;
+      // Owned tokens: l = l0, l0 + G, ... below lim.
+      const int l0 = static_cast<int>(((j - (static_cast<int64_t>(n) * kFsM) % G) % G + G) % G);
+      const int64_t lim64 = a.T - static_cast<int64_t>(X) * kFsM;
+      const int lim = lim64 < kFsM ? static_cast<int>(lim64) : kFsM;
+      const int nown = l0 < lim ? (lim - l0 + G - 1) / G : 0;
+      for (int p0 = 0; p0 < nown; p0 += 8) {
+        const int np = nown - p0 < 8 ? nown - p0 : 8;
+        // Sum each token's G records: lane l adds records l, l + 32, ... (all 28 floats of each,
+        // in that order), then a fixed xor tree joins the lanes. Same order on every run.
+        for (int k = 0; k < np; ++k) {
+          const int l = l0 + (p0 + k) * G;
+          const float4* rt = reinterpret_cast<const float4*>(recs + static_cast<size_t>(l) * G *
+                                                                         kFsRec);
+          float acc[kFsRec];
+#pragma unroll
+          for (int c = 0; c < kFsRec; ++c) acc[c] = 0.f;
+          for (int rr = lane; rr < G; rr += 32) {
+            float4 v[7];
+#pragma unroll
+            for (int c = 0; c < 7; ++c) v[c] = __ldcg(rt + rr * 7 + c);
+#pragma unroll
+            for (int c = 0; c < 7; ++c) {
+              acc[4 * c] += v[c].x;
+              acc[4 * c + 1] += v[c].y;
+              acc[4 * c + 2] += v[c].z;
+              acc[4 * c + 3] += v[c].w;
             }
-            __syncwarp();
           }
-          const int k = lane >> 2;
-          const int r = lane & 3;
-          const bool live = k < nk;
-          const float* tt = tot_s + (live ? k : 0) * kFuTot;
-          const int64_t t = static_cast<int64_t>(j) * kFuM + c + (8 * b + (live ? k : 0)) * a.nsg;
+#pragma unroll
+          for (int sh = 16; sh >= 1; sh >>= 1) {
+#pragma unroll
+            for (int c = 0; c < 25; ++c) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], sh);
+          }
+          if (lane == 0) {
+#pragma unroll
+            for (int c = 0; c < 25; ++c) cs[k * kFsRec + c] = acc[c];
+          }
+        }
+        __syncwarp();
+        // Quad `quad` forms token p0 + quad's coefficients; lane r: pre r, post r, comb row r.
+        const bool live = quad < np;
+        const int l = l0 + (p0 + quad) * G;
+        const int64_t t = static_cast<int64_t>(X) * kFsM + l;
+        float cr[4] = {0.f, 0.f, 0.f, 0.f};
+        float pre_v = 0.f, post_v = 0.f;
+        if (live) {
+          const float* sm = cs + quad * kFsRec;
           const float rstd = __fdiv_rn(
-              1.0f, __fsqrt_rn(__fdiv_rn(tt[24], static_cast<float>(K)) + a.fp.rms_eps));
-          if (pass == 0) {
-            const float lp = fmaf(tt[r] * rstd, __ldg(a.scale), __ldg(a.base + r));
-            if (live) a.pre[t * 4 + r] = sigmoidf_ieee(lp) + a.fp.pre_eps;
-          } else {
-            const float lq = fmaf(tt[4 + r] * rstd, __ldg(a.scale + 1), __ldg(a.base + 4 + r));
-            float cr[4];
+              1.0f, __fsqrt_rn(__fdiv_rn(sm[24], static_cast<float>(a.K)) + a.fp.rms_eps));
+          const float lp = fmaf(sm[r] * rstd, __ldg(a.scale), __ldg(a.base + r));
+          const float lq = fmaf(sm[4 + r] * rstd, __ldg(a.scale + 1), __ldg(a.base + 4 + r));
+          const float s2 = __ldg(a.scale + 2);
 #pragma unroll
-            for (int nn = 0; nn < 4; ++nn)
-              cr[nn] = fmaf(tt[8 + 4 * r + nn] * rstd, __ldg(a.scale + 2),
-                            __ldg(a.base + 8 + 4 * r + nn));
-            sinkhorn_quad(cr, a.fp.iters, a.fp.sinkhorn_eps);  // every lane takes part
-            if (live) {
-              a.post[t * 4 + r] = a.fp.post_mult * sigmoidf_ieee(lq);
-              *reinterpret_cast<float4*>(a.comb + t * 16 + r * 4) =
-                  make_float4(cr[0], cr[1], cr[2], cr[3]);
+          for (int c = 0; c < 4; ++c)
+            cr[c] = fmaf(sm[8 + 4 * r + c] * rstd, s2, __ldg(a.base + 8 + 4 * r + c));
+          pre_v = sigmoidf_ieee(lp) + a.fp.pre_eps;
+          post_v = a.fp.post_mult * sigmoidf_ieee(lq);
+        }
+        sinkhorn_quad(cr, a.fp.iters, a.fp.sinkhorn_eps);  // every lane takes part
+        if (live) {
+          a.pre[t * 4 + r] = pre_v;
+          a.post[t * 4 + r] = post_v;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) a.comb[t * 16 + 4 * r + c] = cr[c];
+          slot_pre[(slot * kFsMaxOwn + p0 + quad) * 4 + r] = pre_v;
+          if (r == 0) slot_tok[slot * kFsMaxOwn + p0 + quad] = l;
+        }
+        __syncwarp();
+      }
+      if (lane == 0) {
+        slot_nown[slot] = nown;
+        mbar_arrive(&cfull[slot]);  // release: the hand-over entries above are visible
+      }
+      __syncwarp();
+    }
+  } else {
+    // ------------------------------------------------------------------ aggregate
+    const int at = threadIdx.x - kFsAggWarp0 * 32;
+    constexpr int kAggThreads = kFsAggWarps * 32;
+    const int64_t H = a.H;
+    const int64_t H8 = H / 8;
+    for (int n = 0; n < ntg; ++n) {
+      const int X = g + n * NG;
+      const int slot = n % kFsSlots;
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(&cfull[slot], static_cast<uint32_t>(n / kFsSlots) & 1u, 50)))
+        break;
+      const int nown = slot_nown[slot];
+      const int64_t units = static_cast<int64_t>(nown) * H8;
+      for (int64_t u0 = at; u0 < units; u0 += 4 * kAggThreads) {
+        uint4 rv[4][4];
+        uint16_t* yp[4];
+        float4 pp[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int64_t u = u0 + e * kAggThreads;
+          yp[e] = nullptr;
+          if (u < units) {
+            const int k = static_cast<int>(u / H8);
+            const int64_t v = u - k * H8;
+            const int64_t t = static_cast<int64_t>(X) * kFsM + slot_tok[slot * kFsMaxOwn + k];
+            pp[e] = *reinterpret_cast<const float4*>(slot_pre + (slot * kFsMaxOwn + k) * 4);
+            const uint16_t* rr = a.R + t * 4 * H + v * 8;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) rv[e][i] = fs_ld_ro(rr + i * H);
+            yp[e] = a.y + t * H + v * 8;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (yp[e] != nullptr) {
+            const uint32_t* r0 = &rv[e][0].x;
+            const uint32_t* r1 = &rv[e][1].x;
+            const uint32_t* r2 = &rv[e][2].x;
+            const uint32_t* r3 = &rv[e][3].x;
+            const float4 p4 = pp[e];
+            uint32_t o[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              float lo = p4.x * bf16_lo(r0[c]);
+              lo = fmaf(p4.y, bf16_lo(r1[c]), lo);
+              lo = fmaf(p4.z, bf16_lo(r2[c]), lo);
+              lo = fmaf(p4.w, bf16_lo(r3[c]), lo);
+              float hi = p4.x * bf16_hi(r0[c]);
+              hi = fmaf(p4.y, bf16_hi(r1[c]), hi);
+              hi = fmaf(p4.z, bf16_hi(r2[c]), hi);
+              hi = fmaf(p4.w, bf16_hi(r3[c]), hi);
+              o[c] = pack_bf16x2(lo, hi);
             }
+            st_stream(yp[e], make_uint4(o[0], o[1], o[2], o[3]));
           }
-          __syncwarp();
-        }
-        if (pass == 0) {
-          __syncwarp();
-          if (lane == 0) red_release_add(&a.ready[j], 1);
         }
       }
-    }
-  } else if (warp >= kFuAggWarp0) {
-    // ---------------------------------------------------------------- aggregate
-    // Units of 8 columns: e = 8q * token + column group. Thread `at` takes units at, at + 192, ...
-    // in batches of 4 (all loads of a batch in flight before any use), so a warp reads 4 tokens x
-    // 128 q bytes of each stream per load instruction.
-    const int at = threadIdx.x - kFuAggWarp0 * 32;
-    const int upt = 8 * a.q;
-    const int units = kFuM * upt;
-    bool dead = false;
-    for (int j = g; j < a.ntiles; j += a.groups) {
-      bool w = true;
-      if (at == 0 && !dead) w = wait_count(&a.ready[j], a.nsg, 30);
-      dead = named_bar_or(3, kFuAggThreads, dead || !w);
-      if (dead) continue;
-      constexpr int kB = 4;
-      for (int e0 = at; e0 < units; e0 += kB * kFuAggThreads) {
-        uint4 r[kB][4];
-        float4 p4[kB];
-        int64_t tok[kB];
-        int hc[kB];
-#pragma unroll
-        for (int u = 0; u < kB; ++u) {
-          const int e = e0 + u * kFuAggThreads;
-          const int tl = e / upt;
-          const int hcol = h0 + (e - tl * upt) * 8;
-          const int64_t t = static_cast<int64_t>(j) * kFuM + tl;
-          hc[u] = hcol;
-          tok[u] = (e < units && t < a.T && hcol < a.H) ? t : -1;
-          if (tok[u] < 0) continue;
-          p4[u] = __ldcg(reinterpret_cast<const float4*>(a.pre + t * 4));
-          const uint16_t* rr = a.R + t * 4 * a.H + hcol;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) r[u][i] = __ldg(reinterpret_cast<const uint4*>(rr + i * a.H));
-        }
-#pragma unroll
-        for (int u = 0; u < kB; ++u) {
-          if (tok[u] < 0) continue;
-          const float p[4] = {p4[u].x, p4[u].y, p4[u].z, p4[u].w};
-          const uint32_t* r0 = &r[u][0].x;
-          const uint32_t* r1 = &r[u][1].x;
-          const uint32_t* r2 = &r[u][2].x;
-          const uint32_t* r3 = &r[u][3].x;
-          uint32_t o[4];
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            float lo = p[0] * bf16_lo(r0[v]);
-            lo = fmaf(p[1], bf16_lo(r1[v]), lo);
-            lo = fmaf(p[2], bf16_lo(r2[v]), lo);
-            lo = fmaf(p[3], bf16_lo(r3[v]), lo);
-            float hi = p[0] * bf16_hi(r0[v]);
-            hi = fmaf(p[1], bf16_hi(r1[v]), hi);
-            hi = fmaf(p[2], bf16_hi(r2[v]), hi);
-            hi = fmaf(p[3], bf16_hi(r3[v]), hi);
-            o[v] = pack_bf16x2(lo, hi);
-          }
-          *reinterpret_cast<uint4*>(a.y + tok[u] * a.H + hc[u]) = make_uint4(o[0], o[1], o[2], o[3]);
-        }
-      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&cempty[slot]);
     }
   }
-  if (warp == kFuRelWarp && lane == 0) {
-    // ---------------------------------------------------------------- count release
-    int it = 0;
-    for (int j = g; j < a.ntiles; j += a.groups, ++it) {
-      const int rs = it & 1;
-      if (!mbar_wait(&recdone[rs], static_cast<uint32_t>(it >> 1) & 1u, 37)) break;
-      if (!status_set()) red_release_add(&a.cnt[j], 1);
-      mbar_arrive(&recfree[rs]);
-    }
-  }
-  tc_fence_before();
+
+  fs_fence_before();
   __syncthreads();
   if (warp == 1) {
-    tc_fence_after();
+    fs_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"(kFuTmemCols)
+                 "r"(kFsTmemCols)
                  : "memory");
   }
 }
 
 // Zeroes the tile counters; launched right before the fused kernel.
 __global__ void pre_fused_zero_kernel(int* cnt, int n) {
+  pdl_wait();
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) cnt[i] = 0;
+  pdl_trigger();
 }
 
-// 3-D bf16 tensor map over [d2][4][H] (H contiguous), box [box2][1][box0].
-static bool make_map_3d(CUtensorMap* m, const void* base, int64_t H, int64_t d2, int box0,
-                        int box2, CUtensorMapSwizzle swz) {
-  EncodeTiledFn fn = encode_tiled();
-  if (!fn) return false;
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(H), 4, static_cast<cuuint64_t>(d2)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(H) * 2, static_cast<cuuint64_t>(H) * 8};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box0), 1, static_cast<cuuint32_t>(box2)};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+// ------------------------------------------------------------------------------ host side
+
+typedef CUresult (*FsEncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static FsEncodeTiledFn fs_encode_tiled() {
+  static FsEncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<FsEncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
 }
 
-// Returns 0, a negative MHC_ERR_* code, or 1 when this device cannot co-schedule the grid (the
-// caller then takes another path).
+// Returns 0, a negative MHC_ERR_* code, or 1 when this device cannot run the plan's grid with all
+// CTAs resident (nothing is launched then).
 int launch_pre_fused(const PreArgs& a, cudaStream_t s) {
-  const FuPlan plan = fu_plan(a.T, a.H);
-  const int sms = device_sm_count();
-  if (plan.nsg > sms) return 1;
-  int64_t groups = sms / plan.nsg;
-  if (groups > plan.gmax) groups = plan.gmax;  // the workspace holds gmax record rings
-  const int q = static_cast<int>(plan.q);
-  const int smem = fu_smem_bytes(q);
-
-  static bool attr_set[64] = {};
-  const int dev = current_device();
-  if (dev < 0) return -4;
-  if (!attr_set[dev]) {
-    const int mx = fu_smem_bytes(1) > fu_smem_bytes(2) ? fu_smem_bytes(1) : fu_smem_bytes(2);
-    if (cudaFuncSetAttribute(pre_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mx) !=
-        cudaSuccess)
-      return -4;
-    attr_set[dev] = true;
-  }
+  const FsPlan plan = fs_plan(a.T, a.H, device_sm_count());
+  if (!plan.ok) return 1;
+  if (!ensure_smem_limit(reinterpret_cast<const void*>(pre_fused_kernel), plan.smem)) return 1;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pre_fused_kernel, kFuThreads, smem) !=
-          cudaSuccess ||
-      per_sm < 1)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pre_fused_kernel, kFsThreads,
+                                                    plan.smem) != cudaSuccess ||
+      per_sm < 1) {
+    cudaGetLastError();
     return 1;
-
-  uint8_t* ws = static_cast<uint8_t*>(a.workspace);
-  uint16_t* Bw = reinterpret_cast<uint16_t*>(ws);
-  int* cnt = reinterpret_cast<int*>(ws + plan.cnt_off);
-  float* part = reinterpret_cast<float*>(ws + plan.part_off);
-  CUtensorMap mR, mB;
-  if (!make_map_3d(&mR, a.R, a.H, a.T, kFuHS, kFuM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_3d(&mB, Bw, a.H, kFuN, kFuHS, kFuN, CU_TENSOR_MAP_SWIZZLE_128B))
-    return -4;
-
+  }
   const int64_t K = 4 * a.H;
-  const int64_t sb = (K + 255) / 256;
-  pre_tc_split_kernel<<<static_cast<int>(sb < 4096 ? sb : 4096), 256, 0, s>>>(a.hc_fn, Bw, K);
-  pre_fused_zero_kernel<<<1, 256, 0, s>>>(cnt, static_cast<int>(2 * plan.ntiles));
-  note_launches(2);
-  if (cudaGetLastError() != cudaSuccess) return -4;
+  FsEncodeTiledFn fn = fs_encode_tiled();
+  if (!fn) return -4;
+  CUtensorMap mR;
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(a.T)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kFsKB), static_cast<cuuint32_t>(kFsM)};
+    const cuuint32_t estr[2] = {1, 1};
+    if (fn(&mR, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.R), dims, strides,
+           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return -4;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+  int* cnt = reinterpret_cast<int*>(ws + plan.cnt_off);
+  float* rec = reinterpret_cast<float*>(ws + plan.rec_off);
 
-  FuArgs fa;
+  if (launch_pdl(pre_fused_zero_kernel, dim3(1), dim3(256), 0, s, cnt,
+                 static_cast<int>(plan.ntiles)) != cudaSuccess)
+    return -4;
+  note_launches(1);
+
+  FsArgs fa;
   fa.R = a.R;
+  fa.hc_fn = a.hc_fn;
   fa.scale = a.hc_scale;
   fa.base = a.hc_base;
   fa.y = a.y;
@@ -631,22 +725,43 @@ int launch_pre_fused(const PreArgs& a, cudaStream_t s) {
   fa.post = a.post;
   fa.comb = a.comb;
   fa.cnt = cnt;
-  fa.ready = cnt + plan.ntiles;
-  fa.part = part;
+  fa.rec = rec;
   fa.T = a.T;
   fa.H = a.H;
+  fa.K = K;
+  fa.KB = static_cast<int>(plan.KB);
   fa.ntiles = static_cast<int>(plan.ntiles);
-  fa.nsg = static_cast<int>(plan.nsg);
-  fa.q = q;
-  fa.groups = static_cast<int>(groups);
+  fa.G = plan.G;
+  fa.NG = plan.NG;
+  fa.nbmax = plan.nbmax;
+  fa.stages = plan.stages;
+  fa.lag = kFsDefaultLag;
   fa.fp = FinishParams{a.iters, a.sinkhorn_eps, a.rms_eps, a.pre_eps, a.post_mult};
 
-  void* args[] = {&mR, &mB, &fa};
-  const dim3 grid(static_cast<unsigned>(plan.nsg * groups));
-  if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(pre_fused_kernel), grid,
-                                  dim3(kFuThreads), args, static_cast<size_t>(smem), s) !=
-      cudaSuccess)
+  // Cooperative launch: every CTA resident at once (the groups' CTAs wait on one another). Also a
+  // programmatic dependent of the zero kernel where the runtime accepts both attributes together.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(plan.NG * plan.G));
+  cfg.blockDim = dim3(kFsThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(plan.smem);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, pre_fused_kernel, mR, fa);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, pre_fused_kernel, mR, fa);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
     return -4;
+  }
   note_launches(1);
   return 0;
 }

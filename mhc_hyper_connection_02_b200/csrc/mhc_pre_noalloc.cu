@@ -6,8 +6,6 @@
 // kernel of the same call, so nothing needs clearing between calls. The array is shared by every
 // call on a device: calls whose kernels overlap on the GPU (different streams, no ordering between
 // them) race on it.
-#include <mutex>
-
 #include "mhc.h"
 #include "mhc_device.cuh"
 #include "mhc_internal.h"
@@ -18,25 +16,17 @@ namespace mhc {
 static __device__ __align__(256) uint8_t g_noalloc_scratch[MHC_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-void* g_noalloc_ptr[64] = {};
-std::mutex g_noalloc_mu;
-
 // Device address of g_noalloc_scratch on the current device. In host code the symbol's name is a
-// host-side stand-in, not a device address, so the address is looked up once per device (with that
-// device current) and cached.
+// host-side stand-in, not a device address, so the address is looked up with the device current.
+// It is looked up on every call rather than cached: after a device reset or a new context the
+// module is loaded again, possibly elsewhere, and a cached address would point at freed memory.
 int noalloc_scratch(void** out) {
-  const int dev = current_device();
-  if (dev < 0) return MHC_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
-      cudaGetLastError();
-      return MHC_ERR_CUDA;
-    }
-    g_noalloc_ptr[dev] = p;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+    cudaGetLastError();
+    return MHC_ERR_CUDA;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = p;
   return MHC_OK;
 }
 

@@ -48,7 +48,7 @@ constexpr int kTcStageBytes = kTcSub * kTcABytes + kTcBBytes;  // 43008 = 42 x 1
 constexpr int kTcThreads = 192;
 constexpr int kTcTmemCols = 512;                   // 2 buffers x 2 sub-tiles x 128 columns
 constexpr int kTcSmem = 1024 + kTcStages * kTcStageBytes + 256;
-constexpr int64_t kTcSms = 148;                    // CTAs of the projection (B200's SM count)
+constexpr int64_t kTcMaxCtas = 148;                // most CTAs the projection plan uses
 constexpr int64_t kTcMinBlocks = 8;                // K blocks per CTA at least (pipeline fill)
 
 // Work plan of the projection: W = ntiles * kblocks block-tiles over P CTAs; CTA c takes
@@ -58,14 +58,17 @@ struct TcPlan {
   size_t bw_bytes;  // workspace bytes of Bw, rounded to 1 KB
 };
 
-static TcPlan tc_plan(int64_t T, int64_t H) {
+// `sms` is the device's SM count at launch; workspace sizing uses the largest plan (kTcMaxCtas),
+// which never needs fewer slots than a plan over fewer CTAs.
+static TcPlan tc_plan(int64_t T, int64_t H, int64_t sms = kTcMaxCtas) {
   TcPlan p;
   const int64_t K = 4 * H;
   p.ntiles = (T + kTcTile - 1) / kTcTile;
   p.kblocks = (K + kTcKB - 1) / kTcKB;
   p.W = p.ntiles * p.kblocks;
   p.P = p.W / kTcMinBlocks;
-  if (p.P > kTcSms) p.P = kTcSms;
+  if (p.P > kTcMaxCtas) p.P = kTcMaxCtas;
+  if (p.P > sms) p.P = sms;
   if (p.P < 1) p.P = 1;
   // A tile spans kblocks consecutive units; a CTA range holds at least floor(W / P) of them, so a
   // tile meets at most floor(kblocks P / W) + 2 ranges.
@@ -533,7 +536,7 @@ static bool make_map(CUtensorMap* m, const void* base, int64_t cols, int64_t row
 // Split + projection: records [S][T][32] (raw[24], ss) in the workspace after Bw. Returns 0 or a
 // negative MHC_ERR_* code; *part_out / *nrec_out receive the records and their slot count.
 int launch_tc_projection(const PreArgs& a, cudaStream_t s, float** part_out, int* nrec_out) {
-  const TcPlan plan = tc_plan(a.T, a.H);
+  const TcPlan plan = tc_plan(a.T, a.H, device_sm_count());
   const int64_t K = 4 * a.H;
   uint8_t* ws = static_cast<uint8_t*>(a.workspace);
   uint16_t* Bw = reinterpret_cast<uint16_t*>(ws);
@@ -542,15 +545,7 @@ int launch_tc_projection(const PreArgs& a, cudaStream_t s, float** part_out, int
   CUtensorMap mR, mB;
   if (!make_map(&mR, a.R, K, a.T, kTcM) || !make_map(&mB, Bw, K, kTcN, kTcN)) return -4;
 
-  static bool attr_set[64] = {};
-  const int dev = current_device();
-  if (dev < 0) return -4;
-  if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(pre_tc_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kTcSmem) != cudaSuccess)
-      return -4;
-    attr_set[dev] = true;
-  }
+  if (!ensure_smem_limit(reinterpret_cast<const void*>(pre_tc_proj_kernel), kTcSmem)) return -4;
 
   const int64_t sb = (K + 255) / 256;
   const int split_blocks = static_cast<int>(sb < 4096 ? sb : 4096);
@@ -570,7 +565,6 @@ int launch_tc_projection(const PreArgs& a, cudaStream_t s, float** part_out, int
 }
 
 int launch_pre_tc(const PreArgs& a, cudaStream_t s) {
-  const TcPlan plan = tc_plan(a.T, a.H);
   float* part = nullptr;
   int nrec = 0;
   const int r = launch_tc_projection(a, s, &part, &nrec);
@@ -582,7 +576,7 @@ int launch_pre_tc(const PreArgs& a, cudaStream_t s) {
     const int64_t cb = (4 * a.T + 255) / 256;
     if (cb > 0x7fffffff) return -5;
     if (launch_pdl(pre_tc_coef_kernel, dim3(static_cast<unsigned>(cb)), dim3(256), 0, s,
-                   static_cast<const float*>(part), static_cast<int>(plan.S), a.hc_scale,
+                   static_cast<const float*>(part), nrec, a.hc_scale,
                    a.hc_base, a.pre, a.post, a.comb, a.T, 4 * a.H, fp) != cudaSuccess)
       return -4;
     note_launches(1);
@@ -597,7 +591,8 @@ int launch_pre_tc(const PreArgs& a, cudaStream_t s) {
     const int64_t nhb = (a.H + kAggCols - 1) / kAggCols;
     if (a.T > 0x7fffffff || 1 + nhb > 65535) return -5;
     const dim3 g2(static_cast<unsigned>(a.T), static_cast<unsigned>(1 + nhb));
-    if (launch_pdl(pre_cc_finish_kernel<false>, g2, dim3(256), 0, s, a.R, part, plan.S,
+    if (launch_pdl(pre_cc_finish_kernel<false>, g2, dim3(256), 0, s, a.R, part,
+                   static_cast<int64_t>(nrec),
                    a.hc_scale, a.hc_base, a.y, a.pre, a.post, a.comb, a.T, a.H, fp) != cudaSuccess)
       return -4;
   }

@@ -41,6 +41,13 @@ def compare(out_dev, w, post, comb, rows=None, label=""):
     assert fail == 0
 
 
+def compare_all(out_dev, w, post, comb, label="", chunk=1024):
+    """Every token, checked in chunks of `chunk` tokens (bounded host memory at the full size)."""
+    for c0 in range(0, w.T, chunk):
+        compare(out_dev, w, post, comb, rows=np.arange(c0, min(w.T, c0 + chunk)),
+                label=f"{label} [{c0}:{min(w.T, c0 + chunk)}]")
+
+
 def run(w, path, post, comb, out=None):
     x, R = dev_bf16(w.x), dev_bf16(w.R)
     o = mhc.post(x, R, dev_f32(post), dev_f32(comb), out=out, path=path)
@@ -143,24 +150,41 @@ def test_post_rejects_host_memory():
 
 @pytest.mark.parametrize("name", ["post4k", "tail"])
 def test_post_workloads(name):
+    """Every token of the post-only (T=4096, H=4096) and tail (T=3000, H=1000) workloads."""
     w = inputs.WORKLOADS[name]()
     post, comb = post_coefficients(w)
     for path in (["vec8", "persistent"] if w.H % 8 == 0 else []) + ["scalar"]:
         out = run(w, PATHS[path], post, comb)
-        rows = np.random.default_rng(0).choice(w.T, size=min(w.T, 300), replace=False)
-        rows = np.unique(np.concatenate([rows, [0, w.T - 1]]))
-        compare(out, w, post, comb, rows=rows, label=f"{name} {path}")
+        compare_all(out, w, post, comb, label=f"{name} {path}")
 
 
 @pytest.mark.slow
-def test_post_large_sampled():
-    """T=8192, H=7168, sampled tokens (the oracle computes them one by one)."""
+def test_post_large_full_batch():
+    """T=8192, H=7168, every token, for the default call (the persistent kernel bench.py times)
+    and the vec8 kernel."""
     w = inputs.large()
     post, comb = post_coefficients(w)
-    for path in ("vec8", "persistent"):
-        out = run(w, PATHS[path], post, comb)
-        rows = np.unique(np.concatenate(
-            [np.random.default_rng(1).choice(w.T, 48, replace=False), [0, w.T - 1]]))
-        compare(out, w, post, comb, rows=rows, label=f"large {path}")
+    for path in (mhc.PATH_AUTO, mhc.POST_PATH_VEC8):
+        out = run(w, path, post, comb)
+        compare_all(out, w, post, comb, label=f"large path={path}")
         del out
         torch.cuda.empty_cache()
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["post4k", "large"])
+def test_post_persistent_in_place_at_size(name):
+    """In place (out == R) on the persistent kernel at sizes where every CTA runs many tiles, so
+    its prefetch ring runs ahead of the in-place writes: equal, bit for bit, to out of place."""
+    w = inputs.WORKLOADS[name]()
+    post, comb = post_coefficients(w)
+    x, p, c = dev_bf16(w.x), dev_f32(post), dev_f32(comb)
+    ref = mhc.post(x, dev_bf16(w.R), p, c, path=mhc.POST_PATH_PERSISTENT)
+    R = dev_bf16(w.R)
+    o = mhc.post(x, R, p, c, out=R, path=mhc.POST_PATH_PERSISTENT)
+    torch.cuda.synchronize()
+    assert mhc.device_status() == 0
+    assert o.data_ptr() == R.data_ptr()
+    assert torch.equal(R.view(torch.int16), ref.view(torch.int16))
+    if name == "post4k":
+        compare_all(R, w, post, comb, label="post4k in place")

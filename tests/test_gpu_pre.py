@@ -34,6 +34,21 @@ def run_pre(w, path=mhc.PATH_AUTO, params=None, R_dev=None):
     return y, pre, post, comb
 
 
+def run_fused(w, R_dev=None):
+    """The single-pass kernel, forced. Returns None where the library reports it cannot run this
+    shape (MHC_ERR_UNSUPPORTED, before any launch); otherwise asserts that exactly its two launches
+    (counter zeroing + the fused kernel) were enqueued, so a pass is the fused kernel's."""
+    n0 = mhc.launch_count()
+    try:
+        outs = run_pre(w, mhc.PRE_PATH_TENSOR_FUSED, R_dev=R_dev)
+    except mhc.MhcError as e:
+        assert e.status == mhc.MHC_ERR_UNSUPPORTED
+        assert mhc.launch_count() == n0
+        return None
+    assert mhc.launch_count() - n0 == 2, "the fused path must be exactly its two launches"
+    return outs
+
+
 def compare_pre(w, outs, rows=None, label="", pre_eps=None, post_mult=None, iters=None, eps=None):
     y, pre, post, comb = outs
     R = w.R if rows is None else w.R[rows]
@@ -57,11 +72,11 @@ def compare_pre(w, outs, rows=None, label="", pre_eps=None, post_mult=None, iter
 @pytest.mark.parametrize("path", ["cuda_core", "tensor", "tensor_split", "tensor_fused"])
 def test_pre_small_workload(path):
     w = inputs.small()
-    try:
+    if path == "tensor_fused":
+        outs = run_fused(w)
+        assert outs is not None, "the single-pass kernel supports T=64, H=512"
+    else:
         outs = run_pre(w, PRE_PATHS[path])
-    except mhc.MhcError as e:
-        assert e.status == mhc.MHC_ERR_UNSUPPORTED
-        pytest.skip(f"{path} path not available at T={w.T}, H={w.H}")
     compare_pre(w, outs, label=f"small {path}")
 
 
@@ -74,8 +89,11 @@ def test_pre_shapes(T, H):
     if H % 2 == 0:
         compare_pre(w, run_pre(w, mhc.PRE_PATH_TENSOR), label=f"T={T} H={H} tensor")
         compare_pre(w, run_pre(w, mhc.PRE_PATH_TENSOR_SPLIT), label=f"T={T} H={H} tensor-split")
-    if H % 8 == 0 and 448 < H <= 9472:
-        compare_pre(w, run_pre(w, mhc.PRE_PATH_TENSOR_FUSED), label=f"T={T} H={H} tensor-fused")
+    fused = run_fused(w)
+    if fused is not None:
+        compare_pre(w, fused, label=f"T={T} H={H} tensor-fused")
+    else:
+        assert H % 8 != 0 or H < 64, f"single-pass kernel refused T={T} H={H}"
 
 
 @pytest.mark.parametrize("T,H", [(300, 7168), (129, 1000), (1, 4096), (520, 512)])
@@ -87,8 +105,9 @@ def test_pre_tensor_path_agrees_with_cuda_core_path(T, H):
     b = run_pre(w, mhc.PRE_PATH_CUDA_CORE)
     c = run_pre(w, mhc.PRE_PATH_TENSOR_SPLIT)
     others = [(b, "cuda_core"), (c, "tensor-split")]
-    if H % 8 == 0 and 448 < H <= 9472:
-        others.append((run_pre(w, mhc.PRE_PATH_TENSOR_FUSED), "tensor-fused"))
+    fused = run_fused(w)
+    if fused is not None:
+        others.append((fused, "tensor-fused"))
     for other, oname in others:
         for x, y, name in zip(a[1:], other[1:], ("pre", "post", "comb")):
             d = (x.double() - y.double()).abs().max().item()
@@ -108,13 +127,39 @@ def test_pre_tail_workload():
     compare_pre(w, run_pre(w), label="tail T=3000 H=1000")
 
 
+def compare_pre_all(w, outs, label="", chunk=1024):
+    """Every token, checked in chunks of `chunk` tokens (bounded host memory at the full size)."""
+    for c0 in range(0, w.T, chunk):
+        compare_pre(w, outs, rows=np.arange(c0, min(w.T, c0 + chunk)),
+                    label=f"{label} [{c0}:{min(w.T, c0 + chunk)}]")
+
+
 @pytest.mark.slow
-def test_pre_large_sampled():
+def test_pre_large_full_batch():
+    """T=8192, H=7168: every token of the default call (the launch bench.py times)."""
     w = inputs.large()
-    outs = run_pre(w)
-    rows = np.unique(np.concatenate([np.random.default_rng(2).choice(w.T, 40, replace=False),
-                                     [0, 127, 128, w.T - 1]]))
-    compare_pre(w, outs, rows=rows, label="large sampled")
+    compare_pre_all(w, run_pre(w), label="large")
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("path", ["tensor_fused", "tensor_split", "cuda_core"])
+def test_pre_large_full_batch_each_path(path):
+    """T=8192, H=7168, every token, on each forced path (the single-pass kernel runs here with
+    every group's record ring wrapping many times)."""
+    w = inputs.large()
+    outs = run_fused(w) if path == "tensor_fused" else run_pre(w, PRE_PATHS[path])
+    assert outs is not None
+    compare_pre_all(w, outs, label=f"large {path}")
+
+
+@pytest.mark.parametrize("T,H", [(3000, 1000), (1000, 7168), (2000, 4096), (129, 64)])
+def test_pre_fused_multi_tile(T, H):
+    """The single-pass kernel over many tiles per group, ragged last tiles and K ranges that are not
+    a multiple of 64 columns (H = 1000)."""
+    w = inputs.custom(T, H, seed=T + 7 * H)
+    outs = run_fused(w)
+    assert outs is not None
+    compare_pre(w, outs, label=f"fused T={T} H={H}")
 
 
 def test_pre_params_other_than_default():
