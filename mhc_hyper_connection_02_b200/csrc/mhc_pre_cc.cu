@@ -126,6 +126,171 @@ __global__ void __launch_bounds__(256) pre_cc_partial_kernel(const uint16_t* __r
   }
 }
 
+// Decode-sized calls (T <= 16): lanes run along K instead of along tokens. Thread i of split s
+// owns k = s*KS + i (and k + 256 when KS > 256): it loads that k's 24 hc_fn weights once and the
+// row's value of every token up front, then per token forms its 24 products and its square, and a
+// butterfly reduce-scatter over the warp (31 shuffles) leaves lane j holding the warp's sum of
+// component j. The 8 warp sums are added in warp order. One hc_fn read per call, every load
+// issued before any is used: the step is a few round trips of latency.
+constexpr int kKlPer = 2;          // k values per thread at most (KS <= 512)
+constexpr int kKlMaxTokens = 16;   // above this the lane-per-token kernel is faster (measured)
+
+template <bool kAlignedW>
+__global__ void __launch_bounds__(256) pre_cc_partial_klane_kernel(const uint16_t* __restrict__ R,
+                                                                   const float* __restrict__ W,
+                                                                   float* __restrict__ part,
+                                                                   int64_t T, int64_t K,
+                                                                   int64_t KS) {
+  pdl_wait();  // launched as a programmatic dependent of the previous grid
+  pdl_trigger();
+  __shared__ float red[kCcWarps][kCcTokens][kCcRec + 1];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t s = blockIdx.y;
+  const int64_t kb = s * KS;
+  const int64_t ke = min(K, kb + KS);
+  float w[kKlPer][kMix];
+  float rv[kKlPer][kCcTokens];
+#pragma unroll
+  for (int i = 0; i < kKlPer; ++i) {
+    const int64_t k = kb + threadIdx.x + i * 256;
+    const bool ok = k < ke;
+    if (kAlignedW) {
+#pragma unroll
+      for (int q = 0; q < 6; ++q) {
+        const float4 v = ok ? __ldg(reinterpret_cast<const float4*>(W + k * kMix) + q)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        w[i][4 * q] = v.x, w[i][4 * q + 1] = v.y, w[i][4 * q + 2] = v.z, w[i][4 * q + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < kMix; ++j) w[i][j] = ok ? __ldg(W + k * kMix + j) : 0.f;
+    }
+#pragma unroll
+    for (int t = 0; t < kCcTokens; ++t)
+      rv[i][t] = (ok && t < T) ? bf16_to_f32(R[t * K + k]) : 0.f;
+  }
+#pragma unroll
+  for (int t = 0; t < kCcTokens; ++t) {
+    if (t >= T) break;
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < kMix; ++j) v[j] = rv[0][t] * w[0][j];
+    v[kMix] = rv[0][t] * rv[0][t];
+#pragma unroll
+    for (int i = 1; i < kKlPer; ++i) {
+#pragma unroll
+      for (int j = 0; j < kMix; ++j) v[j] = fmaf(rv[i][t], w[i][j], v[j]);
+      v[kMix] = fmaf(rv[i][t], rv[i][t], v[kMix]);
+    }
+#pragma unroll
+    for (int j = kMix + 1; j < 32; ++j) v[j] = 0.f;
+    // Reduce-scatter: after the step over offset o, a lane keeps the half of its list that its
+    // lane bit o selects; after five steps lane j holds component j summed over the warp.
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      const bool upper = (lane & o) != 0;
+#pragma unroll
+      for (int i = 0; i < o; ++i) {
+        const float keep = upper ? v[o + i] : v[i];
+        const float give = upper ? v[i] : v[o + i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, give, o);
+      }
+    }
+    red[warp][t][lane] = v[0];
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < T * 25; idx += blockDim.x) {
+    const int tl = idx / 25;
+    const int j = idx - tl * 25;
+    float acc = 0.f;
+#pragma unroll
+    for (int w8 = 0; w8 < kCcWarps; ++w8) acc += red[w8][tl][j];
+    part[(s * T + tl) * kCcRec + j] = acc;
+  }
+}
+
+// Decode-sized calls with more tokens (16 < T <= 32): lane = token as in pre_cc_partial_kernel,
+// but the split's hc_fn rows (KS x 24 fp32, at most 48 KB) are first copied into shared memory
+// with coalesced loads, so the loop reads them from shared memory (one broadcast per row) instead
+// of waiting on global memory for every eight k.
+constexpr int kStMaxKS = 512;
+
+template <bool kVecR, bool kAlignedW>
+__global__ void __launch_bounds__(256) pre_cc_partial_staged_kernel(const uint16_t* __restrict__ R,
+                                                                    const float* __restrict__ W,
+                                                                    float* __restrict__ part,
+                                                                    int64_t T, int64_t K,
+                                                                    int64_t KS) {
+  pdl_wait();  // launched as a programmatic dependent of the previous grid
+  pdl_trigger();
+  __shared__ __align__(16) float sm[kStMaxKS * kMix];  // W slice, then the warp partial sums
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t s = blockIdx.y;
+  const int64_t kb = s * KS;
+  const int64_t ke = min(K, kb + KS);
+  const int nw = static_cast<int>((ke - kb) * kMix);
+  if (kAlignedW) {
+    const float4* src = reinterpret_cast<const float4*>(W + kb * kMix);
+    for (int i = threadIdx.x; i < nw / 4; i += blockDim.x)
+      reinterpret_cast<float4*>(sm)[i] = __ldg(src + i);
+  } else {
+    for (int i = threadIdx.x; i < nw; i += blockDim.x) sm[i] = __ldg(W + kb * kMix + i);
+  }
+  __syncthreads();
+  const int64_t KW = KS / kCcWarps;  // multiple of 8
+  const int64_t k0 = kb + warp * KW;
+  const int64_t k1 = min(ke, k0 + KW);
+  const int64_t t = lane;
+  float acc[kMix];
+#pragma unroll
+  for (int j = 0; j < kMix; ++j) acc[j] = 0.f;
+  float ss = 0.f;
+  auto add_row = [&](float r, int64_t k) {
+    const float4* w4 = reinterpret_cast<const float4*>(sm + (k - kb) * kMix);
+    ss = fmaf(r, r, ss);
+#pragma unroll
+    for (int q = 0; q < 6; ++q) {
+      const float4 v = w4[q];
+      acc[4 * q + 0] = fmaf(r, v.x, acc[4 * q + 0]);
+      acc[4 * q + 1] = fmaf(r, v.y, acc[4 * q + 1]);
+      acc[4 * q + 2] = fmaf(r, v.z, acc[4 * q + 2]);
+      acc[4 * q + 3] = fmaf(r, v.w, acc[4 * q + 3]);
+    }
+  };
+  if (t < T) {
+    const uint16_t* row = R + t * K;
+    int64_t k = k0;
+    if (kVecR) {
+      for (; k + 8 <= k1; k += 8) {
+        const uint4 v = ld_stream_ro(row + k);
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          add_row(bf16_lo(u[e]), k + 2 * e);
+          add_row(bf16_hi(u[e]), k + 2 * e + 1);
+        }
+      }
+    }
+    for (; k < k1; ++k) add_row(bf16_to_f32(row[k]), k);
+  }
+  __syncthreads();  // every warp is done with the W slice
+  float (*red)[kCcTokens][25] = reinterpret_cast<float (*)[kCcTokens][25]>(sm);
+#pragma unroll
+  for (int j = 0; j < kMix; ++j) red[warp][lane][j] = acc[j];
+  red[warp][lane][24] = ss;
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < T * 25; idx += blockDim.x) {
+    const int tl = idx / 25;
+    const int j = idx - tl * 25;
+    float v = 0.f;
+#pragma unroll
+    for (int w8 = 0; w8 < kCcWarps; ++w8) v += red[w8][tl][j];
+    part[(s * T + tl) * kCcRec + j] = v;
+  }
+}
+
 struct FinishParams {
   int iters;
   float sinkhorn_eps;
@@ -270,7 +435,25 @@ int launch_cc_projection(const PreArgs& a, cudaStream_t s, float** part_out, int
   const bool vecR = aligned16(a.R) && (K % 8 == 0);
   const bool alignW = aligned16(a.hc_fn);
   cudaError_t e;
-  if (vecR && alignW)
+  if (a.T <= kKlMaxTokens && plan.KS <= 256 * kKlPer) {
+    e = alignW ? launch_pdl(pre_cc_partial_klane_kernel<true>, g1, dim3(256), 0, s, a.R, a.hc_fn,
+                            part, a.T, K, plan.KS)
+               : launch_pdl(pre_cc_partial_klane_kernel<false>, g1, dim3(256), 0, s, a.R, a.hc_fn,
+                            part, a.T, K, plan.KS);
+  } else if (a.T <= kCcTokens && plan.KS <= kStMaxKS) {
+    if (vecR && alignW)
+      e = launch_pdl(pre_cc_partial_staged_kernel<true, true>, g1, dim3(256), 0, s, a.R, a.hc_fn,
+                     part, a.T, K, plan.KS);
+    else if (vecR)
+      e = launch_pdl(pre_cc_partial_staged_kernel<true, false>, g1, dim3(256), 0, s, a.R, a.hc_fn,
+                     part, a.T, K, plan.KS);
+    else if (alignW)
+      e = launch_pdl(pre_cc_partial_staged_kernel<false, true>, g1, dim3(256), 0, s, a.R, a.hc_fn,
+                     part, a.T, K, plan.KS);
+    else
+      e = launch_pdl(pre_cc_partial_staged_kernel<false, false>, g1, dim3(256), 0, s, a.R,
+                     a.hc_fn, part, a.T, K, plan.KS);
+  } else if (vecR && alignW)
     e = launch_pdl(pre_cc_partial_kernel<true, true>, g1, dim3(256), 0, s, a.R,
                    a.hc_fn, part, a.T, K, plan.KS);
   else if (vecR)

@@ -18,11 +18,12 @@
 //   warps 2-5   sum of squares of each token row from the same stages; after the tile, the
 //               accumulator (tcgen05.ld) gives the partial record rec[token][j] = raw[24], ss, and
 //               one thread release-increments the tile's counter.
-//   warps 6-7   (alternate tiles) once the counter reaches G: for the tokens this CTA owns in the
-//               tile (token l with (l + 128 n) mod G == j), sum the G partial records in a fixed
-//               order, form rstd, the logits, the gates and the Sinkhorn comb, write pre, post and
-//               comb, and hand pre to the aggregate warps through shared memory.
-//   warps 8-15  y = bf16_rn(sum_i pre_i R_i) for the owned tokens, re-reading their rows with
+//   warps 6-9   (tile n by warp 6 + n mod 4) once the counter reaches G: for the tokens this CTA
+//               owns in the tile (token l with (l + 128 n) mod G == j), two at a time, sixteen
+//               lanes per token sum its G partial records in a fixed order; then rstd, the logits,
+//               the gates and the Sinkhorn comb; write pre, post and comb, and hand pre to the
+//               aggregate warps through shared memory.
+//   warps 10-15 y = bf16_rn(sum_i pre_i R_i) for the owned tokens, re-reading their rows with
 //               16-byte loads. The tile came from HBM a few microseconds earlier and is still in
 //               L2, so HBM sees R once.
 //
@@ -52,23 +53,29 @@ constexpr int kFsMinG = 4;                   // fewest CTAs per group
 constexpr int kFsMaxOwn = kFsM / kFsMinG;    // most tokens a CTA owns in one tile
 constexpr int kFsMaxStages = 8;
 constexpr int kFsRec = 28;                   // floats per partial record (raw[24], ss, 3 zero)
-constexpr int kFsRing = 6;                   // tiles of records per group (>= 2 D)
-constexpr int kFsSlots = 4;                  // coefficient -> aggregate hand-over slots
-constexpr int kFsCoefWarps = 2;
+constexpr int kFsEpiDelay = 3;              // stages into the next tile before the records
+constexpr int kFsCoefWarps = 4;
+constexpr int kFsTokLanes = 16;              // lanes that reduce one token's records
+constexpr int kFsTokPerPass = 32 / kFsTokLanes;
+constexpr int kFsSlots = kFsCoefWarps;       // coefficient -> aggregate hand-over slots
 constexpr int kFsCoefWarp0 = 6;
-constexpr int kFsAggWarp0 = 8;
-constexpr int kFsAggWarps = 8;
+constexpr int kFsAggWarp0 = kFsCoefWarp0 + kFsCoefWarps;
+constexpr int kFsAggWarps = 16 - kFsAggWarp0;
 constexpr int kFsThreads = 512;
 constexpr int kFsTmemCols = 256;             // accumulators at columns 0 and 128
 constexpr int kFsMaxCtas = 148;              // most CTAs a plan uses (workspace sizing)
 constexpr int kFsSmemLimit = 227 * 1024;
-constexpr int kFsDefaultLag = 2;             // D
+// D: the stream of tile n waits for this CTA's coefficients of tile n - D. D < kFsSlots keeps that
+// wait unambiguous (the slot cannot have moved on by two phases), and a record ring of 2 D tiles
+// is then never overwritten before every CTA of the group has read it.
+constexpr int kFsLag = 3;
+constexpr int kFsRing = 2 * kFsLag;
+static_assert(kFsLag < kFsSlots, "lag must stay below the hand-over slots");
 
 // Shared-memory scratch after the rings: barriers, TMEM address, coefficient sums, hand-over.
 constexpr int kFsOffBars = 0;      // full[8] empty[8] afull[2] aempty[2] cfull[4] cempty[4] done
 constexpr int kFsOffTmem = 240;
-constexpr int kFsOffCsum = 256;    // float [kFsCoefWarps][8][kFsRec]
-constexpr int kFsOffPre = kFsOffCsum + kFsCoefWarps * 8 * kFsRec * 4;  // float [slots][own][4]
+constexpr int kFsOffPre = 256;                                         // float [slots][own][4]
 constexpr int kFsOffTok = kFsOffPre + kFsSlots * kFsMaxOwn * 16;       // int [slots][own]
 constexpr int kFsOffNown = kFsOffTok + kFsSlots * kFsMaxOwn * 4;       // int [slots]
 constexpr int kFsMisc = (kFsOffNown + kFsSlots * 4 + 127) / 128 * 128;
@@ -255,7 +262,6 @@ __global__ void __launch_bounds__(kFsThreads, 1)
   uint64_t* cempty = cfull + kFsSlots;
   uint64_t* done = cempty + kFsSlots;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + kFsOffTmem);
-  float* csum = reinterpret_cast<float*>(misc + kFsOffCsum);
   float* slot_pre = reinterpret_cast<float*>(misc + kFsOffPre);
   int* slot_tok = reinterpret_cast<int*>(misc + kFsOffTok);
   int* slot_nown = reinterpret_cast<int*>(misc + kFsOffNown);
@@ -416,38 +422,16 @@ __global__ void __launch_bounds__(kFsThreads, 1)
     }
   } else if (warp < kFsCoefWarp0) {
     // ------------------------------------------------------------------ sum of squares + records
-    // TMEM lane quarter q = warp % 4 holds accumulator rows 32q .. 32q + 31.
+    // TMEM lane quarter q = warp % 4 holds accumulator rows 32q .. 32q + 31. The records of tile n
+    // are formed kFsEpiDelay stages into tile n + 1 (or after the last tile): by then the tile's
+    // MMAs have finished, so these warps never hold the stage ring back waiting for them.
     const int q = warp & 3;
     const int row = q * 32 + lane;
-    int64_t it = 0;
-    for (int n = 0; n < ntg; ++n) {
+    // Forms tile n's records and publishes them; returns true when the four warps stop (a wait
+    // ran out here or in another of them). Every warp calls it once per tile, in tile order, so
+    // the named barrier sequence stays matched.
+    auto epilogue = [&](int n, float ss, bool ok) -> bool {
       const int X = g + n * NG;
-      bool ok = true;
-      float ss0 = 0.f, ss1 = 0.f;
-      for (int kb = 0; kb < nb; ++kb, ++it) {
-        const int s = static_cast<int>(it % ST);
-        const uint32_t ph = static_cast<uint32_t>(it / ST) & 1u;
-        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, 46))) {
-          ok = false;
-          break;
-        }
-        // Row `row` of the swizzled block is its own 128 contiguous bytes (chunks permuted within
-        // it); a sum does not depend on the order. Lanes start at different chunks.
-        const uint4* rp = reinterpret_cast<const uint4*>(Aring + s * kFsABytes + row * 128);
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          const uint4 w = rp[cc ^ (lane & 7)];
-          const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float x0 = bf16_lo(w4[e]), x1 = bf16_hi(w4[e]);
-            ss0 = fmaf(x0, x0, ss0);
-            ss1 = fmaf(x1, x1, ss1);
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-      }
       const int b = n & 1;
       if (ok && !__all_sync(0xffffffffu,
                             mbar_wait(&afull[b], static_cast<uint32_t>(n >> 1) & 1u, 47)))
@@ -475,23 +459,74 @@ __global__ void __launch_bounds__(kFsThreads, 1)
 #pragma unroll
           for (int w = 0; w < 6; ++w)
             r4[w] = make_float4(raw[4 * w], raw[4 * w + 1], raw[4 * w + 2], raw[4 * w + 3]);
-          r4[6] = make_float4(ss0 + ss1, 0.f, 0.f, 0.f);
+          r4[6] = make_float4(ss, 0.f, 0.f, 0.f);
         }
         fs_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&aempty[b]);
       }
-      // The four warps agree on going on (a matched barrier sequence even after a timeout), and
-      // their records are published with one release-increment of the tile's counter.
-      if (named_bar_or(1, 128, !ok)) break;
+      // The four warps agree on going on, and their records are published with one
+      // release-increment of the tile's counter.
+      if (named_bar_or(1, 128, !ok)) return true;
       if (warp == 2 && lane == 0) fs_red_release_add(a.cnt + X, 1);
+      return false;
+    };
+    int64_t it = 0;
+    int pend = -1;  // tile whose records are still to be formed
+    float pend_ss = 0.f;
+    bool stop = false;
+    for (int n = 0; n < ntg && !stop; ++n) {
+      bool ok = true;
+      float ss0 = 0.f, ss1 = 0.f;
+      for (int kb = 0; kb < nb; ++kb, ++it) {
+        const int s = static_cast<int>(it % ST);
+        const uint32_t ph = static_cast<uint32_t>(it / ST) & 1u;
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, 46))) {
+          ok = false;
+          break;
+        }
+        // Row `row` of the swizzled block is its own 128 contiguous bytes (chunks permuted within
+        // it); a sum does not depend on the order. Lanes start at different chunks.
+        const uint4* rp = reinterpret_cast<const uint4*>(Aring + s * kFsABytes + row * 128);
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          const uint4 w = rp[cc ^ (lane & 7)];
+          const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float x0 = bf16_lo(w4[e]), x1 = bf16_hi(w4[e]);
+            ss0 = fmaf(x0, x0, ss0);
+            ss1 = fmaf(x1, x1, ss1);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        if (pend >= 0 && kb == kFsEpiDelay) {
+          stop = epilogue(pend, pend_ss, true);
+          pend = -1;
+          if (stop) break;
+        }
+      }
+      if (stop) break;
+      if (!ok) {  // the next barrier of the sequence, carrying the failure
+        epilogue(pend >= 0 ? pend : n, 0.f, false);
+        stop = true;
+        break;
+      }
+      if (pend >= 0) {  // tiles of at most kFsEpiDelay blocks
+        stop = epilogue(pend, pend_ss, true);
+        if (stop) break;
+      }
+      pend = n;
+      pend_ss = ss0 + ss1;
     }
+    if (!stop && pend >= 0) epilogue(pend, pend_ss, true);
   } else if (warp < kFsAggWarp0) {
     // ------------------------------------------------------------------ coefficients
     const int cw = warp - kFsCoefWarp0;
-    float* cs = csum + cw * 8 * kFsRec;
-    const int quad = lane >> 2;
-    const int r = lane & 3;
+    const int grp = lane / kFsTokLanes;  // token of the pass
+    const int gl = lane % kFsTokLanes;   // lane within the token's group
+    const int r = lane & 3;  // lanes gl < 4 form the token's quad: pre r, post r, comb row r
     for (int n = cw; n < ntg; n += kFsCoefWarps) {
       const int X = g + n * NG;
       const int slot = n % kFsSlots;
@@ -506,67 +541,77 @@ __global__ void __launch_bounds__(kFsThreads, 1)
       const int64_t lim64 = a.T - static_cast<int64_t>(X) * kFsM;
       const int lim = lim64 < kFsM ? static_cast<int>(lim64) : kFsM;
       const int nown = l0 < lim ? (lim - l0 + G - 1) / G : 0;
-      for (int p0 = 0; p0 < nown; p0 += 8) {
-        const int np = nown - p0 < 8 ? nown - p0 : 8;
-        // Sum each token's G records: lane l adds records l, l + 32, ... (all 28 floats of each,
-        // in that order), then a fixed xor tree joins the lanes. Same order on every run.
-        for (int k = 0; k < np; ++k) {
-          const int l = l0 + (p0 + k) * G;
-          const float4* rt = reinterpret_cast<const float4*>(recs + static_cast<size_t>(l) * G *
-                                                                         kFsRec);
-          float acc[kFsRec];
+      for (int p0 = 0; p0 < nown; p0 += kFsTokPerPass) {
+        const int k = p0 + grp;
+        const bool live = k < nown;
+        const int l = l0 + k * G;
+        // Lane gl of the token's group adds records gl, gl + kFsTokLanes, ... (all 28 floats of
+        // each, in that order); a fixed xor tree then joins the group's lanes. Same order on
+        // every run, and every lane of the group ends with the token's sums.
+        float acc[kFsRec];
 #pragma unroll
-          for (int c = 0; c < kFsRec; ++c) acc[c] = 0.f;
-          for (int rr = lane; rr < G; rr += 32) {
-            float4 v[7];
-#pragma unroll
-            for (int c = 0; c < 7; ++c) v[c] = __ldcg(rt + rr * 7 + c);
+        for (int c = 0; c < kFsRec; ++c) acc[c] = 0.f;
+        if (live) {
+          const float4* rt =
+              reinterpret_cast<const float4*>(recs + static_cast<size_t>(l) * G * kFsRec);
+          for (int rr = gl; rr < G; rr += 2 * kFsTokLanes) {
+            float4 v0[7], v1[7];
+            const bool two = rr + kFsTokLanes < G;
 #pragma unroll
             for (int c = 0; c < 7; ++c) {
-              acc[4 * c] += v[c].x;
-              acc[4 * c + 1] += v[c].y;
-              acc[4 * c + 2] += v[c].z;
-              acc[4 * c + 3] += v[c].w;
+              v0[c] = __ldcg(rt + rr * 7 + c);
+              v1[c] = two ? __ldcg(rt + (rr + kFsTokLanes) * 7 + c)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int c = 0; c < 7; ++c) {
+              acc[4 * c] += v0[c].x;
+              acc[4 * c + 1] += v0[c].y;
+              acc[4 * c + 2] += v0[c].z;
+              acc[4 * c + 3] += v0[c].w;
+            }
+#pragma unroll
+            for (int c = 0; c < 7; ++c) {
+              acc[4 * c] += v1[c].x;
+              acc[4 * c + 1] += v1[c].y;
+              acc[4 * c + 2] += v1[c].z;
+              acc[4 * c + 3] += v1[c].w;
             }
           }
-#pragma unroll
-          for (int sh = 16; sh >= 1; sh >>= 1) {
-#pragma unroll
-            for (int c = 0; c < 25; ++c) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], sh);
-          }
-          if (lane == 0) {
-#pragma unroll
-            for (int c = 0; c < 25; ++c) cs[k * kFsRec + c] = acc[c];
-          }
         }
-        __syncwarp();
-        // Quad `quad` forms token p0 + quad's coefficients; lane r: pre r, post r, comb row r.
-        const bool live = quad < np;
-        const int l = l0 + (p0 + quad) * G;
+#pragma unroll
+        for (int sh = kFsTokLanes / 2; sh >= 1; sh >>= 1) {
+#pragma unroll
+          for (int c = 0; c < 25; ++c) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], sh);
+        }
         const int64_t t = static_cast<int64_t>(X) * kFsM + l;
         float cr[4] = {0.f, 0.f, 0.f, 0.f};
         float pre_v = 0.f, post_v = 0.f;
         if (live) {
-          const float* sm = cs + quad * kFsRec;
           const float rstd = __fdiv_rn(
-              1.0f, __fsqrt_rn(__fdiv_rn(sm[24], static_cast<float>(a.K)) + a.fp.rms_eps));
-          const float lp = fmaf(sm[r] * rstd, __ldg(a.scale), __ldg(a.base + r));
-          const float lq = fmaf(sm[4 + r] * rstd, __ldg(a.scale + 1), __ldg(a.base + 4 + r));
+              1.0f, __fsqrt_rn(__fdiv_rn(acc[24], static_cast<float>(a.K)) + a.fp.rms_eps));
+          float g0 = acc[0], g1 = acc[4], c0 = acc[8], c1 = acc[9], c2 = acc[10], c3 = acc[11];
+          if (r == 1) g0 = acc[1], g1 = acc[5], c0 = acc[12], c1 = acc[13], c2 = acc[14], c3 = acc[15];
+          if (r == 2) g0 = acc[2], g1 = acc[6], c0 = acc[16], c1 = acc[17], c2 = acc[18], c3 = acc[19];
+          if (r == 3) g0 = acc[3], g1 = acc[7], c0 = acc[20], c1 = acc[21], c2 = acc[22], c3 = acc[23];
+          const float lp = fmaf(g0 * rstd, __ldg(a.scale), __ldg(a.base + r));
+          const float lq = fmaf(g1 * rstd, __ldg(a.scale + 1), __ldg(a.base + 4 + r));
           const float s2 = __ldg(a.scale + 2);
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            cr[c] = fmaf(sm[8 + 4 * r + c] * rstd, s2, __ldg(a.base + 8 + 4 * r + c));
+          cr[0] = fmaf(c0 * rstd, s2, __ldg(a.base + 8 + 4 * r));
+          cr[1] = fmaf(c1 * rstd, s2, __ldg(a.base + 9 + 4 * r));
+          cr[2] = fmaf(c2 * rstd, s2, __ldg(a.base + 10 + 4 * r));
+          cr[3] = fmaf(c3 * rstd, s2, __ldg(a.base + 11 + 4 * r));
           pre_v = sigmoidf_ieee(lp) + a.fp.pre_eps;
           post_v = a.fp.post_mult * sigmoidf_ieee(lq);
         }
         sinkhorn_quad(cr, a.fp.iters, a.fp.sinkhorn_eps);  // every lane takes part
-        if (live) {
+        if (live && gl < 4) {
           a.pre[t * 4 + r] = pre_v;
           a.post[t * 4 + r] = post_v;
 #pragma unroll
           for (int c = 0; c < 4; ++c) a.comb[t * 16 + 4 * r + c] = cr[c];
-          slot_pre[(slot * kFsMaxOwn + p0 + quad) * 4 + r] = pre_v;
-          if (r == 0) slot_tok[slot * kFsMaxOwn + p0 + quad] = l;
+          slot_pre[(slot * kFsMaxOwn + k) * 4 + r] = pre_v;
+          if (r == 0) slot_tok[slot * kFsMaxOwn + k] = l;
         }
         __syncwarp();
       }
@@ -735,7 +780,7 @@ int launch_pre_fused(const PreArgs& a, cudaStream_t s) {
   fa.NG = plan.NG;
   fa.nbmax = plan.nbmax;
   fa.stages = plan.stages;
-  fa.lag = kFsDefaultLag;
+  fa.lag = kFsLag;
   fa.fp = FinishParams{a.iters, a.sinkhorn_eps, a.rms_eps, a.pre_eps, a.post_mult};
 
   // Cooperative launch: every CTA resident at once (the groups' CTAs wait on one another). Also a

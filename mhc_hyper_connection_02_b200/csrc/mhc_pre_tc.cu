@@ -16,11 +16,12 @@
 //           issues TMA loads of two R sub-tiles [128 x 64] and one Bw tile [80 x 64] (128-byte
 //           swizzle) per stage into a 4-stage ring that runs on across pieces; warp 1 issues
 //           tcgen05.mma M=128 N=80 K=16 (four per 64-wide K block and sub-tile) into two TMEM
-//           accumulators sharing the B tile, double-buffered across pieces (512 columns), so the
-//           epilogue of one piece overlaps the loads of the next; warps 2-5 sum the squares of
-//           their token rows from the same shared-memory tiles and, after a piece, read its
-//           accumulators (tcgen05.ld) and write the record [slot][t][32] = raw[0..23], ss, slot =
-//           the piece's rank among its tile's pieces. The CTA holding a tile's last piece writes
+//           accumulators sharing the B tile. A piece is accumulated in sub-pieces of at most 16 K
+//           blocks, double-buffered in TMEM (512 columns), so the epilogue of one overlaps the
+//           loads of the next; warps 2-5 sum the squares of their token rows from the same
+//           shared-memory tiles, add each sub-piece's accumulators (tcgen05.ld) into registers,
+//           and after the piece write the record [slot][t][32] = raw[0..23], ss, slot = the
+//           piece's rank among its tile's pieces. The CTA holding a tile's last piece writes
 //           zero records into the tile's unused slots, so readers sum a fixed number of slots.
 //   coef    one token per lane quad: sums the slots in order, forms rstd, the logits, the gates
 //           and the Sinkhorn comb.
@@ -50,6 +51,11 @@ constexpr int kTcTmemCols = 512;                   // 2 buffers x 2 sub-tiles x 
 constexpr int kTcSmem = 1024 + kTcStages * kTcStageBytes + 256;
 constexpr int64_t kTcMaxCtas = 148;                // most CTAs the projection plan uses
 constexpr int64_t kTcMinBlocks = 8;                // K blocks per CTA at least (pipeline fill)
+// The tensor-core accumulator is restarted every kTcSubBlocks K blocks of a piece and the sub-piece
+// sums are added in registers: shorter accumulation chains in TMEM keep the projection's fp32
+// rounding error well inside the coefficient tolerance over K = 4H = 28672.
+constexpr int kTcSubBlocks = 16;
+constexpr int kTcAccDelay = 2;  // stages into the next sub-piece before a finished one is added
 
 // Work plan of the projection: W = ntiles * kblocks block-tiles over P CTAs; CTA c takes
 // [c W / P, (c + 1) W / P). A tile's K range is cut into at most S pieces.
@@ -263,20 +269,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) pre_tc_proj_kernel(
   } else if (warp == 1) {
     if (lane == 0) {
       int64_t n = 0;
-      int64_t p = 0;
+      int64_t sp = 0;  // sub-pieces issued (accumulator buffer sp & 1)
       bool ok = true;
-      for (int64_t u = lo; u < hi && ok; ++p) {
+      uint32_t dt = tmem;
+      for (int64_t u = lo; u < hi && ok;) {
         const int64_t tile = u / KB;
         const int kbs = static_cast<int>(u - tile * KB);
         const int kbe = static_cast<int>(min(static_cast<int64_t>(KB), kbs + (hi - u)));
-        const int b = static_cast<int>(p & 1);
-        if (p >= 2 && !mbar_wait(&aempty[b], static_cast<uint32_t>((p >> 1) - 1) & 1u, 16)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t dt = tmem + static_cast<uint32_t>(b * kTcSub * kTcM);
         for (int kb = kbs; kb < kbe; ++kb, ++n) {
+          const int ks = (kb - kbs) % kTcSubBlocks;  // position within the sub-piece
+          if (ks == 0) {
+            const int b = static_cast<int>(sp & 1);
+            if (sp >= 2 && !mbar_wait(&aempty[b], static_cast<uint32_t>((sp >> 1) - 1) & 1u, 16)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            dt = tmem + static_cast<uint32_t>(b * kTcSub * kTcM);
+          }
           const int s = static_cast<int>(n % kTcStages);
           const uint32_t ph = static_cast<uint32_t>(n / kTcStages) & 1u;
           if (!mbar_wait(&full[s], ph, 11)) {
@@ -292,12 +302,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) pre_tc_proj_kernel(
 #pragma unroll
             for (int k = 0; k < kTcKB / 16; ++k)  // +32 bytes along the swizzled row per K=16 step
               umma_bf16(dt + static_cast<uint32_t>(v * kTcM), adesc + 2 * k, bdesc + 2 * k,
-                        (kb > kbs || k > 0) ? 1u : 0u);
+                        (ks > 0 || k > 0) ? 1u : 0u);
           }
           umma_commit(&empty[s]);
+          if (kb + 1 == kbe || ks + 1 == kTcSubBlocks) {
+            umma_commit(&afull[sp & 1]);
+            ++sp;
+          }
         }
-        if (!ok) break;
-        umma_commit(&afull[b]);
         u += kbe - kbs;
       }
       // Every issued MMA has finished before TMEM is released.
@@ -307,18 +319,51 @@ __global__ void __launch_bounds__(kTcThreads, 1) pre_tc_proj_kernel(
   } else {
     // Warps 2..5: TMEM lane quarter q = warp % 4 holds rows 32q..32q+31 of each sub-tile's
     // accumulator; the same thread sums the squares of those rows (one per sub-tile).
-    const int q = warp & 3;
-    const int row = q * 32 + lane;
+    const int q_lane = warp & 3;
+    const int row = q_lane * 32 + lane;
     int64_t n = 0;
-    int64_t p = 0;
+    int64_t sp = 0;     // sub-pieces the MMA warp has been asked to finish
+    int64_t pend = -1;  // finished sub-piece whose accumulators are not yet added
     bool ok = true;
-    for (int64_t u = lo; u < hi && ok; ++p) {
+    float racc[kTcSub][kMix];
+    // Adds sub-piece q's accumulators (TMEM buffer q & 1) to the piece's sums; false on timeout.
+    auto add_sub = [&](int64_t q) -> bool {
+      const int b = static_cast<int>(q & 1);
+      if (!__all_sync(0xffffffffu, mbar_wait(&afull[b], static_cast<uint32_t>(q >> 1) & 1u, 13)))
+        return false;
+      tc_fence_after();
+#pragma unroll
+      for (int v = 0; v < kTcSub; ++v) {
+        uint32_t d[5][16];
+        const uint32_t tbase = tmem + static_cast<uint32_t>((b * kTcSub + v) * kTcM) +
+                               (static_cast<uint32_t>(q_lane * 32) << 16);
+#pragma unroll
+        for (int cc = 0; cc < 5; ++cc) tmem_ld16(tbase + cc * 16, d[cc]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < kMix; ++j) {
+          const float hi3 = __uint_as_float(d[j / 16][j % 16]);
+          const float mid = __uint_as_float(d[(kMix + j) / 16][(kMix + j) % 16]);
+          const float lo3 = __uint_as_float(d[(2 * kMix + j) / 16][(2 * kMix + j) % 16]);
+          racc[v][j] += (lo3 + mid) + hi3;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&aempty[b]);
+      return true;
+    };
+    for (int64_t u = lo; u < hi && ok;) {
       const int64_t tile = u / KB;
       const int kbs = static_cast<int>(u - tile * KB);
       const int kbe = static_cast<int>(min(static_cast<int64_t>(KB), kbs + (hi - u)));
       float ss0[kTcSub], ss1[kTcSub];
 #pragma unroll
-      for (int v = 0; v < kTcSub; ++v) ss0[v] = ss1[v] = 0.f;
+      for (int v = 0; v < kTcSub; ++v) {
+        ss0[v] = ss1[v] = 0.f;
+#pragma unroll
+        for (int j = 0; j < kMix; ++j) racc[v][j] = 0.f;
+      }
       for (int kb = kbs; kb < kbe; ++kb, ++n) {
         const int s = static_cast<int>(n % kTcStages);
         const uint32_t ph = static_cast<uint32_t>(n / kTcStages) & 1u;
@@ -349,38 +394,38 @@ __global__ void __launch_bounds__(kTcThreads, 1) pre_tc_proj_kernel(
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
+        const int ks = (kb - kbs) % kTcSubBlocks;
+        // A finished sub-piece is added a few stages into the next one (its MMAs are done by
+        // then, so this never holds the stage ring back); the last one at the end of the piece.
+        if (pend >= 0 && ks == kTcAccDelay) {
+          if (!add_sub(pend)) {
+            ok = false;
+            break;
+          }
+          pend = -1;
+        }
+        if (kb + 1 == kbe || ks + 1 == kTcSubBlocks) {
+          if (pend >= 0 && !add_sub(pend)) {
+            ok = false;
+            break;
+          }
+          pend = sp++;
+        }
       }
+      if (ok && pend >= 0 && !add_sub(pend)) ok = false;
+      pend = -1;
       if (!ok) break;
-      const int b = static_cast<int>(p & 1);
-      if (!__all_sync(0xffffffffu, mbar_wait(&afull[b], static_cast<uint32_t>(p >> 1) & 1u, 13))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
       const int64_t slot = c - tc_first_cta(tile * KB, P, W);
       const bool last_piece = (kbe == KB);
 #pragma unroll
       for (int v = 0; v < kTcSub; ++v) {
-        uint32_t d[5][16];
-        const uint32_t tbase = tmem + static_cast<uint32_t>((b * kTcSub + v) * kTcM) +
-                               (static_cast<uint32_t>(q * 32) << 16);
-#pragma unroll
-        for (int cc = 0; cc < 5; ++cc) tmem_ld16(tbase + cc * 16, d[cc]);
-        tmem_wait_ld();
         const int64_t t = tile * kTcTile + v * kTcM + row;
         if (t < T) {
-          float raw[kMix];
-#pragma unroll
-          for (int j = 0; j < kMix; ++j) {
-            const float hi3 = __uint_as_float(d[j / 16][j % 16]);
-            const float mid = __uint_as_float(d[(kMix + j) / 16][(kMix + j) % 16]);
-            const float lo3 = __uint_as_float(d[(2 * kMix + j) / 16][(2 * kMix + j) % 16]);
-            raw[j] = (lo3 + mid) + hi3;
-          }
           float4* rec = reinterpret_cast<float4*>(part + (slot * T + t) * 32);
 #pragma unroll
           for (int w = 0; w < 6; ++w)
-            rec[w] = make_float4(raw[4 * w], raw[4 * w + 1], raw[4 * w + 2], raw[4 * w + 3]);
+            rec[w] = make_float4(racc[v][4 * w], racc[v][4 * w + 1], racc[v][4 * w + 2],
+                                 racc[v][4 * w + 3]);
           rec[6] = make_float4(ss0[v] + ss1[v], 0.f, 0.f, 0.f);
           if (last_piece) {
             const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -392,9 +437,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) pre_tc_proj_kernel(
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&aempty[b]);
       u += kbe - kbs;
     }
   }

@@ -40,13 +40,18 @@ def call_noalloc(R, W, S, B, T, H, params):
     return y, pre, post, comb
 
 
-def assert_close(new, ref):
+def assert_close(new, ref, R_bits):
+    """The entry against mhc_pre: coefficients within the tolerance (1e-5); y under the bf16 rule,
+    or, where y cancels, within one ulp plus what the two calls' admitted coefficient differences
+    (each within 1e-5 of the oracle, so 2e-5 apart) and fp32 evaluation carry into y."""
     for a, b, name in zip(new[1:], ref[1:], ("pre", "post", "comb")):
         d = (a.double() - b.double()).abs().max().item()
         assert d <= COEF_TOL, f"{name}: {d}"
     yn = bf16_bits_to_f64(new[0].view(torch.int16).cpu().numpy().view(np.uint16))
     yr = bf16_bits_to_f64(ref[0].view(torch.int16).cpu().numpy().view(np.uint16))
-    tol = np.maximum(ulp_bf16(yr), REL * np.abs(yr))
+    rsum = np.abs(bf16_bits_to_f64(R_bits)).sum(axis=1)
+    u = ulp_bf16(yr)
+    tol = np.maximum(np.maximum(u, REL * np.abs(yr)), 2 * u + (2 * COEF_TOL + 12 * U32) * rsum)
     assert np.all(np.abs(yn - yr) <= tol)
 
 
@@ -73,7 +78,7 @@ def test_noalloc_matches_mhc_pre_on_two_calls_in_a_row():
         ref = mhc.pre(R, W, S, B, params=params)
         torch.cuda.synchronize()
         assert mhc.device_status() == 0
-        assert_close(new, ref)
+        assert_close(new, ref, w.R)
         assert_matches_oracle(new, w, np.arange(w.T))
 
 
@@ -88,7 +93,7 @@ def test_noalloc_at_its_exact_scratch_limit():
     ref = mhc.pre(R, W, S, B, params=params)
     torch.cuda.synchronize()
     assert mhc.device_status() == 0
-    assert_close(new, ref)
+    assert_close(new, ref, w.R)
     rows = np.unique(np.concatenate([np.arange(0, 64), np.arange(w.T - 64, w.T),
                                      np.random.default_rng(5).choice(w.T, 256, replace=False)]))
     assert_matches_oracle(new, w, rows)
