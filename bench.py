@@ -120,19 +120,45 @@ def oracle_sample(w, n_tokens):
     return n_tokens / dt, dt, oracle.threads()
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(w, budget_s=12.0, max_passes=50):
     """Bounded sample: calibrate on a few tokens, then time about budget_s seconds of oracle work
     (the first n tokens, n <= T; when one pass over them takes less than budget_s, repeated
-    passes until budget_s has elapsed)."""
-    rate, _, _ = oracle_sample(w, 16)
-    n = int(max(16, min(w.T, rate * budget_s)))
-    tot, passes, cores = 0.0, 0, 1
-    while passes < max_passes and (passes == 0 or tot < budget_s):
-        _, dt, cores = oracle_sample(w, n)
-        tot += dt
-        passes += 1
-    return {"value": n * passes / tot, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"first {n} of {w.T} tokens (pre+post), {passes} pass(es), {tot:.1f} s"}
+    passes until budget_s has elapsed), on all of the host's OpenMP threads and then on one."""
+    import oracle
+
+    def timed(budget):
+        rate, _, _ = oracle_sample(w, 16)
+        n = int(max(16, min(w.T, rate * budget)))
+        tot, passes, cores = 0.0, 0, 1
+        while passes < max_passes and (passes == 0 or tot < budget):
+            _, dt, cores = oracle_sample(w, n)
+            tot += dt
+            passes += 1
+        return n * passes / tot, n, passes, tot, cores
+
+    all_threads = oracle.threads()
+    v, n, passes, tot, cores = timed(budget_s)
+    oracle.set_threads(1)
+    try:
+        v1, n1, p1, t1, _ = timed(budget_s / 3)
+    finally:
+        oracle.set_threads(all_threads)
+    return {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"first {n} of {w.T} tokens (pre+post), {passes} pass(es), {tot:.1f} s",
+            "value_1_thread": v1,
+            "sample_1_thread": f"first {n1} of {w.T} tokens (pre+post), {p1} pass(es), {t1:.1f} s",
+            "cpu_model": cpu_model()}
 
 
 def dist_env():
@@ -312,6 +338,30 @@ def time_configs(mhc, inputs, dev, stream, reps=20):
             ts.append(a.elapsed_time(b) * 1e3)
         return statistics.median(ts)
 
+    def graph_timed(call, n=10, reps=10):
+        """Device time per call when n calls replay from one CUDA graph (a serving loop's setting:
+        no per-call launch or event overhead), queued behind the spin like timed()."""
+        gs = torch.cuda.Stream(dev)
+        gs.wait_stream(stream)
+        with torch.cuda.stream(gs):
+            call(gs)  # first-call setup outside the capture
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=gs):
+            for _ in range(n):
+                call(gs)
+        ts = []
+        for _ in range(reps):
+            torch.cuda._sleep(2000000)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b) * 1e3 / n)
+        del g
+        return statistics.median(ts)
+
     def one(w, do_pre=True):
         R, x = dev_bf16(w.R), dev_bf16(w.x)
         W, sc, bs = (torch.from_numpy(a).to(dev) for a in (w.hc_fn, w.hc_scale, w.hc_base))
@@ -333,10 +383,21 @@ def time_configs(mhc, inputs, dev, stream, reps=20):
             us = timed(fq, flushed)
             rec[f"post_us_{tag}"] = us
             rec[f"post_GBps_{tag}"] = post_bytes(w.T, w.H) / us / 1e3
+        if w.T <= 64:  # latency-bound shapes: also per call from a replayed CUDA graph
+            if do_pre:
+                rec["pre_us_graph"] = graph_timed(
+                    lambda st: mhc.pre(R, W, sc, bs, y=y, pre=pre, post=post, comb=comb,
+                                       workspace=ws, params=prm, stream=st))
+            rec["post_us_graph"] = graph_timed(
+                lambda st: mhc.post(x, R, post, comb, out=out, stream=st))
         return rec
 
     res = {"small": one(inputs.small()), "post4k": one(inputs.post4k(), do_pre=False),
            "tail": one(inputs.tail())}
+    # What the event-timed method reports for one trivial kernel: a floor under every *_us figure
+    # above (launch and event timestamp latency), not time spent in the library's kernels.
+    tiny = torch.empty(1, device=dev)
+    res["event_floor_us"] = timed(lambda: tiny.add_(1), False)
     for T in (1, 4, 16, 32):
         res[f"decode_T{T}"] = one(inputs.decode(T))
     assert mhc.device_status() == 0
@@ -566,6 +627,17 @@ def main():
             "e2e": e2e,
         }
         if do_pre:
+            # The pre-map's own roofline object: the whole call (its kernels chained by
+            # programmatic dependent launch), algorithmic bytes over the call's event time.
+            pre_traffic_rec = load_traffic().get(f"pre:{args.workload}")
+            pre_traffic = None
+            if pre_traffic_rec and pre_traffic_rec.get("source") == source_digest("pre"):
+                pre_traffic = pre_traffic_rec.get("bytes_per_call")
+            line["pre_roofline"] = {
+                "bound": "hbm", "kernel": "mhc_pre (whole call)", "achieved": pre_gbs,
+                "peak": hbm, "unit": "GB/s", "frac": pre_gbs / hbm, "traffic": pre_traffic,
+                "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)",
+                "path": args.pre_path}
             line["kernels"]["pre"] = {
                 "us": pre_avg_s * 1e6, "algo_bytes": qb, "GBps": pre_gbs,
                 "frac_measured": pre_gbs / hbm, "frac_8TBps": pre_gbs / 8000.0,

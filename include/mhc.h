@@ -112,6 +112,11 @@ MHC_API mhc_params mhc_default_params(void);
  * MHC_ERR_WORKSPACE_TOO_SMALL; MHC_ERR_ALIAS when y, pre, post or comb overlaps R or one another.
  * Any H >= 1 is accepted (FlashInfer requires H % 8 == 0; here other H take a scalar path), as is
  * any alignment of the arrays.
+ *
+ * Kernel choice (MHC_PATH_AUTO): T < 128, odd H or unaligned R / workspace: the CUDA-core split-K
+ * path; otherwise the tcgen05 projection, as the single-pass kernel where it is faster (up to
+ * about 1.5k tokens with H >= ~2k, 16-byte aligned y, H % 8 == 0), else the split chain. Every
+ * path computes the same values within the stated tolerances.
  */
 MHC_API int mhc_pre(const uint16_t* R, const float* hc_fn, const float* hc_scale, const float* hc_base,
             uint16_t* y, float* pre, float* post, float* comb, void* workspace,
@@ -162,13 +167,16 @@ enum mhc_path {
     MHC_PATH_AUTO = 0,
     /* pre */
     MHC_PRE_PATH_CUDA_CORE = 1, /* fp32 CUDA-core split-K projection + finish kernel */
-    MHC_PRE_PATH_TENSOR = 2,    /* tcgen05 projection (exact bf16 x3 split of hc_fn), the
-                                   fastest tensor-core variant: currently the split pair */
+    MHC_PRE_PATH_TENSOR = 2,    /* tcgen05 projection (exact bf16 x3 split of hc_fn) as the split
+                                   chain (MHC_PATH_AUTO may take the single pass instead) */
     MHC_PRE_PATH_TENSOR_SPLIT = 3, /* tcgen05 split-K projection kernel, then a coefficient kernel
                                       and a streaming aggregate kernel; H even */
-    MHC_PRE_PATH_TENSOR_FUSED = 4, /* one persistent kernel (projection, cross-CTA reduction,
-                                      coefficients, aggregate); H % 8 == 0 and R, y, pre, comb and
-                                      the workspace 16-byte aligned */
+    MHC_PRE_PATH_TENSOR_FUSED = 4, /* one pass over R: a persistent cooperative kernel (projection
+                                      with hc_fn slices resident in shared memory, cross-CTA
+                                      reduction, coefficients, aggregate from L2) after a counter
+                                      reset; H % 8 == 0, H >= 64, R, y and the workspace 16-byte
+                                      aligned; MHC_ERR_UNSUPPORTED, with nothing launched, when
+                                      the device cannot hold its grid resident */
     /* post */
     MHC_POST_PATH_VEC8 = 11,       /* 16-byte vector loads/stores; H % 8 == 0, 16-byte aligned */
     MHC_POST_PATH_PERSISTENT = 12, /* persistent, bulk-copy (TMA) staged; same requirements */

@@ -256,8 +256,10 @@ int mhc_pre_with_path(const uint16_t* R, const float* hc_fn, const float* hc_sca
   // The fused kernel also uses 16-byte accesses on y, pre and comb.
   const bool fused_ok = tc_ok && pre_fused_supported(T, H) && aligned16(y) && aligned16(pre) &&
                         aligned16(comb);
+  bool auto_fused = false;
   if (path == MHC_PATH_AUTO) {
     path = (tc_ok && T >= kPreTensorMinTokens) ? MHC_PRE_PATH_TENSOR : MHC_PRE_PATH_CUDA_CORE;
+    auto_fused = path == MHC_PRE_PATH_TENSOR && fused_ok && pre_fused_preferred(T, H);
   } else if ((path == MHC_PRE_PATH_TENSOR || path == MHC_PRE_PATH_TENSOR_SPLIT) && !tc_ok) {
     return MHC_ERR_UNSUPPORTED;
   } else if (path == MHC_PRE_PATH_TENSOR_FUSED && !fused_ok) {
@@ -268,10 +270,12 @@ int mhc_pre_with_path(const uint16_t* R, const float* hc_fn, const float* hc_sca
   PreArgs a{R, hc_fn, hc_scale, hc_base, y, pre, post, comb, workspace, workspace_bytes, T, H,
             prm.sinkhorn_iters, prm.sinkhorn_eps, prm.rms_eps, prm.pre_eps, prm.post_mult};
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (path == MHC_PRE_PATH_TENSOR_FUSED) {
-    // 1: the grid cannot be co-scheduled on this device right now; nothing was launched.
+  if (path == MHC_PRE_PATH_TENSOR_FUSED || auto_fused) {
+    // 1: the grid cannot run with every CTA resident on this device; nothing was launched. A
+    // forced single pass reports it; the automatic choice falls back to the split chain.
     const int r = launch_pre_fused(a, s);
-    return r == 1 ? MHC_ERR_UNSUPPORTED : r;
+    if (r != 1) return r;
+    if (!auto_fused) return MHC_ERR_UNSUPPORTED;
   }
   if (path != MHC_PRE_PATH_CUDA_CORE) return launch_pre_tc(a, s);
   return launch_pre_cc(a, s);

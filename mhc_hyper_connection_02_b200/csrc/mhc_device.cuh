@@ -218,4 +218,36 @@ __device__ __forceinline__ void sinkhorn_quad(float (&a)[4], int iters, float ep
   }
 }
 
+// The same Sinkhorn for one whole 4x4 block in one thread (a[4 * o + n], [old][new]): no
+// shuffles, half the instructions per token of the lane-quad form, for calls with many tokens.
+// Sums are associated exactly as in sinkhorn_quad (rows ((a0 + a1) + a2) + a3, columns
+// (a0 + a1) + (a2 + a3)), so the two forms give identical results.
+__device__ __forceinline__ void sinkhorn_thread(float (&a)[16], int iters, float eps) {
+#pragma unroll
+  for (int o = 0; o < 4; ++o) {
+    float* r = a + 4 * o;
+    const float m = fmaxf(fmaxf(r[0], r[1]), fmaxf(r[2], r[3]));
+#pragma unroll
+    for (int n = 0; n < 4; ++n) r[n] = expf(r[n] - m);
+    const float rs0 = recip_nr(((r[0] + r[1]) + r[2]) + r[3]);
+#pragma unroll
+    for (int n = 0; n < 4; ++n) r[n] = fmaf(r[n], rs0, eps);
+  }
+  for (int it = 0; it < iters; ++it) {
+#pragma unroll
+    for (int o = 0; o < 4; ++o) {
+      float* r = a + 4 * o;
+      const float rr = recip_nr(((r[0] + r[1]) + r[2]) + r[3]);
+#pragma unroll
+      for (int n = 0; n < 4; ++n) r[n] *= rr;
+    }
+#pragma unroll
+    for (int n = 0; n < 4; ++n) {
+      const float rc = recip_nr((a[n] + a[4 + n]) + (a[8 + n] + a[12 + n]));
+#pragma unroll
+      for (int o = 0; o < 4; ++o) a[4 * o + n] *= rc;
+    }
+  }
+}
+
 }  // namespace mhc

@@ -82,9 +82,10 @@ int launch_pre_cc(const PreArgs& a, cudaStream_t s);
 // Its projection step alone: records [nrec][T][32] (raw[24], ss) at the workspace start.
 int launch_cc_projection(const PreArgs& a, cudaStream_t s, float** part, int* nrec);
 
-// Tensor-core path: persistent fused kernel (launch returns 1 when the device cannot co-schedule
-// its grid; the caller then takes the split pair).
+// Tensor-core path: single-pass persistent kernel (launch returns 1, having launched nothing, when
+// the device cannot run its grid with every CTA resident).
 bool pre_fused_supported(int64_t T, int64_t H);
+bool pre_fused_preferred(int64_t T, int64_t H);
 size_t pre_fused_workspace_bytes(int64_t T, int64_t H);
 int launch_pre_fused(const PreArgs& a, cudaStream_t s);
 

@@ -126,6 +126,15 @@ static FsPlan fs_plan(int64_t T, int64_t H, int sms) {
 
 bool pre_fused_supported(int64_t T, int64_t H) { return fs_plan(T, H, kFsMaxCtas).ok; }
 
+// Where the single pass is the faster of the two tensor-core forms (measured on B200, device time):
+// a few tiles per group (T up to ~1.5k tokens) and groups wide enough that each CTA owns at most
+// 8 tokens of a tile. T=256..1024 at H=4096/7168: 24-50 us against 32-69 us for the split chain;
+// from T=2048 (H=4096) and T=3072 (H=7168), or with narrow groups (H=1000), the split chain wins.
+bool pre_fused_preferred(int64_t T, int64_t H) {
+  const FsPlan p = fs_plan(T, H, kFsMaxCtas);
+  return p.ok && T <= 1536 && p.G >= 16;
+}
+
 size_t pre_fused_workspace_bytes(int64_t T, int64_t H) {
   // The largest plan: records for every CTA of a full-size launch. Plans on devices with fewer SMs
   // need no more.

@@ -25,6 +25,7 @@ from .c_oracle import (  # noqa: F401
     pre,
     post,
     threads,
+    set_threads,
 )
 from .big_fuse import big_fuse, big_fuse_with_prenorm, sum_of_squares  # noqa: F401
 from . import boundary  # noqa: F401

@@ -63,6 +63,7 @@ def _load():
                                    ctypes.c_double, _D, _D, _D, _D, _D, _D]
     lib.mhc_oracle_post.argtypes = [_U16, _U16, _F, _F, _I64, _I64, _D]
     lib.mhc_oracle_threads.restype = ctypes.c_int
+    lib.mhc_oracle_set_threads.argtypes = [ctypes.c_int]
     _lib = lib
     return lib
 
@@ -74,6 +75,11 @@ def _c(a, dtype, ptr):
 
 def threads() -> int:
     return int(_load().mhc_oracle_threads())
+
+
+def set_threads(n: int) -> None:
+    """OpenMP threads for later oracle calls (the CPU baseline times 1 thread and all of them)."""
+    _load().mhc_oracle_set_threads(int(n))
 
 
 def bf16_bits_to_f64(bits) -> np.ndarray:

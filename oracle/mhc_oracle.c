@@ -25,6 +25,14 @@ int mhc_oracle_threads(void) {
 #endif
 }
 
+void mhc_oracle_set_threads(int n) {
+#ifdef _OPENMP
+    if (n >= 1) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 double mhc_oracle_bf16_to_double(uint16_t bits) {
     uint32_t u = (uint32_t)bits << 16;
     float f;

@@ -88,6 +88,9 @@ void mhc_oracle_post(const uint16_t* x, const uint16_t* R, const float* post, co
 /* Number of OpenMP threads the oracle runs with (1 when built without OpenMP). */
 int mhc_oracle_threads(void);
 
+/* Sets the number of OpenMP threads later calls use (n >= 1; no effect without OpenMP). */
+void mhc_oracle_set_threads(int n);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,6 +1,7 @@
 """The library's calls under CUDA graph capture (the launch-bound serving loop): one pre-map +
 post-map step captured once and replayed gives bitwise the eager results, for the tensor-core
-path (chained with programmatic dependent launch) and the CUDA-core decode path."""
+split chain (chained with programmatic dependent launch), the single-pass cooperative kernel
+(T=512, H=7168) and the CUDA-core decode path."""
 
 import numpy as np
 import pytest
@@ -13,7 +14,7 @@ from gpu_util import dev_bf16, dev_f32
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("T,H", [(4, 7168), (256, 1024)])
+@pytest.mark.parametrize("T,H", [(4, 7168), (256, 1024), (512, 7168)])
 def test_graph_replay_matches_eager(T, H):
     w = inputs.custom(T, H, seed=T + H)
     R, x = dev_bf16(w.R), dev_bf16(w.x)

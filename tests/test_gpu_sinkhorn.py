@@ -56,3 +56,28 @@ def test_sinkhorn_large_eps_and_many_rounds():
         torch.cuda.synchronize()
         check_coef(got.cpu().numpy(), oracle.sinkhorn(logits.astype(np.float64), iters, eps),
                    f"iters={iters} eps={eps}")
+
+
+@pytest.mark.parametrize("std,iters", [(1.0, 20), (3.0, 50)])
+def test_sinkhorn_one_thread_per_token_form(std, iters):
+    """From 65536 tokens the call runs one thread per token (16 registers, no shuffles). Every
+    token against the oracle, aligned, unaligned and in place; and bit for bit the lane-quad
+    form's result on the same logits (the sums are associated the same way)."""
+    T = 70001
+    rng = np.random.default_rng(int(std * 100) + iters)
+    logits = (rng.standard_normal((T, 4, 4)) * std).astype(np.float32)
+    ref = oracle.sinkhorn(logits.astype(np.float64), iters=iters, eps=1e-6)
+    dev = torch.from_numpy(logits).cuda()
+    got = mhc.sinkhorn(dev, iters=iters, eps=1e-6)
+    big = torch.zeros(T * 16 + 1, device="cuda")
+    big[1:] = dev.view(-1)
+    got_u = mhc.sinkhorn(big[1:].view(T, 4, 4), iters=iters, eps=1e-6)
+    inplace = dev.clone()
+    mhc.sinkhorn(inplace, comb=inplace, iters=iters, eps=1e-6)
+    quad = mhc.sinkhorn(dev[:4000].contiguous(), iters=iters, eps=1e-6)  # the lane-quad form
+    torch.cuda.synchronize()
+    assert mhc.device_status() == 0
+    for g, name in ((got, "aligned"), (got_u, "unaligned"), (inplace, "in place")):
+        d = check_coef(g.cpu().numpy(), ref, f"thread form {name}")
+        print(f"[sinkhorn thread form {name} std={std} iters={iters}] max|d|={d:.2e}")
+    assert torch.equal(got[:4000], quad)
