@@ -18,12 +18,12 @@
 //   warps 2-5   sum of squares of each token row from the same stages; after the tile, the
 //               accumulator (tcgen05.ld) gives the partial record rec[token][j] = raw[24], ss, and
 //               one thread release-increments the tile's counter.
-//   warps 6-9   (tile n by warp 6 + n mod 4) once the counter reaches G: for the tokens this CTA
+//   warps 6-7   (tile n by warp 6 + n mod 2) once the counter reaches G: for the tokens this CTA
 //               owns in the tile (token l with (l + 128 n) mod G == j), two at a time, sixteen
 //               lanes per token sum its G partial records in a fixed order; then rstd, the logits,
 //               the gates and the Sinkhorn comb; write pre, post and comb, and hand pre to the
 //               aggregate warps through shared memory.
-//   warps 10-15 y = bf16_rn(sum_i pre_i R_i) for the owned tokens, re-reading their rows with
+//   warps 8-15  y = bf16_rn(sum_i pre_i R_i) for the owned tokens, re-reading their rows with
 //               16-byte loads. The tile came from HBM a few microseconds earlier and is still in
 //               L2, so HBM sees R once.
 //
@@ -54,28 +54,28 @@ constexpr int kFsMaxOwn = kFsM / kFsMinG;    // most tokens a CTA owns in one ti
 constexpr int kFsMaxStages = 8;
 constexpr int kFsRec = 28;                   // floats per partial record (raw[24], ss, 3 zero)
 constexpr int kFsEpiDelay = 3;              // stages into the next tile before the records
-constexpr int kFsCoefWarps = 4;
+constexpr int kFsCoefWarps = 2;
 constexpr int kFsTokLanes = 16;              // lanes that reduce one token's records
 constexpr int kFsTokPerPass = 32 / kFsTokLanes;
-constexpr int kFsSlots = kFsCoefWarps;       // coefficient -> aggregate hand-over slots
+constexpr int kFsSlots = 8;                  // coefficient -> aggregate hand-over slots
 constexpr int kFsCoefWarp0 = 6;
 constexpr int kFsAggWarp0 = kFsCoefWarp0 + kFsCoefWarps;
-constexpr int kFsAggWarps = 16 - kFsAggWarp0;
-constexpr int kFsThreads = 512;
+constexpr int kFsAggWarps = 8;
+constexpr int kFsThreads = 32 * (kFsAggWarp0 + kFsAggWarps);
 constexpr int kFsTmemCols = 256;             // accumulators at columns 0 and 128
 constexpr int kFsMaxCtas = 148;              // most CTAs a plan uses (workspace sizing)
 constexpr int kFsSmemLimit = 227 * 1024;
 // D: the stream of tile n waits for this CTA's coefficients of tile n - D. D < kFsSlots keeps that
 // wait unambiguous (the slot cannot have moved on by two phases), and a record ring of 2 D tiles
 // is then never overwritten before every CTA of the group has read it.
-constexpr int kFsLag = 3;
+constexpr int kFsLag = 4;
 constexpr int kFsRing = 2 * kFsLag;
 static_assert(kFsLag < kFsSlots, "lag must stay below the hand-over slots");
 
 // Shared-memory scratch after the rings: barriers, TMEM address, coefficient sums, hand-over.
-constexpr int kFsOffBars = 0;      // full[8] empty[8] afull[2] aempty[2] cfull[4] cempty[4] done
-constexpr int kFsOffTmem = 240;
-constexpr int kFsOffPre = 256;                                         // float [slots][own][4]
+constexpr int kFsOffBars = 0;  // full[8] empty[8] afull[2] aempty[2] cfull[slots] cempty[slots] done
+constexpr int kFsOffTmem = (2 * kFsMaxStages + 4 + 2 * kFsSlots + 1) * 8;
+constexpr int kFsOffPre = (kFsOffTmem + 4 + 127) / 128 * 128;          // float [slots][own][4]
 constexpr int kFsOffTok = kFsOffPre + kFsSlots * kFsMaxOwn * 16;       // int [slots][own]
 constexpr int kFsOffNown = kFsOffTok + kFsSlots * kFsMaxOwn * 4;       // int [slots]
 constexpr int kFsMisc = (kFsOffNown + kFsSlots * 4 + 127) / 128 * 128;
@@ -274,7 +274,6 @@ __global__ void __launch_bounds__(kFsThreads, 1)
   float* slot_pre = reinterpret_cast<float*>(misc + kFsOffPre);
   int* slot_tok = reinterpret_cast<int*>(misc + kFsOffTok);
   int* slot_nown = reinterpret_cast<int*>(misc + kFsOffNown);
-  static_assert((2 * kFsMaxStages + 4 + 2 * kFsSlots + 1) * 8 <= kFsOffTmem, "barrier area");
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
