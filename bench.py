@@ -212,7 +212,7 @@ def load_traffic():
 # DRAM traffic figure is used only while their digest matches the one it was recorded with.
 KERNEL_SOURCES = {
     "post": ["mhc_post.cu", "mhc_device.cuh"],
-    "pre": ["mhc_pre_tc.cu", "mhc_pre_cc.cu", "mhc_device.cuh"],
+    "pre": ["mhc_pre_tc.cu", "mhc_pre_cc.cu", "mhc_pre_fused.cu", "mhc_api.cu", "mhc_device.cuh"],
 }
 
 

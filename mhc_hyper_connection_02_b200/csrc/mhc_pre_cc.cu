@@ -126,14 +126,14 @@ __global__ void __launch_bounds__(256) pre_cc_partial_kernel(const uint16_t* __r
   }
 }
 
-// Decode-sized calls (T <= 16): lanes run along K instead of along tokens. Thread i of split s
+// Decode-sized calls (T <= 8): lanes run along K instead of along tokens. Thread i of split s
 // owns k = s*KS + i (and k + 256 when KS > 256): it loads that k's 24 hc_fn weights once and the
 // row's value of every token up front, then per token forms its 24 products and its square, and a
 // butterfly reduce-scatter over the warp (31 shuffles) leaves lane j holding the warp's sum of
 // component j. The 8 warp sums are added in warp order. One hc_fn read per call, every load
 // issued before any is used: the step is a few round trips of latency.
 constexpr int kKlPer = 2;          // k values per thread at most (KS <= 512)
-constexpr int kKlMaxTokens = 16;   // above this the lane-per-token kernel is faster (measured)
+constexpr int kKlMaxTokens = 8;    // above this the staged lane-per-token kernel is faster (measured)
 
 template <bool kAlignedW>
 __global__ void __launch_bounds__(256) pre_cc_partial_klane_kernel(const uint16_t* __restrict__ R,
@@ -210,7 +210,7 @@ __global__ void __launch_bounds__(256) pre_cc_partial_klane_kernel(const uint16_
   }
 }
 
-// Decode-sized calls with more tokens (16 < T <= 32): lane = token as in pre_cc_partial_kernel,
+// Decode-sized calls with more tokens (8 < T <= 32): lane = token as in pre_cc_partial_kernel,
 // but the split's hc_fn rows (KS x 24 fp32, at most 48 KB) are first copied into shared memory
 // with coalesced loads, so the loop reads them from shared memory (one broadcast per row) instead
 // of waiting on global memory for every eight k.

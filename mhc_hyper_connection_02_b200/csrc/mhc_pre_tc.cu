@@ -23,11 +23,11 @@
 //           and after the piece write the record [slot][t][32] = raw[0..23], ss, slot = the
 //           piece's rank among its tile's pieces. The CTA holding a tile's last piece writes
 //           zero records into the tile's unused slots, so readers sum a fixed number of slots.
-//   coef    one token per lane quad: sums the slots in order, forms rstd, the logits, the gates
-//           and the Sinkhorn comb.
-//   agg     y = bf16_rn(sum_i pre_i R_i), one thread per (token, 8 columns): R read once more,
-//           y written once. (Unaligned R / y / pre or H % 8 != 0: the CUDA-core path's finish
-//           kernel replaces coef + agg, on the same records.)
+//   coef+agg  four tokens per CTA: warp 0 sums each token's slots in order (a lane quad per
+//           token), forms rstd, the logits and the pre gates; then the whole CTA writes
+//           y = bf16_rn(sum_i pre_i R_i) for those tokens (R read once more, y written once); then
+//           warp 0 runs the Sinkhorn and writes post and comb. (Unaligned R / y or H % 8 != 0: the
+//           CUDA-core path's finish kernel takes the same records instead.)
 #include <cuda.h>
 
 #include <mutex>
@@ -450,54 +450,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) pre_tc_proj_kernel(
   }
 }
 
-// Coefficients from the records [slot][t][32] (raw[0..23], ss): one token per lane quad, 8 tokens
-// per warp. Lane r of a quad sums, over the slots in order, the components it needs (pre r, post
-// r, comb row r, ss) and runs its row of the Sinkhorn.
-__global__ void __launch_bounds__(256) pre_tc_coef_kernel(const float* __restrict__ part,
-                                                          int nslot,
-                                                          const float* __restrict__ scale,
-                                                          const float* __restrict__ base,
-                                                          float* __restrict__ pre,
-                                                          float* __restrict__ post,
-                                                          float* __restrict__ comb, int64_t T,
-                                                          int64_t K, FinishParams fp) {
-  const int lane = threadIdx.x & 31;
-  const int r = lane & 3;
-  const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 2;
-  const bool live = t < T;
-  const int64_t tt = live ? t : 0;
-  pdl_wait();
-  pdl_trigger();
-  float4 g0 = make_float4(0.f, 0.f, 0.f, 0.f), g1 = g0, gc = g0;
-  float g6 = 0.f;
-#pragma unroll 2
-  for (int s = 0; s < nslot; ++s) {
-    const float4* rec = reinterpret_cast<const float4*>(part + (s * T + tt) * 32);
-    const float4 a0 = __ldg(rec), a1 = __ldg(rec + 1), ac = __ldg(rec + 2 + r);
-    const float a6 = __ldg(reinterpret_cast<const float*>(rec + 6));
-    g0.x += a0.x, g0.y += a0.y, g0.z += a0.z, g0.w += a0.w;
-    g1.x += a1.x, g1.y += a1.y, g1.z += a1.z, g1.w += a1.w;
-    gc.x += ac.x, gc.y += ac.y, gc.z += ac.z, gc.w += ac.w;
-    g6 += a6;
-  }
-  const float rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fdiv_rn(g6, static_cast<float>(K)) + fp.rms_eps));
-  const float g0r = r == 0 ? g0.x : r == 1 ? g0.y : r == 2 ? g0.z : g0.w;
-  const float g1r = r == 0 ? g1.x : r == 1 ? g1.y : r == 2 ? g1.z : g1.w;
-  const float lp = fmaf(g0r * rstd, __ldg(scale), __ldg(base + r));
-  const float lq = fmaf(g1r * rstd, __ldg(scale + 1), __ldg(base + 4 + r));
-  const float s2 = __ldg(scale + 2);
-  float cr[4] = {fmaf(gc.x * rstd, s2, __ldg(base + 8 + 4 * r)),
-                 fmaf(gc.y * rstd, s2, __ldg(base + 9 + 4 * r)),
-                 fmaf(gc.z * rstd, s2, __ldg(base + 10 + 4 * r)),
-                 fmaf(gc.w * rstd, s2, __ldg(base + 11 + 4 * r))};
-  if (live) pre[t * 4 + r] = sigmoidf_ieee(lp) + fp.pre_eps;
-  sinkhorn_quad(cr, fp.iters, fp.sinkhorn_eps);  // every lane takes part
-  if (live) {
-    post[t * 4 + r] = fp.post_mult * sigmoidf_ieee(lq);
-    *reinterpret_cast<float4*>(comb + t * 16 + r * 4) = make_float4(cr[0], cr[1], cr[2], cr[3]);
-  }
-}
-
 // y = bf16_rn(sum_i pre_i * R_i): one thread per (token, 8 columns), a streaming pass (R read once,
 // y written once). Requires H % 8 == 0 and 16-byte aligned R, y and pre.
 __global__ void __launch_bounds__(256) pre_agg_vec8_kernel(const uint16_t* __restrict__ R,
@@ -535,6 +487,109 @@ __global__ void __launch_bounds__(256) pre_agg_vec8_kernel(const uint16_t* __res
       o[e] = pack_bf16x2(a, b);
     }
     st_plain(y + t * H + v * 8, make_uint4(o[0], o[1], o[2], o[3]));
+  }
+}
+
+// Coefficients and aggregate in one kernel, kCaTok tokens per CTA (the split chain's last step).
+// Warp 0 forms the tokens' logits from the slot records (one lane quad per token) and their pre
+// gates; after a block barrier all 256 threads write y for those tokens with 16-byte accesses (eight
+// CTAs per SM keep the loads in flight); then warp 0 runs the tokens' Sinkhorn and writes post and comb, while
+// the SM's other CTAs keep the stream going. One kernel fewer in the chain than coef + aggregate.
+// Requires H % 8 == 0 and 16-byte aligned R and y.
+constexpr int kCaTok = 4;  // measured: 4 beats 2, 8 and 16 at T = 3072 and 8192
+static_assert(kCaTok <= 8, "warp 0 holds one lane quad per token");
+
+__global__ void __launch_bounds__(256, 8) pre_tc_coef_agg_kernel(
+    const uint16_t* __restrict__ R, const float* __restrict__ part, int nslot,
+    const float* __restrict__ scale, const float* __restrict__ base, uint16_t* __restrict__ y,
+    float* __restrict__ pre, float* __restrict__ post, float* __restrict__ comb, int64_t T,
+    int64_t H8, int64_t K, FinishParams fp) {
+  __shared__ float4 spre[kCaTok];
+  __shared__ float slog[32][5];  // comb row logits and post logit of each lane of warp 0
+  pdl_wait();
+  pdl_trigger();
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kCaTok;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int r = lane & 3;
+    const int qd = lane >> 2;  // token of this quad within the CTA (quads kCaTok.. are idle)
+    const int64_t t = t0 + qd;
+    const bool live = qd < kCaTok && t < T;
+    const int64_t tt = live ? t : 0;
+    float4 g0 = make_float4(0.f, 0.f, 0.f, 0.f), g1 = g0, gc = g0;
+    float g6 = 0.f;
+    for (int s = 0; s < nslot; ++s) {
+      const float4* rec = reinterpret_cast<const float4*>(part + (s * T + tt) * 32);
+      const float4 a0 = __ldg(rec), a1 = __ldg(rec + 1), ac = __ldg(rec + 2 + r);
+      const float a6 = __ldg(reinterpret_cast<const float*>(rec + 6));
+      g0.x += a0.x, g0.y += a0.y, g0.z += a0.z, g0.w += a0.w;
+      g1.x += a1.x, g1.y += a1.y, g1.z += a1.z, g1.w += a1.w;
+      gc.x += ac.x, gc.y += ac.y, gc.z += ac.z, gc.w += ac.w;
+      g6 += a6;
+    }
+    const float rstd =
+        __fdiv_rn(1.0f, __fsqrt_rn(__fdiv_rn(g6, static_cast<float>(K)) + fp.rms_eps));
+    const float g0r = r == 0 ? g0.x : r == 1 ? g0.y : r == 2 ? g0.z : g0.w;
+    const float g1r = r == 0 ? g1.x : r == 1 ? g1.y : r == 2 ? g1.z : g1.w;
+    const float lp = fmaf(g0r * rstd, __ldg(scale), __ldg(base + r));
+    slog[lane][4] = fmaf(g1r * rstd, __ldg(scale + 1), __ldg(base + 4 + r));
+    const float s2 = __ldg(scale + 2);
+    slog[lane][0] = fmaf(gc.x * rstd, s2, __ldg(base + 8 + 4 * r));
+    slog[lane][1] = fmaf(gc.y * rstd, s2, __ldg(base + 9 + 4 * r));
+    slog[lane][2] = fmaf(gc.z * rstd, s2, __ldg(base + 10 + 4 * r));
+    slog[lane][3] = fmaf(gc.w * rstd, s2, __ldg(base + 11 + 4 * r));
+    const float pv = sigmoidf_ieee(lp) + fp.pre_eps;
+    if (live) pre[t * 4 + r] = pv;
+    if (qd < kCaTok) reinterpret_cast<float*>(spre)[qd * 4 + r] = pv;
+  }
+  __syncthreads();
+  const int64_t ntok = min(static_cast<int64_t>(kCaTok), T - t0);
+  const int64_t units = ntok * H8;
+  const int64_t H = H8 * 8;
+  for (int64_t u = threadIdx.x; u < units; u += 256) {
+    const int64_t k = u / H8;
+    const int64_t v = u - k * H8;
+    const uint16_t* rr = R + (t0 + k) * 4 * H + v * 8;
+    uint4 rv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) rv[i] = ld_stream_ro(rr + i * H);
+    const float4 p4 = spre[k];
+    const uint32_t* r0 = &rv[0].x;
+    const uint32_t* r1 = &rv[1].x;
+    const uint32_t* r2 = &rv[2].x;
+    const uint32_t* r3 = &rv[3].x;
+    uint32_t o[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float a = p4.x * bf16_lo(r0[c]);
+      a = fmaf(p4.y, bf16_lo(r1[c]), a);
+      a = fmaf(p4.z, bf16_lo(r2[c]), a);
+      a = fmaf(p4.w, bf16_lo(r3[c]), a);
+      float b = p4.x * bf16_hi(r0[c]);
+      b = fmaf(p4.y, bf16_hi(r1[c]), b);
+      b = fmaf(p4.z, bf16_hi(r2[c]), b);
+      b = fmaf(p4.w, bf16_hi(r3[c]), b);
+      o[c] = pack_bf16x2(a, b);
+    }
+    st_plain(y + (t0 + k) * H + v * 8, make_uint4(o[0], o[1], o[2], o[3]));
+  }
+  if (threadIdx.x < 32) {  // warp 0 wrote slog before the barrier above
+    const int lane = threadIdx.x;
+    const int r = lane & 3;
+    const int qd = lane >> 2;
+    const int64_t t = t0 + qd;
+    const bool live = qd < kCaTok && t < T;
+    float cr[4] = {0.f, 0.f, 0.f, 0.f};
+    if (qd < kCaTok) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) cr[c] = slog[lane][c];
+    }
+    sinkhorn_quad(cr, fp.iters, fp.sinkhorn_eps);  // every lane of warp 0 takes part
+    if (live) {
+      post[t * 4 + r] = fp.post_mult * sigmoidf_ieee(slog[lane][4]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) comb[t * 16 + 4 * r + c] = cr[c];
+    }
   }
 }
 
@@ -613,21 +668,13 @@ int launch_pre_tc(const PreArgs& a, cudaStream_t s) {
   if (r != 0) return r;
 
   const FinishParams fp{a.iters, a.sinkhorn_eps, a.rms_eps, a.pre_eps, a.post_mult};
-  const bool vec = aligned16(a.R) && aligned16(a.y) && aligned16(a.comb) && (a.H % 8 == 0);
-  if (vec && aligned16(a.pre)) {
-    const int64_t cb = (4 * a.T + 255) / 256;
+  const bool vec = aligned16(a.R) && aligned16(a.y) && (a.H % 8 == 0);
+  if (vec) {
+    const int64_t cb = (a.T + kCaTok - 1) / kCaTok;
     if (cb > 0x7fffffff) return -5;
-    if (launch_pdl(pre_tc_coef_kernel, dim3(static_cast<unsigned>(cb)), dim3(256), 0, s,
-                   static_cast<const float*>(part), nrec, a.hc_scale,
-                   a.hc_base, a.pre, a.post, a.comb, a.T, 4 * a.H, fp) != cudaSuccess)
-      return -4;
-    note_launches(1);
-    const int64_t units = a.T * (a.H / 8);
-    int64_t ab = (units + 255) / 256;
-    const int64_t cap = static_cast<int64_t>(device_sm_count()) * 16;
-    if (ab > cap) ab = cap;
-    if (launch_pdl(pre_agg_vec8_kernel, dim3(static_cast<unsigned>(ab)), dim3(256), 0, s, a.R,
-                   static_cast<const float*>(a.pre), a.y, a.T, a.H / 8) != cudaSuccess)
+    if (launch_pdl(pre_tc_coef_agg_kernel, dim3(static_cast<unsigned>(cb)), dim3(256), 0, s, a.R,
+                   static_cast<const float*>(part), nrec, a.hc_scale, a.hc_base, a.y, a.pre,
+                   a.post, a.comb, a.T, a.H / 8, 4 * a.H, fp) != cudaSuccess)
       return -4;
   } else {
     const int64_t nhb = (a.H + kAggCols - 1) / kAggCols;

@@ -20,9 +20,14 @@ CASES = {
     "pre_decode_T32": ("mhc_pre T=32 H=7168", "pre_cc_partial_staged_kernel, pre_cc_finish_kernel"),
     "pre_small": ("mhc_pre T=64 H=512", "pre_cc_partial_kernel, pre_cc_finish_kernel"),
     "pre_split_T3072": ("mhc_pre T=3072 H=7168, split tensor path",
-                        "pre_tc_split_kernel, pre_tc_proj_kernel, pre_tc_coef_kernel, "
-                        "pre_agg_vec8_kernel"),
+                        "pre_tc_split_kernel, pre_tc_proj_kernel, pre_tc_coef_agg_kernel"),
     "pre_fused_T3072": ("mhc_pre T=3072 H=7168, single-pass path",
+                        "pre_fused_zero_kernel, pre_fused_kernel"),
+    "pre_large": ("mhc_pre T=8192 H=7168 (default path: the split chain)",
+                  "pre_tc_split_kernel, pre_tc_proj_kernel, pre_tc_coef_agg_kernel"),
+    "pre_fused_large": ("mhc_pre T=8192 H=7168, single-pass path",
+                        "pre_fused_zero_kernel, pre_fused_kernel"),
+    "pre_fused_T1024": ("mhc_pre T=1024 H=7168 (default path: the single pass)",
                         "pre_fused_zero_kernel, pre_fused_kernel"),
     "post_large": ("mhc_post T=8192 H=7168", "post_persistent_kernel"),
     "post_scalar_H1001": ("mhc_post T=8192 H=1001", "post_scalar_kernel"),
@@ -76,6 +81,12 @@ def make_call(case):
         return pre_call(3072, 7168, PRE_PATH_TENSOR_SPLIT)
     if case == "pre_fused_T3072":
         return pre_call(3072, 7168, PRE_PATH_TENSOR_FUSED)
+    if case == "pre_large":
+        return pre_call(8192, 7168)
+    if case == "pre_fused_large":
+        return pre_call(8192, 7168, PRE_PATH_TENSOR_FUSED)
+    if case == "pre_fused_T1024":
+        return pre_call(1024, 7168)
     if case in ("post_large", "post_scalar_H1001"):
         T, H = (8192, 7168) if case == "post_large" else (8192, 1001)
         g, R, x, _, _, _ = _inputs(T, H)
