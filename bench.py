@@ -489,6 +489,11 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     launches0 = mhc.launch_count()
+    # A spin kernel ahead of the start event lets the host queue the steps before the device
+    # reaches them: the first step then does not include the host's enqueue latency after the
+    # synchronize (the device work timed is the same).
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(4000000)
     start.record(stream)
     for i in range(args.steps):
         ev[i][0].record(stream)
