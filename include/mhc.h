@@ -177,6 +177,14 @@ enum mhc_path {
                                       reset; H % 8 == 0, H >= 64, R, y and the workspace 16-byte
                                       aligned; MHC_ERR_UNSUPPORTED, with nothing launched, when
                                       the device cannot hold its grid resident */
+    MHC_PRE_PATH_TENSOR_WAVE = 5,  /* one pass over R in wavefront order: every CTA projects a short
+                                      K range of the same few token tiles (persistent cooperative
+                                      kernel, hc_fn tiles streamed from L2), per-tile counters
+                                      release the aggregate units, which re-read the rows from L2;
+                                      then the Sinkhorn pass. H % 8 == 0, H >= 64, R, y, comb and
+                                      the workspace 16-byte aligned; MHC_ERR_UNSUPPORTED, with
+                                      nothing launched, when the device cannot hold its grid
+                                      resident */
     /* post */
     MHC_POST_PATH_VEC8 = 11,       /* 16-byte vector loads/stores; H % 8 == 0, 16-byte aligned */
     MHC_POST_PATH_PERSISTENT = 12, /* persistent, bulk-copy (TMA) staged; same requirements */

@@ -33,6 +33,7 @@ PRE_PATH_CUDA_CORE = 1
 PRE_PATH_TENSOR = 2
 PRE_PATH_TENSOR_SPLIT = 3
 PRE_PATH_TENSOR_FUSED = 4
+PRE_PATH_TENSOR_WAVE = 5
 POST_PATH_VEC8 = 11
 POST_PATH_PERSISTENT = 12
 POST_PATH_SCALAR = 13

@@ -7,6 +7,7 @@
 #include "mhc_pre_cc.cu"
 #include "mhc_pre_tc.cu"
 #include "mhc_pre_fused.cu"
+#include "mhc_pre_wave.cu"
 #include "mhc_pre_noalloc.cu"
 #include "mhc_pre_bigfuse.cu"
 #include "mhc_boundary.cu"

@@ -161,8 +161,10 @@ size_t mhc_pre_workspace_bytes(int64_t T, int64_t H) {
   if (T <= 0 || H <= 0) return 0;
   size_t m = pre_cc_workspace_bytes(T, H);
   const size_t b = pre_tc_workspace_bytes(T, H), c = pre_fused_workspace_bytes(T, H);
+  const size_t d = pre_wave_workspace_bytes(T, H);
   if (b > m) m = b;
   if (c > m) m = c;
+  if (d > m) m = d;
   return (m + 255) / 256 * 256;
 }
 
@@ -229,7 +231,8 @@ int mhc_pre_with_path(const uint16_t* R, const float* hc_fn, const float* hc_sca
       !isfinite(prm.pre_eps) || !isfinite(prm.post_mult))
     return MHC_ERR_INVALID_ARG;
   if (path != MHC_PATH_AUTO && path != MHC_PRE_PATH_CUDA_CORE && path != MHC_PRE_PATH_TENSOR &&
-      path != MHC_PRE_PATH_TENSOR_SPLIT && path != MHC_PRE_PATH_TENSOR_FUSED)
+      path != MHC_PRE_PATH_TENSOR_SPLIT && path != MHC_PRE_PATH_TENSOR_FUSED &&
+      path != MHC_PRE_PATH_TENSOR_WAVE)
     return MHC_ERR_INVALID_ARG;
   if (T == 0) return MHC_OK;
   if (!R || !hc_fn || !hc_scale || !hc_base || !y || !pre || !post || !comb)
@@ -256,6 +259,9 @@ int mhc_pre_with_path(const uint16_t* R, const float* hc_fn, const float* hc_sca
   // The fused kernel also uses 16-byte accesses on y, pre and comb.
   const bool fused_ok = tc_ok && pre_fused_supported(T, H) && aligned16(y) && aligned16(pre) &&
                         aligned16(comb);
+  // The wavefront single pass: 16-byte accesses on y and comb as well.
+  const bool wave_ok =
+      tc_ok && pre_wave_supported(T, H) && aligned16(y) && aligned16(comb);
   bool auto_fused = false;
   if (path == MHC_PATH_AUTO) {
     path = (tc_ok && T >= kPreTensorMinTokens) ? MHC_PRE_PATH_TENSOR : MHC_PRE_PATH_CUDA_CORE;
@@ -264,12 +270,19 @@ int mhc_pre_with_path(const uint16_t* R, const float* hc_fn, const float* hc_sca
     return MHC_ERR_UNSUPPORTED;
   } else if (path == MHC_PRE_PATH_TENSOR_FUSED && !fused_ok) {
     return MHC_ERR_UNSUPPORTED;
+  } else if (path == MHC_PRE_PATH_TENSOR_WAVE && !wave_ok) {
+    return MHC_ERR_UNSUPPORTED;
   }
   int st = bind_device(R);
   if (st != MHC_OK) return st;
   PreArgs a{R, hc_fn, hc_scale, hc_base, y, pre, post, comb, workspace, workspace_bytes, T, H,
             prm.sinkhorn_iters, prm.sinkhorn_eps, prm.rms_eps, prm.pre_eps, prm.post_mult};
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (path == MHC_PRE_PATH_TENSOR_WAVE) {
+    // 1: the grid cannot run with every CTA resident on this device; nothing was launched.
+    const int r = launch_pre_wave(a, s);
+    return r == 1 ? MHC_ERR_UNSUPPORTED : r;
+  }
   if (path == MHC_PRE_PATH_TENSOR_FUSED || auto_fused) {
     // 1: the grid cannot run with every CTA resident on this device; nothing was launched. A
     // forced single pass reports it; the automatic choice falls back to the split chain.

@@ -173,6 +173,22 @@ __device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
   return r != 0;
 }
 
+// ------------------------------------------------------------------------------ cross-CTA counters
+
+// Acquire load at gpu scope: later reads of this thread see what the releasing writers published.
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Everything this thread has observed (including, through a CTA-scope barrier before it, other
+// threads' stores) is visible at gpu scope before the add.
+__device__ __forceinline__ void red_release_add_gpu(int* p, int v) {
+  asm volatile("fence.acq_rel.gpu;\n\tred.relaxed.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v)
+               : "memory");
+}
+
 // ------------------------------------------------------------------------------ coefficient math
 
 __device__ __forceinline__ float sigmoidf_ieee(float v) { return 1.0f / (1.0f + expf(-v)); }

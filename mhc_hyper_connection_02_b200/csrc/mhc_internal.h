@@ -89,6 +89,12 @@ bool pre_fused_preferred(int64_t T, int64_t H);
 size_t pre_fused_workspace_bytes(int64_t T, int64_t H);
 int launch_pre_fused(const PreArgs& a, cudaStream_t s);
 
+// Tensor-core path: single pass in wavefront order (mhc_pre_wave.cu; launch returns 1, having
+// launched nothing, when the device cannot run its grid with every CTA resident).
+bool pre_wave_supported(int64_t T, int64_t H);
+size_t pre_wave_workspace_bytes(int64_t T, int64_t H);
+int launch_pre_wave(const PreArgs& a, cudaStream_t s);
+
 // Pre-map from an external projection (mhc_pre_big_fuse; sqrsum == nullptr selects the variant
 // that forms the sum of squares from R, k = 4H).
 struct BigFuseArgs {

@@ -200,26 +200,13 @@ __device__ __forceinline__ void fs_tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) 
       : "memory");
 }
 
-__device__ __forceinline__ int fs_ld_acquire(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// Everything this thread has observed (including, through the CTA-scope barrier before it, the
-// other epilogue threads' record stores) is visible at gpu scope before the add.
-__device__ __forceinline__ void fs_red_release_add(int* p, int v) {
-  asm volatile("fence.acq_rel.gpu;\n\tred.relaxed.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v)
-               : "memory");
-}
-
 // Waits until *p >= target (acquire); false on timeout or once another wait has timed out.
 __device__ __noinline__ bool fs_wait_count(const int* p, int target, int where) {
-  if (fs_ld_acquire(p) >= target) return true;
+  if (ld_acquire_gpu(p) >= target) return true;
   const unsigned long long t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     __nanosleep(32);
-    if (fs_ld_acquire(p) >= target) return true;
+    if (ld_acquire_gpu(p) >= target) return true;
     if ((i & 63u) == 0) {
       if (*reinterpret_cast<volatile int*>(&g_device_status) != 0) return false;
       if (global_timer_ns() - t0 > kWaitLimitNs) {
@@ -476,7 +463,7 @@ __global__ void __launch_bounds__(kFsThreads, 1)
       // The four warps agree on going on, and their records are published with one
       // release-increment of the tile's counter.
       if (named_bar_or(1, 128, !ok)) return true;
-      if (warp == 2 && lane == 0) fs_red_release_add(a.cnt + X, 1);
+      if (warp == 2 && lane == 0) red_release_add_gpu(a.cnt + X, 1);
       return false;
     };
     int64_t it = 0;

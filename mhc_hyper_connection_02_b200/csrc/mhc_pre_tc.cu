@@ -166,27 +166,31 @@ __device__ __forceinline__ void tmem_wait_ld() {
 // hc_fn [K][24] fp32 -> Bw [80][K] bf16: rows j, 24+j, 48+j hold the hi, mid, lo terms of column
 // j (w = hi + mid + lo exactly: each remainder is exact in fp32 and the last fits 8 bits); rows
 // 72..79 are zero.
+__device__ __forceinline__ void split_hc_fn_row(const float* __restrict__ W,
+                                                uint16_t* __restrict__ Bw, int64_t K, int64_t k) {
+#pragma unroll 4
+  for (int j = 0; j < kMix; ++j) {
+    const float w = W[k * kMix + j];
+    const uint16_t hi = f32_to_bf16(w);
+    const float r1 = w - bf16_to_f32(hi);
+    const uint16_t mid = f32_to_bf16(r1);
+    const float r2 = r1 - bf16_to_f32(mid);
+    const uint16_t lo = f32_to_bf16(r2);
+    Bw[j * K + k] = hi;
+    Bw[(kMix + j) * K + k] = mid;
+    Bw[(2 * kMix + j) * K + k] = lo;
+  }
+#pragma unroll
+  for (int j = 3 * kMix; j < kTcN; ++j) Bw[j * K + k] = 0;
+}
+
 __global__ void __launch_bounds__(256) pre_tc_split_kernel(const float* __restrict__ W,
                                                            uint16_t* __restrict__ Bw, int64_t K) {
   pdl_wait();  // the previous call's projection may still read Bw
   pdl_trigger();
   for (int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; k < K;
-       k += (int64_t)gridDim.x * blockDim.x) {
-#pragma unroll 4
-    for (int j = 0; j < kMix; ++j) {
-      const float w = W[k * kMix + j];
-      const uint16_t hi = f32_to_bf16(w);
-      const float r1 = w - bf16_to_f32(hi);
-      const uint16_t mid = f32_to_bf16(r1);
-      const float r2 = r1 - bf16_to_f32(mid);
-      const uint16_t lo = f32_to_bf16(r2);
-      Bw[j * K + k] = hi;
-      Bw[(kMix + j) * K + k] = mid;
-      Bw[(2 * kMix + j) * K + k] = lo;
-    }
-#pragma unroll
-    for (int j = 3 * kMix; j < kTcN; ++j) Bw[j * K + k] = 0;
-  }
+       k += (int64_t)gridDim.x * blockDim.x)
+    split_hc_fn_row(W, Bw, K, k);
 }
 
 __global__ void __launch_bounds__(kTcThreads, 1) pre_tc_proj_kernel(
@@ -571,7 +575,7 @@ __global__ void __launch_bounds__(256, 8) pre_tc_coef_agg_kernel(
       b = fmaf(p4.w, bf16_hi(r3[c]), b);
       o[c] = pack_bf16x2(a, b);
     }
-    st_plain(y + (t0 + k) * H + v * 8, make_uint4(o[0], o[1], o[2], o[3]));
+    st_stream(y + (t0 + k) * H + v * 8, make_uint4(o[0], o[1], o[2], o[3]));  // not re-read here
   }
   if (threadIdx.x < 32) {  // warp 0 wrote slog before the barrier above
     const int lane = threadIdx.x;

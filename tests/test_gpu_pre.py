@@ -20,7 +20,8 @@ from tolerance import COEF_TOL, U32, bf16_bits_to_f64, check_bf16, check_coef
 pytestmark = pytest.mark.gpu
 
 PRE_PATHS = {"cuda_core": mhc.PRE_PATH_CUDA_CORE, "tensor": mhc.PRE_PATH_TENSOR,
-             "tensor_split": mhc.PRE_PATH_TENSOR_SPLIT, "tensor_fused": mhc.PRE_PATH_TENSOR_FUSED}
+             "tensor_split": mhc.PRE_PATH_TENSOR_SPLIT, "tensor_fused": mhc.PRE_PATH_TENSOR_FUSED,
+             "tensor_wave": mhc.PRE_PATH_TENSOR_WAVE}
 
 
 def run_pre(w, path=mhc.PATH_AUTO, params=None, R_dev=None):
@@ -49,6 +50,21 @@ def run_fused(w, R_dev=None):
     return outs
 
 
+def run_wave(w, R_dev=None):
+    """The wavefront single pass, forced. None where the library reports it cannot run this shape
+    (MHC_ERR_UNSUPPORTED, nothing launched); otherwise asserts its three launches (hc_fn split and
+    counter reset, the wave kernel, the Sinkhorn pass), so a pass is the wave kernel's."""
+    n0 = mhc.launch_count()
+    try:
+        outs = run_pre(w, mhc.PRE_PATH_TENSOR_WAVE, R_dev=R_dev)
+    except mhc.MhcError as e:
+        assert e.status == mhc.MHC_ERR_UNSUPPORTED
+        assert mhc.launch_count() == n0
+        return None
+    assert mhc.launch_count() - n0 == 3, "the wave path must be exactly its three launches"
+    return outs
+
+
 def compare_pre(w, outs, rows=None, label="", pre_eps=None, post_mult=None, iters=None, eps=None):
     y, pre, post, comb = outs
     R = w.R if rows is None else w.R[rows]
@@ -69,12 +85,16 @@ def compare_pre(w, outs, rows=None, label="", pre_eps=None, post_mult=None, iter
     return max(dp, dq, dc)
 
 
-@pytest.mark.parametrize("path", ["cuda_core", "tensor", "tensor_split", "tensor_fused"])
+@pytest.mark.parametrize("path", ["cuda_core", "tensor", "tensor_split", "tensor_fused",
+                                  "tensor_wave"])
 def test_pre_small_workload(path):
     w = inputs.small()
     if path == "tensor_fused":
         outs = run_fused(w)
         assert outs is not None, "the single-pass kernel supports T=64, H=512"
+    elif path == "tensor_wave":
+        outs = run_wave(w)
+        assert outs is not None, "the wave kernel supports T=64, H=512"
     else:
         outs = run_pre(w, PRE_PATHS[path])
     compare_pre(w, outs, label=f"small {path}")
@@ -94,6 +114,11 @@ def test_pre_shapes(T, H):
         compare_pre(w, fused, label=f"T={T} H={H} tensor-fused")
     else:
         assert H % 8 != 0 or H < 64, f"single-pass kernel refused T={T} H={H}"
+    wave = run_wave(w)
+    if wave is not None:
+        compare_pre(w, wave, label=f"T={T} H={H} tensor-wave")
+    else:
+        assert H % 8 != 0 or H < 64, f"wave kernel refused T={T} H={H}"
 
 
 @pytest.mark.parametrize("T,H", [(300, 7168), (129, 1000), (1, 4096), (520, 512)])
@@ -108,6 +133,9 @@ def test_pre_tensor_path_agrees_with_cuda_core_path(T, H):
     fused = run_fused(w)
     if fused is not None:
         others.append((fused, "tensor-fused"))
+    wave = run_wave(w)
+    if wave is not None:
+        others.append((wave, "tensor-wave"))
     for other, oname in others:
         for x, y, name in zip(a[1:], other[1:], ("pre", "post", "comb")):
             d = (x.double() - y.double()).abs().max().item()
@@ -142,12 +170,17 @@ def test_pre_large_full_batch():
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("path", ["tensor_fused", "tensor_split", "cuda_core"])
+@pytest.mark.parametrize("path", ["tensor_fused", "tensor_wave", "tensor_split", "cuda_core"])
 def test_pre_large_full_batch_each_path(path):
-    """T=8192, H=7168, every token, on each forced path (the single-pass kernel runs here with
-    every group's record ring wrapping many times)."""
+    """T=8192, H=7168, every token, on each forced path (the single-pass kernels run here with
+    their record rings wrapping many times)."""
     w = inputs.large()
-    outs = run_fused(w) if path == "tensor_fused" else run_pre(w, PRE_PATHS[path])
+    if path == "tensor_fused":
+        outs = run_fused(w)
+    elif path == "tensor_wave":
+        outs = run_wave(w)
+    else:
+        outs = run_pre(w, PRE_PATHS[path])
     assert outs is not None
     compare_pre_all(w, outs, label=f"large {path}")
 
@@ -162,12 +195,33 @@ def test_pre_fused_multi_tile(T, H):
     compare_pre(w, outs, label=f"fused T={T} H={H}")
 
 
+@pytest.mark.parametrize("T,H", [(3000, 1000), (1000, 7168), (2000, 4096), (129, 64), (3072, 7168),
+                                 (700, 16392), (1, 7168)])
+def test_pre_wave_multi_tile(T, H):
+    """The wavefront kernel: ranges that cross tile boundaries, ragged last tiles, K not a multiple
+    of 64 columns (H = 1000), more than 64 pieces of a tile in flight over the record ring (T=3072)
+    and y units narrower than a row (H = 16392: seventeen per token)."""
+    w = inputs.custom(T, H, seed=T + 11 * H)
+    outs = run_wave(w)
+    assert outs is not None
+    compare_pre(w, outs, label=f"wave T={T} H={H}")
+
+
+def test_pre_wave_refuses_what_it_cannot_run():
+    """H % 8 != 0 or H < 64: MHC_ERR_UNSUPPORTED with nothing launched."""
+    for T, H in ((10, 1001), (10, 56)):
+        w = inputs.custom(T, H, seed=5)
+        assert run_wave(w) is None
+
+
 def test_pre_params_other_than_default():
     w = inputs.custom(50, 256, seed=77)
     p = mhc.make_params(iters=50, eps=1e-3, rms_eps=1e-4, pre_eps=1e-6, post_mult=1.0)
     w.rms_eps = 1e-4
     outs = run_pre(w, params=p)
     compare_pre(w, outs, label="params", pre_eps=1e-6, post_mult=1.0, iters=50, eps=1e-3)
+    outs = run_pre(w, mhc.PRE_PATH_TENSOR_WAVE, params=p)
+    compare_pre(w, outs, label="params wave", pre_eps=1e-6, post_mult=1.0, iters=50, eps=1e-3)
 
 
 @pytest.mark.parametrize("stream", range(4))
