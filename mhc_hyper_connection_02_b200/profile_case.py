@@ -29,6 +29,10 @@ CASES = {
                         "pre_fused_zero_kernel, pre_fused_kernel"),
     "pre_fused_T1024": ("mhc_pre T=1024 H=7168 (default path: the single pass)",
                         "pre_fused_zero_kernel, pre_fused_kernel"),
+    "pre_wave_T3072": ("mhc_pre T=3072 H=7168, wavefront single pass",
+                       "pre_wave_prep_kernel, pre_wave_kernel, sinkhorn_kernel"),
+    "pre_wave_large": ("mhc_pre T=8192 H=7168, wavefront single pass",
+                       "pre_wave_prep_kernel, pre_wave_kernel, sinkhorn_kernel"),
     "post_large": ("mhc_post T=8192 H=7168", "post_persistent_kernel"),
     "post_scalar_H1001": ("mhc_post T=8192 H=1001", "post_scalar_kernel"),
     "sinkhorn_T1M": ("mhc_sinkhorn T=1048576", "sinkhorn_kernel"),
@@ -62,7 +66,8 @@ def _coefficients(g, T):
 
 def make_call(case):
     import torch
-    from . import (PRE_PATH_TENSOR_FUSED, PRE_PATH_TENSOR_SPLIT, POST_PATH_SCALAR, expand,
+    from . import (PRE_PATH_TENSOR_FUSED, PRE_PATH_TENSOR_SPLIT, PRE_PATH_TENSOR_WAVE,
+                   POST_PATH_SCALAR, expand,
                    head_mean, post, pre, pre_backward, pre_big_fuse, sinkhorn, workspace_bytes)
 
     def pre_call(T, H, path=0):
@@ -85,6 +90,10 @@ def make_call(case):
         return pre_call(8192, 7168)
     if case == "pre_fused_large":
         return pre_call(8192, 7168, PRE_PATH_TENSOR_FUSED)
+    if case == "pre_wave_T3072":
+        return pre_call(3072, 7168, PRE_PATH_TENSOR_WAVE)
+    if case == "pre_wave_large":
+        return pre_call(8192, 7168, PRE_PATH_TENSOR_WAVE)
     if case == "pre_fused_T1024":
         return pre_call(1024, 7168)
     if case in ("post_large", "post_scalar_H1001"):
