@@ -13,3 +13,4 @@
 #include "mhc_boundary.cu"
 #include "mhc_post_project.cu"
 #include "mhc_backward.cu"
+#include "mhc_backward_tc.cu"

@@ -13,8 +13,9 @@
 //   3. per token (lane quad): rstd, logits, gates, the Sinkhorn forward (states checkpointed)
 //      and the reverse pass -> d_raw, d_ss, the gates, and the per-token terms of d_scale, d_base;
 //   4. d_scale, d_base: fixed-order sums over tokens;
-//   5. d_R = d_raw . hc_fn^T + 2 R d_ss + pre_i d_y (column slice x token chunk per CTA, a
-//      thread's hc_fn weights in registers, fp32 on CUDA cores);
+//   5. d_R = d_raw . hc_fn^T + 2 R d_ss + pre_i d_y: on tcgen05 tensor cores where H % 128 == 0
+//      and d_y is given (mhc_backward_tc.cu), else column slice x token chunk per CTA, a thread's
+//      hc_fn weights in registers, fp32 on CUDA cores;
 //   6. d_hc_fn = R_flat^T d_raw (column slice x token chunk per CTA, tokens summed in order, then
 //      the chunks in order).
 #include "mhc_device.cuh"
@@ -666,7 +667,7 @@ __global__ void __launch_bounds__(256) pre_bwd_dw_sum_kernel(const float* __rest
 }
 
 struct BwPlan {
-  size_t proj, dpt, brec, dwp, total;
+  size_t proj, dpt, brec, dwp, drtc, total;
   int64_t tchunk;
   int nchunk;
 };
@@ -688,7 +689,8 @@ static BwPlan bw_plan(int64_t T, int64_t H) {
   p.tchunk = ((T + nchunk - 1) / nchunk + kDwTok - 1) / kDwTok * kDwTok;
   p.nchunk = static_cast<int>((T + p.tchunk - 1) / p.tchunk);
   p.dwp = up(static_cast<size_t>(p.nchunk) * 4 * H * kMix * 4);
-  p.total = p.proj + p.dpt + p.brec + p.dwp;
+  p.drtc = up(pre_bwd_dr_tc_workspace_bytes(T, H));  // split operands of the tensor-core d_R
+  p.total = p.proj + p.dpt + p.brec + p.dwp + p.drtc;
   return p;
 }
 
@@ -703,6 +705,7 @@ int launch_pre_backward(const PreBwdArgs& a, cudaStream_t s) {
   float* dpt = reinterpret_cast<float*>(ws + plan.proj);
   float* brec = reinterpret_cast<float*>(ws + plan.proj + plan.dpt);
   float* dwp = reinterpret_cast<float*>(ws + plan.proj + plan.dpt + plan.brec);
+  void* drtc_ws = ws + plan.proj + plan.dpt + plan.brec + plan.dwp;
   const int64_t K = 4 * a.H;
   if (a.T > 0x7fffffff) return -5;
 
@@ -738,8 +741,17 @@ int launch_pre_backward(const PreBwdArgs& a, cudaStream_t s) {
   e = launch_pdl(pre_bwd_param_kernel, dim3(3 + kMix), dim3(256), 0, s,
                  static_cast<const float*>(brec), a.dscale, a.dbase, a.T);
   if (e != cudaSuccess) return -4;
-  // 5. d_R: column slices x token chunks, one wave of kDxSlotsPerSm CTAs per SM.
-  if (vec) {
+  // 5. d_R: on tensor cores where the shape allows (1: not this shape, nothing launched), else
+  // column slices x token chunks on CUDA cores, one wave of kDxSlotsPerSm CTAs per SM.
+  int dr = 1;
+  if (vec && a.dy != nullptr) {
+    dr = launch_pre_bwd_dr_tc(a.R, a.dy, a.hc_fn, static_cast<const float*>(brec), kBrec, a.dR,
+                              drtc_ws, a.T, a.H, s);
+    if (dr < 0) return dr;
+  }
+  if (dr == 0) {
+    e = cudaSuccess;
+  } else if (vec) {
     if (!ensure_smem_limit(reinterpret_cast<const void*>(pre_bwd_dx_kernel), kDxSmem)) return -4;
     const int64_t xcols = (K + kDxCols - 1) / kDxCols;
     int64_t xch = (kDxSlotsPerSm * static_cast<int64_t>(device_sm_count())) / xcols;
@@ -771,7 +783,8 @@ int launch_pre_backward(const PreBwdArgs& a, cudaStream_t s) {
   e = launch_pdl(pre_bwd_dw_sum_kernel, dim3(static_cast<unsigned>(nb)), dim3(256), 0, s,
                  static_cast<const float*>(dwp), a.dW, K * kMix, plan.nchunk);
   if (e != cudaSuccess) return -4;
-  note_launches(7);
+  // dpre, coef, param, d_R on CUDA cores (the tensor-core form counts its own two), dw, dw_sum.
+  note_launches(dr == 0 ? 5 : 6);
   return 0;
 }
 

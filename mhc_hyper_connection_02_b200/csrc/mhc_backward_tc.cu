@@ -1,0 +1,531 @@
+// Pre-map backward, d_R on tcgen05 tensor cores.
+//
+// d_R[t][k] = sum_j d_raw[t][j] hc_fn[k][j] + 2 R[t][k] d_ss[t] + pre_i[t] d_y[t][h], k = i*H + h
+// (the chain rule through raw = R_flat . hc_fn, the sum of squares and y = sum_i pre_i R_i;
+// "FlashInfer mHC module deep dive" §3.4 / §5.2 forward). The contraction has inner dimension 24:
+// on CUDA cores that is 24 FMAs per element of d_R and the kernel is bound by issue; on tensor
+// cores it is bound by its traffic (R and d_y read, d_R written).
+//
+// Operands (written by pre_bwd_split_kernel, bf16, 128 columns per row, zero past 72; the MMAs
+// read columns 0..79: four K=16 steps in a 128-byte-swizzled box, one in a 32-byte-swizzled box):
+//   A[t] = [hi(d_raw) | hi(d_raw) | lo(d_raw)],  B[k] = [hi(w) | lo(w) | hi(w)],  w = hc_fn[k][.]
+// so A.B = hi.hi + hi.lo + lo.hi of each product, exact in the fp32 accumulator; the dropped
+// lo.lo term and the split's remainders are below 2^-15 of each product.
+//
+// pre_bwd_dr_kernel: persistent, one CTA per SM. Work items (token tile tt of 128, column block
+// hc of 128 columns within a stream, stream i), numbered with i fastest, so the four items of a
+// (tt, hc) group share one d_y tile; the list is cut into equal contiguous ranges, one per CTA.
+//   warp 0      TMA: A of the token tile (32 KB, reloaded when the tile changes), the group's d_y
+//               tile (two buffers), and per item the R tile and the B tile (rings of two: an R
+//               slot is free once its d_R has been stored, a B slot once its MMAs have read it);
+//               all [128 x 64] boxes with the 128-byte swizzle.
+//   warp 1      tcgen05.mma M=128 N=128 K=16, five steps (K columns 0..79), into one of two TMEM
+//               accumulators.
+//   warps 2-5   epilogue, thread = token row (its TMEM lane): 64 accumulator columns at a time
+//               (tcgen05.ld), R and d_y from the staged tiles, out = bf16_rn(fma(pre_i, d_y,
+//               fma(2 d_ss, R, acc))) written over R in place.
+//   warp 6      stores each finished d_R tile with a TMA bulk-tensor store and releases its R slot
+//               once the store has read it (the epilogue warps go on to the next item meanwhile).
+// Every wait is bounded; copies in flight are drained and stores completed before exit.
+// Requires H % 128 == 0, d_y present, 16-byte aligned R, d_y, d_R and workspace.
+// The TMA, descriptor, MMA and TMEM helpers and the tensor-map encoder are mhc_pre_tc.cu's (same
+// translation unit).
+#include <cuda.h>
+
+#include "mhc_device.cuh"
+#include "mhc_internal.h"
+
+namespace mhc {
+
+constexpr int kDrM = 128;                      // tokens per tile
+constexpr int kDrN = 128;                      // columns of d_R per item
+constexpr int kDrKd = 128;                     // split inner dimension (72 used), two swizzle atoms
+constexpr int kDrAtom = 128 * 64 * 2;          // one [128 x 64] bf16 box: 16 KB
+constexpr int kDrTile = 2 * kDrAtom;           // [128 x 128] bf16: 32 KB
+// A and B operand tiles: split columns 0..63 as one [128 x 64] box with the 128-byte swizzle and
+// columns 64..79 as a [128 x 16] box with the 32-byte swizzle (columns 80..127 are never loaded).
+constexpr int kDrAtomNarrow = 128 * 16 * 2;    // 4 KB
+constexpr int kDrOpTile = kDrAtom + kDrAtomNarrow;  // 20 KB
+constexpr int kDrRSlots = 3;                   // R ring (the HBM stream); d_R is staged in place
+constexpr int kDrBSlots = 2;                   // B ring (L2; freed as soon as the MMAs read it)
+constexpr int kDrOffA = 0;
+constexpr int kDrOffDy = kDrOffA + kDrOpTile;          // two buffers
+constexpr int kDrOffB = kDrOffDy + 2 * kDrTile;
+constexpr int kDrOffR = kDrOffB + kDrBSlots * kDrOpTile;
+constexpr int kDrOffBars = kDrOffR + kDrRSlots * kDrTile;  // 225280
+constexpr int kDrSmem = 1024 + kDrOffBars + 256;
+constexpr int kDrThreads = 224;
+constexpr int kDrTmemCols = 256;
+constexpr uint32_t kDrIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                              (static_cast<uint32_t>(kDrN >> 3) << 17) |
+                              (static_cast<uint32_t>(kDrM >> 4) << 24);
+static_assert(kDrSmem <= 227 * 1024, "shared memory");
+
+bool pre_bwd_dr_tc_supported(int64_t T, int64_t H) {
+  return T >= 1 && H >= 128 && H % 128 == 0 && (T + kDrM - 1) / kDrM <= (int64_t(1) << 24);
+}
+
+size_t pre_bwd_dr_tc_workspace_bytes(int64_t T, int64_t H) {
+  if (!pre_bwd_dr_tc_supported(T, H)) return 0;
+  auto up = [](size_t v) { return (v + 1023) / 1024 * 1024; };
+  return up(static_cast<size_t>(T) * kDrKd * 2) + up(static_cast<size_t>(4 * H) * kDrKd * 2);
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void dr_umma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(kDrIdesc), "r"(accumulate)
+      : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 32-byte swizzle, 8-row groups 256 bytes apart (one
+// K=16 step of bf16 per 32-byte row).
+__device__ __forceinline__ uint64_t sw32_desc(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
+         (static_cast<uint64_t>(256 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+         (static_cast<uint64_t>(6) << 61);
+}
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y,
+                                             const void* src) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(x), "r"(y), "r"(smem_u32(src))
+      : "memory");
+}
+
+// A[t] = [hi | hi | lo] of d_raw (backward record floats 0..23), B[k] = [hi | lo | hi] of
+// hc_fn[k]; columns 72..127 zero. One thread per row, 16-byte stores.
+__global__ void __launch_bounds__(256) pre_bwd_split_kernel(const float* __restrict__ brec,
+                                                            const float* __restrict__ W,
+                                                            uint16_t* __restrict__ A,
+                                                            uint16_t* __restrict__ B, int64_t T,
+                                                            int64_t K, int rec_stride) {
+  pdl_wait();
+  pdl_trigger();
+  for (int64_t r = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; r < T + K;
+       r += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const bool is_a = r < T;
+    const float* src = is_a ? brec + r * rec_stride : W + (r - T) * kMix;
+    uint16_t* dst = is_a ? A + r * kDrKd : B + (r - T) * kDrKd;
+    uint16_t hi[kMix], lo[kMix];
+#pragma unroll
+    for (int j = 0; j < kMix; ++j) {
+      const float v = src[j];
+      hi[j] = f32_to_bf16(v);
+      lo[j] = f32_to_bf16(v - bf16_to_f32(hi[j]));
+    }
+    uint32_t row[64];  // 128 bf16
+#pragma unroll
+    for (int c = 0; c < 64; ++c) {
+      uint16_t e[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int col = 2 * c + u;
+        const int grp = col / kMix, j = col - grp * kMix;
+        e[u] = col >= 3 * kMix ? 0
+               : grp == 0       ? hi[j]
+               : grp == 1       ? (is_a ? hi[j] : lo[j])
+                                : (is_a ? lo[j] : hi[j]);
+      }
+      row[c] = static_cast<uint32_t>(e[0]) | (static_cast<uint32_t>(e[1]) << 16);
+    }
+#pragma unroll
+    for (int q = 0; q < 16; ++q)
+      reinterpret_cast<uint4*>(dst)[q] =
+          make_uint4(row[4 * q], row[4 * q + 1], row[4 * q + 2], row[4 * q + 3]);
+  }
+}
+
+struct DrArgs {
+  const float* brec;
+  int64_t T, H, ntt, nhc, W;
+  int rec_stride;
+};
+
+__global__ void __launch_bounds__(kDrThreads, 1)
+    pre_bwd_dr_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      const __grid_constant__ CUtensorMap tmA16, const __grid_constant__ CUtensorMap tmB16,
+                      const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmDy,
+                      const __grid_constant__ CUtensorMap tmDR, const DrArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
+  uint8_t* sA = smem + kDrOffA;
+  uint8_t* sDy = smem + kDrOffDy;
+  uint8_t* sB = smem + kDrOffB;
+  uint8_t* sRr = smem + kDrOffR;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kDrOffBars);
+  uint64_t* rfull = bars;          // [3] R tile landed
+  uint64_t* rempty = bars + 3;     // [3] d_R stored from the slot (the store has read it)
+  uint64_t* afull = bars + 6;      // [2] accumulator ready
+  uint64_t* aempty = bars + 8;     // [2] accumulator read out (4 warps)
+  uint64_t* dyfull = bars + 10;    // [2] d_y buffer landed
+  uint64_t* dyempty = bars + 12;   // [2] d_y buffer's group finished (4 warps)
+  uint64_t* abar = bars + 14;      // A landed
+  uint64_t* afree = bars + 15;     // MMAs on the previous A finished
+  uint64_t* adone = bars + 16;     // MMA warp's own commit point
+  uint64_t* done = bars + 17;
+  uint64_t* bfull = bars + 18;     // [2] B landed
+  uint64_t* bempty = bars + 20;    // [2] MMAs on B finished
+  uint64_t* drready = bars + 22;   // [2] d_R tile of an R slot written (4 warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t P = gridDim.x;
+  const int64_t lo = blockIdx.x * a.W / P, hi = (blockIdx.x + 1) * a.W / P;
+  const int64_t per_tt = a.nhc * 4;
+
+  if (threadIdx.x == 0) {
+    for (int r = 0; r < kDrRSlots; ++r) {
+      mbar_init(&rfull[r], 1);
+      mbar_init(&rempty[r], 1);
+      mbar_init(&drready[r], 4);
+    }
+    for (int b = 0; b < kDrBSlots; ++b) {
+      mbar_init(&bfull[b], 1);
+      mbar_init(&bempty[b], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&afull[b], 1);
+      mbar_init(&aempty[b], 4);
+      mbar_init(&dyfull[b], 1);
+      mbar_init(&dyempty[b], 4);
+    }
+    mbar_init(abar, 1);
+    mbar_init(afree, 1);
+    mbar_init(adone, 1);
+    mbar_init(done, 1);
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kDrTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // the records, the split operands and d_R's previous readers are done
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int64_t it = 0, nbl = 0, na = 0, ng = 0, cur_tt = -1, cur_g = -1;
+      bool ok = true;
+      for (int64_t w = lo; w < hi && ok; ++w) {
+        const int64_t tt = w / per_tt;
+        const int64_t rem = w - tt * per_tt;
+        const int64_t hc = rem >> 2;
+        const int64_t i = rem & 3;
+        const int64_t g = w >> 2;
+        const int y = static_cast<int>(tt * kDrM);
+        if (tt != cur_tt) {
+          if (na > 0 && !mbar_wait(afree, static_cast<uint32_t>(na - 1) & 1u, 90)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(abar, kDrOpTile);
+          tma_load_2d(sA, &tmA, 0, y, abar);
+          tma_load_2d(sA + kDrAtom, &tmA16, 64, y, abar);
+          ++na;
+          cur_tt = tt;
+        }
+        if (g != cur_g) {
+          const int gb = static_cast<int>(ng & 1);
+          if (ng >= 2 &&
+              !mbar_wait(&dyempty[gb], static_cast<uint32_t>((ng - 2) >> 1) & 1u, 91)) {
+            ok = false;
+            break;
+          }
+          uint8_t* d = sDy + gb * kDrTile;
+          mbar_arrive_expect_tx(&dyfull[gb], kDrTile);
+          tma_load_2d(d, &tmDy, static_cast<int>(hc * kDrN), y, &dyfull[gb]);
+          tma_load_2d(d + kDrAtom, &tmDy, static_cast<int>(hc * kDrN + 64), y, &dyfull[gb]);
+          ++ng;
+          cur_g = g;
+        }
+        const int k0 = static_cast<int>(i * a.H + hc * kDrN);
+        // R first (the HBM stream; the ring slot is free once the item three back is stored),
+        // then B (one buffer: free once the previous item's MMAs have read it).
+        const int rs = static_cast<int>(it % kDrRSlots);
+        if (it >= kDrRSlots &&
+            !mbar_wait(&rempty[rs], static_cast<uint32_t>((it - kDrRSlots) / kDrRSlots) & 1u, 92)) {
+          ok = false;
+          break;
+        }
+        uint8_t* rt = sRr + rs * kDrTile;
+        mbar_arrive_expect_tx(&rfull[rs], kDrTile);
+        tma_load_2d(rt, &tmR, k0, y, &rfull[rs]);
+        tma_load_2d(rt + kDrAtom, &tmR, k0 + 64, y, &rfull[rs]);
+        ++it;
+        const int bs = static_cast<int>(nbl % kDrBSlots);
+        if (nbl >= kDrBSlots &&
+            !mbar_wait(&bempty[bs], static_cast<uint32_t>((nbl - kDrBSlots) / kDrBSlots) & 1u, 92)) {
+          ok = false;
+          break;
+        }
+        uint8_t* bt = sB + bs * kDrOpTile;
+        mbar_arrive_expect_tx(&bfull[bs], kDrOpTile);
+        tma_load_2d(bt, &tmB, 0, k0, &bfull[bs]);
+        tma_load_2d(bt + kDrAtom, &tmB16, 64, k0, &bfull[bs]);
+        ++nbl;
+      }
+      // Do not leave while copies into shared memory are in flight (every issued load completes
+      // its barrier; waiting on the last phases of each is enough).
+      if (!ok) {
+        for (int64_t k = it - kDrRSlots; k < it; ++k)
+          if (k >= 0)
+            mbar_wait(&rfull[k % kDrRSlots], static_cast<uint32_t>(k / kDrRSlots) & 1u, 93);
+        for (int64_t k = nbl - kDrBSlots; k < nbl; ++k)
+          if (k >= 0)
+            mbar_wait(&bfull[k % kDrBSlots], static_cast<uint32_t>(k / kDrBSlots) & 1u, 93);
+        if (ng > 0) mbar_wait(&dyfull[(ng - 1) & 1], static_cast<uint32_t>((ng - 1) >> 1) & 1u, 93);
+        if (ng > 1) mbar_wait(&dyfull[(ng - 2) & 1], static_cast<uint32_t>((ng - 2) >> 1) & 1u, 93);
+        if (na > 0) mbar_wait(abar, static_cast<uint32_t>(na - 1) & 1u, 93);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int64_t it = 0, na = 0, cur_tt = -1;
+      bool ok = true;
+      for (int64_t w = lo; w < hi && ok; ++w) {
+        const int64_t tt = w / per_tt;
+        if (tt != cur_tt) {
+          if (na > 0) {  // every MMA on the previous A has finished before the producer reloads it
+            umma_commit(adone);
+            if (!mbar_wait(adone, static_cast<uint32_t>(na - 1) & 1u, 94)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive(afree);
+          }
+          if (!mbar_wait(abar, static_cast<uint32_t>(na) & 1u, 95)) {
+            ok = false;
+            break;
+          }
+          ++na;
+          cur_tt = tt;
+        }
+        const int b = static_cast<int>(it & 1);
+        const int bs = static_cast<int>(it % kDrBSlots);
+        if (!mbar_wait(&bfull[bs], static_cast<uint32_t>(it / kDrBSlots) & 1u, 96)) {
+          ok = false;
+          break;
+        }
+        if (it >= 2 && !mbar_wait(&aempty[b], static_cast<uint32_t>((it - 2) >> 1) & 1u, 97)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t aaddr = smem_u32(sA);
+        const uint32_t baddr = smem_u32(sB + bs * kDrOpTile);
+        const uint32_t dt = tmem + static_cast<uint32_t>(b * kDrN);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)  // split columns 0..63: +32 bytes along the row per step
+          dr_umma(dt, sw128_desc(aaddr) + 2 * k, sw128_desc(baddr) + 2 * k, k > 0 ? 1u : 0u);
+        dr_umma(dt, sw32_desc(aaddr + kDrAtom), sw32_desc(baddr + kDrAtom), 1u);  // 64..79
+        umma_commit(&bempty[bs]);  // B read: the slot may take a later item's B
+        umma_commit(&afull[b]);
+        ++it;
+      }
+      umma_commit(done);  // every issued MMA has finished before TMEM is released
+      mbar_wait(done, 0, 98);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter
+    const int row = q * 32 + lane;
+    int64_t it = 0, ng = 0, cur_g = -1;
+    int gb = 0;
+    uint32_t gph = 0;
+    for (int64_t w = lo; w < hi; ++w) {
+      const int64_t tt = w / per_tt;
+      const int64_t rem = w - tt * per_tt;
+      const int64_t hc = rem >> 2;
+      const int64_t i = rem & 3;
+      const int64_t g = w >> 2;
+      if (g != cur_g) {
+        if (cur_g >= 0) {  // this warp is done with the previous group's d_y buffer
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&dyempty[gb]);
+        }
+        gb = static_cast<int>(ng & 1);
+        gph = static_cast<uint32_t>(ng >> 1) & 1u;
+        ++ng;
+        cur_g = g;
+      }
+      const int rs = static_cast<int>(it % kDrRSlots);
+      const int b = static_cast<int>(it & 1);
+      bool ok = __all_sync(
+          0xffffffffu,
+          mbar_wait(&rfull[rs], static_cast<uint32_t>(it / kDrRSlots) & 1u, 99));
+      ok = ok && __all_sync(0xffffffffu, mbar_wait(&dyfull[gb], gph, 100));
+      ok = ok && __all_sync(0xffffffffu,
+                            mbar_wait(&afull[b], static_cast<uint32_t>(it >> 1) & 1u, 101));
+      // The four warps agree on going on (a stop keeps the named-barrier sequence matched).
+      if (named_bar_or(1, 128, !ok)) break;
+      tc_fence_after();
+      const int64_t tok = tt * kDrM + row;
+      float dss2 = 0.f, pi = 0.f;
+      if (tok < a.T) {
+        dss2 = 2.0f * __ldg(a.brec + tok * a.rec_stride + 24);
+        pi = __ldg(a.brec + tok * a.rec_stride + 25 + i);
+      }
+      uint8_t* sR = sRr + rs * kDrTile;
+      const uint8_t* sY = sDy + gb * kDrTile;
+      const uint32_t tbase =
+          tmem + static_cast<uint32_t>(b * kDrN) + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        uint32_t acc[2][32];
+        tmem_ld32(tbase + half * 64, acc[0]);
+        tmem_ld32(tbase + half * 64 + 32, acc[1]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int hq = 0; hq < 2; ++hq) {
+          const int cq = half * 2 + hq;
+          const int atom = cq >> 1;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            // 16-byte chunk c of the row's 128-byte swizzled line sits at chunk c ^ (row & 7).
+            const int c = (cq & 1) * 4 + u;
+            const int off = atom * kDrAtom + row * 128 + ((c ^ (row & 7)) << 4);
+            const uint4 rv = *reinterpret_cast<const uint4*>(sR + off);
+            const uint4 yv = *reinterpret_cast<const uint4*>(sY + off);
+            const uint32_t r4[4] = {rv.x, rv.y, rv.z, rv.w};
+            const uint32_t y4[4] = {yv.x, yv.y, yv.z, yv.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float a0 = __uint_as_float(acc[hq][8 * u + 2 * e]);
+              const float a1 = __uint_as_float(acc[hq][8 * u + 2 * e + 1]);
+              o[e] = pack_bf16x2(fmaf(pi, bf16_lo(y4[e]), fmaf(dss2, bf16_lo(r4[e]), a0)),
+                                 fmaf(pi, bf16_hi(y4[e]), fmaf(dss2, bf16_hi(r4[e]), a1)));
+            }
+            *reinterpret_cast<uint4*>(sR + off) = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        }
+      }
+      tc_fence_before();
+      // The rows are written: the accumulator goes back to the MMA warp, and the d_R tile (in R's
+      // slot) to the storer, with the generic-proxy writes made visible to the TMA engine.
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&aempty[b]);
+        mbar_arrive(&drready[rs]);
+      }
+      ++it;
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------------ d_R storer
+    if (lane == 0) {
+      int64_t it = 0;
+      for (int64_t w = lo; w < hi; ++w, ++it) {
+        const int64_t tt = w / per_tt;
+        const int64_t rem = w - tt * per_tt;
+        const int64_t hc = rem >> 2;
+        const int64_t i = rem & 3;
+        const int rs = static_cast<int>(it % kDrRSlots);
+        if (!mbar_wait(&drready[rs], static_cast<uint32_t>(it / kDrRSlots) & 1u, 102)) break;
+        const uint8_t* sR = sRr + rs * kDrTile;
+        const int x = static_cast<int>(i * a.H + hc * kDrN);
+        const int y = static_cast<int>(tt * kDrM);
+        tma_store_2d(&tmDR, x, y, sR);
+        tma_store_2d(&tmDR, x + 64, y, sR + kDrAtom);
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // the slot has been read
+        mbar_arrive(&rempty[rs]);
+      }
+      asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");  // stores complete before exit
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kDrTmemCols)
+                 : "memory");
+  }
+}
+
+// Returns 0, a negative MHC_ERR_* code, or 1 when this form cannot run (nothing launched).
+int launch_pre_bwd_dr_tc(const uint16_t* R, const uint16_t* dy, const float* hc_fn,
+                         const float* brec, int rec_stride, uint16_t* dR, void* ws, int64_t T,
+                         int64_t H, cudaStream_t s) {
+  if (!pre_bwd_dr_tc_supported(T, H) || dy == nullptr || !aligned16(R) || !aligned16(dy) ||
+      !aligned16(dR) || !aligned16(ws))
+    return 1;
+  if (!ensure_smem_limit(reinterpret_cast<const void*>(pre_bwd_dr_kernel), kDrSmem)) return 1;
+  const int64_t K = 4 * H;
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  uint16_t* A = reinterpret_cast<uint16_t*>(w8);
+  uint16_t* B = reinterpret_cast<uint16_t*>(
+      w8 + (static_cast<size_t>(T) * kDrKd * 2 + 1023) / 1024 * 1024);
+  CUtensorMap mA, mB, mA16, mB16, mR, mDy, mDR;
+  // [rows x 16] boxes of columns 64..79, 32-byte swizzle.
+  auto narrow_map = [](CUtensorMap* m, const void* base, int64_t rows) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDrKd), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDrKd) * 2};
+    const cuuint32_t box[2] = {16, 128};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  };
+  if (!make_map(&mA, A, kDrKd, T, kDrM) || !make_map(&mB, B, kDrKd, K, kDrN) ||
+      !narrow_map(&mA16, A, T) || !narrow_map(&mB16, B, K) ||
+      !make_map(&mR, R, K, T, kDrM) || !make_map(&mDy, dy, H, T, kDrM) ||
+      !make_map(&mDR, dR, K, T, kDrM))
+    return -4;
+  int64_t nb = (T + K + 255) / 256;
+  if (nb > 148 * 8) nb = 148 * 8;
+  if (launch_pdl(pre_bwd_split_kernel, dim3(static_cast<unsigned>(nb)), dim3(256), 0, s, brec,
+                 hc_fn, A, B, T, K, rec_stride) != cudaSuccess)
+    return -4;
+  DrArgs da;
+  da.brec = brec;
+  da.T = T;
+  da.H = H;
+  da.ntt = (T + kDrM - 1) / kDrM;
+  da.nhc = H / kDrN;
+  da.W = da.ntt * da.nhc * 4;
+  da.rec_stride = rec_stride;
+  int P = device_sm_count();
+  if (P > 148) P = 148;
+  if (static_cast<int64_t>(P) > da.W) P = static_cast<int>(da.W);
+  if (launch_pdl(pre_bwd_dr_kernel, dim3(static_cast<unsigned>(P)), dim3(kDrThreads),
+                 static_cast<size_t>(kDrSmem), s, mA, mB, mA16, mB16, mR, mDy, mDR, da) !=
+      cudaSuccess)
+    return -4;
+  note_launches(2);
+  return 0;
+}
+
+}  // namespace mhc

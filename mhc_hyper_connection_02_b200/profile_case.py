@@ -41,6 +41,8 @@ CASES = {
     "expand_scalar_H1001": ("mhc_expand T=8192 H=1001", "expand_scalar_kernel"),
     "head_mean_scalar_H1001": ("mhc_head_mean T=8192 H=1001", "head_mean_scalar_kernel"),
     "pre_backward_H1001": ("mhc_pre_backward T=4096 H=1001", "pre_bwd_* (dx scalar form)"),
+    "pre_backward_large": ("mhc_pre_backward T=8192 H=7168",
+                           "pre_bwd_* (d_R on tensor cores: pre_bwd_split_kernel, pre_bwd_dr_kernel)"),
 }
 
 
@@ -124,8 +126,8 @@ def make_call(case):
         _, R, _, _, _, _ = _inputs(8192, 1001)
         y = torch.empty((8192, 1001), dtype=torch.bfloat16, device="cuda")
         return lambda: head_mean(R, y=y)
-    if case == "pre_backward_H1001":
-        T, H = 4096, 1001
+    if case in ("pre_backward_H1001", "pre_backward_large"):
+        T, H = (4096, 1001) if case == "pre_backward_H1001" else (8192, 7168)
         g, R, x, W, S, B = _inputs(T, H)
         dy = torch.randn((T, H), device="cuda", generator=g).to(torch.bfloat16)
         return lambda: pre_backward(R, W, S, B, d_y=dy)
