@@ -16,8 +16,9 @@
 //   5. d_R = d_raw . hc_fn^T + 2 R d_ss + pre_i d_y: on tcgen05 tensor cores where H % 128 == 0
 //      and d_y is given (mhc_backward_tc.cu), else column slice x token chunk per CTA, a thread's
 //      hc_fn weights in registers, fp32 on CUDA cores;
-//   6. d_hc_fn = R_flat^T d_raw (column slice x token chunk per CTA, tokens summed in order, then
-//      the chunks in order).
+//   6. d_hc_fn = R_flat^T d_raw: on tcgen05 where 4H % 128 == 0 (mhc_backward_tc.cu: R read
+//      MN-major as the A operand), else column slice x token chunk per CTA on CUDA cores; the
+//      partials are summed in order.
 #include "mhc_device.cuh"
 #include "mhc_internal.h"
 
@@ -667,7 +668,7 @@ __global__ void __launch_bounds__(256) pre_bwd_dw_sum_kernel(const float* __rest
 }
 
 struct BwPlan {
-  size_t proj, dpt, brec, dwp, drtc, total;
+  size_t proj, dpt, brec, dwp, drtc, dwtc, total;
   int64_t tchunk;
   int nchunk;
 };
@@ -690,7 +691,8 @@ static BwPlan bw_plan(int64_t T, int64_t H) {
   p.nchunk = static_cast<int>((T + p.tchunk - 1) / p.tchunk);
   p.dwp = up(static_cast<size_t>(p.nchunk) * 4 * H * kMix * 4);
   p.drtc = up(pre_bwd_dr_tc_workspace_bytes(T, H));  // split operands of the tensor-core d_R
-  p.total = p.proj + p.dpt + p.brec + p.dwp + p.drtc;
+  p.dwtc = up(pre_bwd_dw_tc_workspace_bytes(T, H));  // B operand and partials of its d_hc_fn
+  p.total = p.proj + p.dpt + p.brec + p.dwp + p.drtc + p.dwtc;
   return p;
 }
 
@@ -706,6 +708,7 @@ int launch_pre_backward(const PreBwdArgs& a, cudaStream_t s) {
   float* brec = reinterpret_cast<float*>(ws + plan.proj + plan.dpt);
   float* dwp = reinterpret_cast<float*>(ws + plan.proj + plan.dpt + plan.brec);
   void* drtc_ws = ws + plan.proj + plan.dpt + plan.brec + plan.dwp;
+  void* dwtc_ws = ws + plan.proj + plan.dpt + plan.brec + plan.dwp + plan.drtc;
   const int64_t K = 4 * a.H;
   if (a.T > 0x7fffffff) return -5;
 
@@ -769,22 +772,29 @@ int launch_pre_backward(const PreBwdArgs& a, cudaStream_t s) {
                    a.R, a.dy, a.hc_fn, static_cast<const float*>(brec), a.dR, a.T, a.H);
   }
   if (e != cudaSuccess) return -4;
-  // 6. d_hc_fn.
-  const dim3 gw(static_cast<unsigned>((K + kDwCols - 1) / kDwCols),
-                static_cast<unsigned>(plan.nchunk));
-  const bool dwvec = a.H % 8 == 0 && aligned16(a.R);
-  e = dwvec ? launch_pdl(pre_bwd_dw_kernel<true>, gw, dim3(kDwThreads), 0, s, a.R,
-                         static_cast<const float*>(brec), dwp, a.T, a.H, plan.tchunk)
-            : launch_pdl(pre_bwd_dw_kernel<false>, gw, dim3(kDwThreads), 0, s, a.R,
-                         static_cast<const float*>(brec), dwp, a.T, a.H, plan.tchunk);
-  if (e != cudaSuccess) return -4;
-  int64_t nb = (K * kMix + 255) / 256;
-  if (nb > 148 * 8) nb = 148 * 8;
-  e = launch_pdl(pre_bwd_dw_sum_kernel, dim3(static_cast<unsigned>(nb)), dim3(256), 0, s,
-                 static_cast<const float*>(dwp), a.dW, K * kMix, plan.nchunk);
-  if (e != cudaSuccess) return -4;
-  // dpre, coef, param, d_R on CUDA cores (the tensor-core form counts its own two), dw, dw_sum.
-  note_launches(dr == 0 ? 5 : 6);
+  // 6. d_hc_fn: on tensor cores where 4H % 128 == 0 (1: not this shape, nothing launched), else
+  // CUDA-core partials over token chunks; then the partials' in-order sum.
+  int dwr = launch_pre_bwd_dw_tc(a.R, static_cast<const float*>(brec), kBrec, a.dW, dwtc_ws, a.T,
+                                 a.H, s);
+  if (dwr < 0) return dwr;
+  if (dwr == 1) {
+    const dim3 gw(static_cast<unsigned>((K + kDwCols - 1) / kDwCols),
+                  static_cast<unsigned>(plan.nchunk));
+    const bool dwvec = a.H % 8 == 0 && aligned16(a.R);
+    e = dwvec ? launch_pdl(pre_bwd_dw_kernel<true>, gw, dim3(kDwThreads), 0, s, a.R,
+                           static_cast<const float*>(brec), dwp, a.T, a.H, plan.tchunk)
+              : launch_pdl(pre_bwd_dw_kernel<false>, gw, dim3(kDwThreads), 0, s, a.R,
+                           static_cast<const float*>(brec), dwp, a.T, a.H, plan.tchunk);
+    if (e != cudaSuccess) return -4;
+    int64_t nb = (K * kMix + 255) / 256;
+    if (nb > 148 * 8) nb = 148 * 8;
+    e = launch_pdl(pre_bwd_dw_sum_kernel, dim3(static_cast<unsigned>(nb)), dim3(256), 0, s,
+                   static_cast<const float*>(dwp), a.dW, K * kMix, plan.nchunk);
+    if (e != cudaSuccess) return -4;
+    note_launches(2);
+  }
+  // dpre, coef, param, d_R on CUDA cores (the tensor-core forms count their own launches).
+  note_launches(dr == 0 ? 3 : 4);
   return 0;
 }
 

@@ -473,6 +473,328 @@ __global__ void __launch_bounds__(kDrThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------------------ d_hc_fn
+//
+// d_hc_fn[k][j] = sum_t R[t][k] d_raw[t][j]: a contraction over tokens. The MMA's M is 128 features
+// k, its K the tokens, so the A operand is R itself read MN-major: a TMA box [64 tokens x 64
+// features] of R lands as 64 lines of 128 bytes (one token each, features contiguous) with the
+// 128-byte swizzle, which is the MN-major swizzled atom (64 features x 8 tokens, 1 KB); the two
+// boxes of a 128-feature tile are the two atoms along M. B = [hi(d_raw) | lo(d_raw)] transposed,
+// [48][tokens] bf16 (K-major), so each product is hi.R + lo.R, exact in fp32 (R is exact in bf16;
+// hi + lo leaves below 2^-16 of d_raw).
+//
+// pre_bwd_dw_kernel_tc: persistent, two CTAs per SM; the (feature tile, 64-token block) units,
+// tile-major, cut into equal contiguous ranges; a range covers pieces (tile, token interval) whose
+// rank among the tile's pieces is their slot. Warp 0: TMA of both R boxes and the B block per
+// stage (4 stages of 22 KB); warp 1: four M=128 N=48 K=16 MMAs per block into one of two TMEM
+// accumulators, restarted every 16 blocks (1024 tokens: short fp32 chains); warps 2-5: each
+// finished sub-piece's accumulator (tcgen05.ld) added, as hi + lo, into registers in order; at
+// the piece's end the thread of feature k writes the partial [slot][k][24]. The CTA holding a
+// tile's last piece zero-fills the tile's unused slots; pre_bwd_dw_sum_kernel adds the slots in
+// order.
+
+constexpr int kWtM = 128;
+constexpr int kWtN = 48;
+constexpr int kWtTok = 64;                         // tokens per block
+constexpr int kWtABytes = 2 * kWtTok * 128;        // two [64 x 64] boxes of R: 16 KB
+constexpr int kWtBBytes = kWtN * 128;              // [48 x 64 tokens]: 6 KB
+constexpr int kWtStageBytes = kWtABytes + kWtBBytes;  // 22528 = 22 x 1024
+constexpr int kWtStages = 4;
+// Slack after the stages: an MMA reading through a misread descriptor stride stays inside the
+// allocation (the tile spans at most 16 KB from its base whatever the strides' roles).
+constexpr int kWtSlack = 16384;
+constexpr int kWtOffBars = kWtStages * kWtStageBytes + kWtSlack;
+constexpr int kWtSmem = 1024 + kWtOffBars + 256;
+constexpr int kWtThreads = 192;
+constexpr int kWtTmemCols = 128;                   // two accumulators of 48 columns (0, 64)
+constexpr int kWtSubBlocks = 16;
+constexpr int kWtMinUnits = 8;
+// kind::f16, D fp32, A and B bf16, A MN-major (bit 15), B K-major, N = 48, M = 128.
+constexpr uint32_t kWtIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) |
+                              (static_cast<uint32_t>(kWtN >> 3) << 17) |
+                              (static_cast<uint32_t>(kWtM >> 4) << 24);
+
+// MN-major, 128-byte swizzle: the second 64-feature atom 8 KB on (leading byte offset), the next
+// 8 tokens 1 KB on (stride byte offset).
+__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) |
+         (static_cast<uint64_t>(kWtTok * 128 >> 4) << 16) |
+         (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+         (static_cast<uint64_t>(2) << 61);
+}
+
+__device__ __forceinline__ void wt_umma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(kWtIdesc), "r"(accumulate)
+      : "memory");
+}
+
+struct WtPlan {
+  int64_t nk, NB, Tp, W, P, S;
+};
+
+static WtPlan wt_plan(int64_t T, int64_t H, int64_t sms) {
+  WtPlan p;
+  p.nk = 4 * H / kWtM;
+  p.NB = (T + kWtTok - 1) / kWtTok;
+  p.Tp = p.NB * kWtTok;
+  p.W = p.nk * p.NB;
+  p.P = 2 * sms;
+  if (p.P > 2 * 148) p.P = 2 * 148;
+  if (p.P > p.W / kWtMinUnits) p.P = p.W / kWtMinUnits;
+  if (p.P < 1) p.P = 1;
+  p.S = p.NB * p.P / p.W + 2;  // pieces one tile meets at most
+  if (p.S > p.P) p.S = p.P;
+  return p;
+}
+
+bool pre_bwd_dw_tc_supported(int64_t T, int64_t H) {
+  return T >= 1 && H >= 32 && (4 * H) % kWtM == 0 && (T + kWtTok - 1) / kWtTok <= (1 << 24);
+}
+
+size_t pre_bwd_dw_tc_workspace_bytes(int64_t T, int64_t H) {
+  if (!pre_bwd_dw_tc_supported(T, H)) return 0;
+  const WtPlan p = wt_plan(T, H, 148);
+  auto up = [](size_t v) { return (v + 1023) / 1024 * 1024; };
+  return up(static_cast<size_t>(kWtN) * p.Tp * 2) +
+         up(static_cast<size_t>(p.S) * 4 * H * kMix * 4);
+}
+
+// Bt[n][t] = hi(d_raw[t][n]) for n < 24, lo(...) for 24 <= n < 48 (zero for t >= T): consecutive
+// threads take consecutive tokens, so each row's stores coalesce.
+__global__ void __launch_bounds__(256) pre_bwd_bt_kernel(const float* __restrict__ brec,
+                                                         uint16_t* __restrict__ Bt, int64_t T,
+                                                         int64_t Tp, int rec_stride) {
+  pdl_wait();
+  pdl_trigger();
+  for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < Tp;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+#pragma unroll 4
+    for (int j = 0; j < kMix; ++j) {
+      const float v = t < T ? brec[t * rec_stride + j] : 0.f;
+      const uint16_t hi = f32_to_bf16(v);
+      Bt[j * Tp + t] = hi;
+      Bt[(kMix + j) * Tp + t] = f32_to_bf16(v - bf16_to_f32(hi));
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kWtThreads, 2) pre_bwd_dw_kernel_tc(
+    const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmBt,
+    float* __restrict__ dwp, int64_t K, int64_t NB, int64_t W, int S) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWtOffBars);
+  uint64_t* full = bars;                    // [4]
+  uint64_t* empty = bars + kWtStages;       // [4] MMA commit
+  uint64_t* afull = bars + 2 * kWtStages;   // [2]
+  uint64_t* aempty = afull + 2;             // [2] 4 warps
+  uint64_t* done = aempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t P = gridDim.x;
+  const int64_t c = blockIdx.x;
+  const int64_t lo = c * W / P, hi = (c + 1) * W / P;
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kWtStages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&afull[b], 1);
+      mbar_init(&aempty[b], 4);
+    }
+    mbar_init(done, 1);
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kWtTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int64_t n = 0;
+      bool ok = true;
+      for (int64_t u = lo; u < hi; ++u, ++n) {
+        const int64_t kt = u / NB;
+        const int tb = static_cast<int>(u - kt * NB);
+        const int st = static_cast<int>(n % kWtStages);
+        if (n >= kWtStages &&
+            !mbar_wait(&empty[st], static_cast<uint32_t>((n / kWtStages) - 1) & 1u, 110)) {
+          ok = false;
+          break;
+        }
+        uint8_t* sa = smem + st * kWtStageBytes;
+        mbar_arrive_expect_tx(&full[st], kWtStageBytes);
+        tma_load_2d(sa, &tmR, static_cast<int>(kt * kWtM), tb * kWtTok, &full[st]);
+        tma_load_2d(sa + kWtTok * 128, &tmR, static_cast<int>(kt * kWtM + 64), tb * kWtTok,
+                    &full[st]);
+        tma_load_2d(sa + kWtABytes, &tmBt, tb * kWtTok, 0, &full[st]);
+      }
+      if (!ok) {  // do not leave while copies into shared memory are in flight
+        for (int64_t i = n - kWtStages; i < n; ++i)
+          if (i >= 0)
+            mbar_wait(&full[i % kWtStages], static_cast<uint32_t>(i / kWtStages) & 1u, 111);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int64_t n = 0, sp = 0;
+      bool ok = true;
+      uint32_t dt = tmem;
+      for (int64_t u = lo; u < hi && ok;) {
+        const int64_t kt = u / NB;
+        const int64_t tbs = u - kt * NB;
+        const int64_t tbe = min(NB, tbs + (hi - u));
+        for (int64_t tb = tbs; tb < tbe; ++tb, ++n) {
+          const int ks = static_cast<int>((tb - tbs) % kWtSubBlocks);
+          if (ks == 0) {
+            const int b = static_cast<int>(sp & 1);
+            if (sp >= 2 &&
+                !mbar_wait(&aempty[b], static_cast<uint32_t>((sp >> 1) - 1) & 1u, 112)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            dt = tmem + static_cast<uint32_t>(b * 64);
+          }
+          const int st = static_cast<int>(n % kWtStages);
+          if (!mbar_wait(&full[st], static_cast<uint32_t>(n / kWtStages) & 1u, 113)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + st * kWtStageBytes);
+          const uint64_t adesc = sw128_mn_desc(sa);
+          const uint64_t bdesc = sw128_desc(sa + kWtABytes);
+#pragma unroll
+          for (int k = 0; k < kWtTok / 16; ++k)  // 16 tokens: +2 KB of A, +32 bytes of B's rows
+            wt_umma(dt, adesc + 128 * k, bdesc + 2 * k, (ks > 0 || k > 0) ? 1u : 0u);
+          umma_commit(&empty[st]);
+          if (tb + 1 == tbe || ks + 1 == kWtSubBlocks) {
+            umma_commit(&afull[sp & 1]);
+            ++sp;
+          }
+        }
+        u += tbe - tbs;
+      }
+      umma_commit(done);
+      mbar_wait(done, 0, 114);
+    }
+  } else {
+    // Warps 2..5: TMEM lane quarter q holds features 32q .. 32q + 31 of the tile.
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    int64_t sp = 0;
+    bool ok = true;
+    for (int64_t u = lo; u < hi && ok;) {
+      const int64_t kt = u / NB;
+      const int64_t tbs = u - kt * NB;
+      const int64_t tbe = min(NB, tbs + (hi - u));
+      float racc[kMix];
+#pragma unroll
+      for (int j = 0; j < kMix; ++j) racc[j] = 0.f;
+      for (int64_t b0 = tbs; b0 < tbe; b0 += kWtSubBlocks, ++sp) {
+        const int b = static_cast<int>(sp & 1);
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(&afull[b], static_cast<uint32_t>(sp >> 1) & 1u, 115))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t d[3][16];
+        const uint32_t tbase =
+            tmem + static_cast<uint32_t>(b * 64) + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll
+        for (int cc = 0; cc < 3; ++cc) tmem_ld16(tbase + cc * 16, d[cc]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < kMix; ++j) {
+          const float h = __uint_as_float(d[j / 16][j % 16]);
+          const float l = __uint_as_float(d[(kMix + j) / 16][(kMix + j) % 16]);
+          racc[j] += l + h;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&aempty[b]);
+      }
+      if (!ok) break;
+      const int64_t slot = c - tc_first_cta(kt * NB, P, W);
+      const int64_t k = kt * kWtM + row;
+      float4* dst = reinterpret_cast<float4*>(dwp + (slot * K + k) * kMix);
+#pragma unroll
+      for (int w4 = 0; w4 < kMix / 4; ++w4)
+        dst[w4] = make_float4(racc[4 * w4], racc[4 * w4 + 1], racc[4 * w4 + 2], racc[4 * w4 + 3]);
+      if (tbe == NB) {  // the tile's last piece: zero its unused slots
+        for (int64_t sl = slot + 1; sl < S; ++sl) {
+          float4* z = reinterpret_cast<float4*>(dwp + (sl * K + k) * kMix);
+#pragma unroll
+          for (int w4 = 0; w4 < kMix / 4; ++w4) z[w4] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      u += tbe - tbs;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kWtTmemCols)
+                 : "memory");
+  }
+}
+
+// d_hc_fn on tensor cores: Bt, the partials, their in-order sum. Returns 0, a negative MHC_ERR_*
+// code, or 1 when this form cannot run (nothing launched).
+int launch_pre_bwd_dw_tc(const uint16_t* R, const float* brec, int rec_stride, float* dW,
+                         void* ws, int64_t T, int64_t H, cudaStream_t s) {
+  if (!pre_bwd_dw_tc_supported(T, H) || !aligned16(R) || !aligned16(ws)) return 1;
+  if (!ensure_smem_limit(reinterpret_cast<const void*>(pre_bwd_dw_kernel_tc), kWtSmem)) return 1;
+  const int64_t K = 4 * H;
+  const WtPlan plan = wt_plan(T, H, device_sm_count());
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  uint16_t* Bt = reinterpret_cast<uint16_t*>(w8);
+  float* dwp = reinterpret_cast<float*>(
+      w8 + (static_cast<size_t>(kWtN) * plan.Tp * 2 + 1023) / 1024 * 1024);
+  CUtensorMap mR, mBt;
+  if (!make_map(&mR, R, K, T, kWtTok) || !make_map(&mBt, Bt, plan.Tp, kWtN, kWtN)) return -4;
+  int64_t nb = (plan.Tp + 255) / 256;
+  if (nb > 148 * 8) nb = 148 * 8;
+  if (launch_pdl(pre_bwd_bt_kernel, dim3(static_cast<unsigned>(nb)), dim3(256), 0, s, brec, Bt, T,
+                 plan.Tp, rec_stride) != cudaSuccess)
+    return -4;
+  if (launch_pdl(pre_bwd_dw_kernel_tc, dim3(static_cast<unsigned>(plan.P)), dim3(kWtThreads),
+                 static_cast<size_t>(kWtSmem), s, mR, mBt, dwp, K, plan.NB, plan.W,
+                 static_cast<int>(plan.S)) != cudaSuccess)
+    return -4;
+  int64_t sb = (K * kMix + 255) / 256;
+  if (sb > 148 * 8) sb = 148 * 8;
+  if (launch_pdl(pre_bwd_dw_sum_kernel, dim3(static_cast<unsigned>(sb)), dim3(256), 0, s,
+                 static_cast<const float*>(dwp), dW, K * kMix, static_cast<int>(plan.S)) !=
+      cudaSuccess)
+    return -4;
+  note_launches(3);
+  return 0;
+}
+
 // Returns 0, a negative MHC_ERR_* code, or 1 when this form cannot run (nothing launched).
 int launch_pre_bwd_dr_tc(const uint16_t* R, const uint16_t* dy, const float* hc_fn,
                          const float* brec, int rec_stride, uint16_t* dR, void* ws, int64_t T,

@@ -172,6 +172,11 @@ size_t pre_bwd_dr_tc_workspace_bytes(int64_t T, int64_t H);
 int launch_pre_bwd_dr_tc(const uint16_t* R, const uint16_t* dy, const float* hc_fn,
                          const float* brec, int rec_stride, uint16_t* dR, void* ws, int64_t T,
                          int64_t H, cudaStream_t s);
+// d_hc_fn of the pre-map backward on tensor cores: same return convention.
+bool pre_bwd_dw_tc_supported(int64_t T, int64_t H);
+size_t pre_bwd_dw_tc_workspace_bytes(int64_t T, int64_t H);
+int launch_pre_bwd_dw_tc(const uint16_t* R, const float* brec, int rec_stride, float* dW,
+                         void* ws, int64_t T, int64_t H, cudaStream_t s);
 int launch_pre_backward(const PreBwdArgs& a, cudaStream_t s);
 
 // Model-boundary operations (mhc_boundary.cu).

@@ -75,7 +75,8 @@ def _pre_case(T, H, seed, with_dy=True, with_comb=True):
 
 
 @pytest.mark.parametrize("T,H", [(1, 8), (5, 127), (64, 512), (130, 1000), (300, 2048),
-                                 (20, 7168), (3, 1001), (1000, 1024), (513, 4096), (777, 256)])
+                                 (20, 7168), (3, 1001), (1000, 1024), (513, 4096), (777, 256),
+                                 (200, 1056), (3000, 64)])
 def test_pre_backward(T, H):
     w, d_y, d_pre, d_post, d_comb = _pre_case(T, H, seed=7 * T + H)
     prm = mhc.make_params(iters=w.iters, eps=w.eps, rms_eps=w.rms_eps, pre_eps=w.pre_eps,
@@ -104,11 +105,15 @@ def test_pre_backward(T, H):
     _check_sum(db.cpu().numpy(), rb, np.abs(pt["dl"]).sum(0), 1e-4, "d_base")
 
 
-@pytest.mark.parametrize("T,H,dr_tensor", [(300, 2048, True), (130, 1000, False)])
-def test_pre_backward_d_R_form(T, H, dr_tensor):
+@pytest.mark.parametrize("T,H,dr_tensor,dw_tensor", [(300, 2048, True, True),
+                                                    (130, 1000, False, False),
+                                                    (200, 1056, False, True)])
+def test_pre_backward_d_R_form(T, H, dr_tensor, dw_tensor):
     """H % 128 == 0 with d_y given takes the tcgen05 d_R (split operands + the tensor kernel: two
-    launches); otherwise the CUDA-core kernel (one). Both projections here are the tensor form
-    (split + projection); then d_pre, coefficients, parameters, d_hc_fn and its sum."""
+    launches), otherwise the CUDA-core kernel (one); 4H % 128 == 0 takes the tcgen05 d_hc_fn
+    (transposed d_raw split, the tensor kernel, the partials' sum: three launches), otherwise
+    CUDA-core partials and their sum (two). Both projections here are the tensor form (split +
+    projection); then d_pre, coefficients and parameters."""
     w, d_y, d_pre, d_post, d_comb = _pre_case(T, H, seed=11)
     n0 = mhc.launch_count()
     mhc.pre_backward(dev_bf16(w.R), dev_f32(w.hc_fn), dev_f32(w.hc_scale), dev_f32(w.hc_base),
@@ -116,7 +121,7 @@ def test_pre_backward_d_R_form(T, H, dr_tensor):
                      d_comb=dev_f32(d_comb), params=mhc.make_params(iters=w.iters))
     torch.cuda.synchronize()
     assert mhc.device_status() == 0
-    assert mhc.launch_count() - n0 == 2 + 3 + (2 if dr_tensor else 1) + 2
+    assert mhc.launch_count() - n0 == 2 + 3 + (2 if dr_tensor else 1) + (3 if dw_tensor else 2)
 
 
 def test_pre_backward_optional_gradients_and_tensor_path():
