@@ -9,7 +9,8 @@
 //           gradients, a fixed-order block reduction.
 // pre-map   (upstream d_y, d_pre, d_post, d_comb; any may be absent)
 //   1. the projection is recomputed by the forward's own kernels (records of raw and ss);
-//   2. d_pre += sum_h d_y R_i (one CTA per token);
+//   2. d_pre += sum_h d_y R_i: with the tensor projection (H % 64 == 0) the projection kernel forms
+//      it from the R tiles it streams anyway (record floats 28..31), else one CTA per token;
 //   3. per token (lane quad): rstd, logits, gates, the Sinkhorn forward (states checkpointed)
 //      and the reverse pass -> d_raw, d_ss, the gates, and the per-token terms of d_scale, d_base;
 //   4. d_scale, d_base: fixed-order sums over tokens;
@@ -262,6 +263,7 @@ constexpr int kSkCk = 16;  // Sinkhorn forward checkpoints kept by the reverse p
 // d_scale, [32..55] d_l (the token's term of d_base).
 __global__ void __launch_bounds__(256) pre_bwd_coef_kernel(
     const float* __restrict__ part, int nrec, const float* __restrict__ dpt,
+    const float* __restrict__ dpre_in, int dp_in_records,
     const float* __restrict__ dpost, const float* __restrict__ dcomb,
     const float* __restrict__ scale, const float* __restrict__ base, float* __restrict__ brec,
     int64_t T, int64_t K, FinishParams fp) {
@@ -272,7 +274,7 @@ __global__ void __launch_bounds__(256) pre_bwd_coef_kernel(
   const int64_t tt = live ? t : 0;
   pdl_wait();
   pdl_trigger();
-  float g0 = 0.f, g1 = 0.f, gc[4] = {0.f, 0.f, 0.f, 0.f}, ss = 0.f;
+  float g0 = 0.f, g1 = 0.f, gc[4] = {0.f, 0.f, 0.f, 0.f}, ss = 0.f, dy_r = 0.f;
   for (int s = 0; s < nrec; ++s) {
     const float* rec = part + (static_cast<int64_t>(s) * T + tt) * 32;
     g0 += __ldg(rec + r);
@@ -280,6 +282,7 @@ __global__ void __launch_bounds__(256) pre_bwd_coef_kernel(
 #pragma unroll
     for (int n = 0; n < 4; ++n) gc[n] += __ldg(rec + 8 + 4 * r + n);
     ss += __ldg(rec + 24);
+    if (dp_in_records) dy_r += __ldg(rec + 28 + r);  // sum_h d_y R_r, formed with the projection
   }
   const float rstd = 1.0f / sqrtf(ss / static_cast<float>(K) + fp.rms_eps);
   const float s0 = __ldg(scale), s1 = __ldg(scale + 1), s2 = __ldg(scale + 2);
@@ -292,7 +295,8 @@ __global__ void __launch_bounds__(256) pre_bwd_coef_kernel(
   }
   const float sg0 = 1.0f / (1.0f + expf(-fmaf(m0, s0, __ldg(base + r))));
   const float sg1 = 1.0f / (1.0f + expf(-fmaf(m1, s1, __ldg(base + 4 + r))));
-  const float dl0 = dpt[tt * 4 + r] * sg0 * (1.0f - sg0);
+  const float dpr = dp_in_records ? (dpre_in ? dpre_in[tt * 4 + r] : 0.f) + dy_r : dpt[tt * 4 + r];
+  const float dl0 = dpr * sg0 * (1.0f - sg0);
   const float dl1 = (dpost ? dpost[tt * 4 + r] : 0.f) * fp.post_mult * sg1 * (1.0f - sg1);
 
   // Sinkhorn reverse pass. The forward starts from P = softmax(row) and A0 = P + eps; its states
@@ -720,24 +724,31 @@ int launch_pre_backward(const PreBwdArgs& a, cudaStream_t s) {
   int nrec = 0;
   const bool tc = pre_tc_supported(a.T, a.H) && aligned16(a.R) && aligned16(a.workspace) &&
                   a.T >= 128;
-  int r = tc ? launch_tc_projection(f, s, &part, &nrec) : launch_cc_projection(f, s, &part, &nrec);
+  // With d_y, the tensor projection also forms d_pre's sum_h d_y R_i from the tiles it streams
+  // (one pass over R instead of two); H % 64 == 0 keeps each K block within one stream.
+  const bool dy_fold = tc && a.dy != nullptr && a.H % 64 == 0 && aligned16(a.dy);
+  int r = tc ? launch_tc_projection(f, s, &part, &nrec, dy_fold ? a.dy : nullptr)
+             : launch_cc_projection(f, s, &part, &nrec);
   if (r != 0) return r;
 
   const bool vec = a.H % 8 == 0 && aligned16(a.R) && aligned16(a.dR) &&
                    (a.dy == nullptr || aligned16(a.dy));
   const dim3 tok(static_cast<unsigned>(a.T));
   cudaError_t e;
-  // 2. d_pre.
-  e = vec ? launch_pdl(pre_bwd_dpre_kernel<true>, tok, dim3(kBwThreads), 0, s, a.dy, a.dpre, a.R,
-                       dpt, a.H)
-          : launch_pdl(pre_bwd_dpre_kernel<false>, tok, dim3(kBwThreads), 0, s, a.dy, a.dpre, a.R,
-                       dpt, a.H);
-  if (e != cudaSuccess) return -4;
+  // 2. d_pre (unless the projection formed it).
+  if (!dy_fold) {
+    e = vec ? launch_pdl(pre_bwd_dpre_kernel<true>, tok, dim3(kBwThreads), 0, s, a.dy, a.dpre,
+                         a.R, dpt, a.H)
+            : launch_pdl(pre_bwd_dpre_kernel<false>, tok, dim3(kBwThreads), 0, s, a.dy, a.dpre,
+                         a.R, dpt, a.H);
+    if (e != cudaSuccess) return -4;
+  }
   // 3. Coefficients' reverse pass.
   const FinishParams fp{a.iters, a.sinkhorn_eps, a.rms_eps, a.pre_eps, a.post_mult};
   e = launch_pdl(pre_bwd_coef_kernel, dim3(static_cast<unsigned>((4 * a.T + 255) / 256)),
                  dim3(256), 0, s, static_cast<const float*>(part), nrec,
-                 static_cast<const float*>(dpt), a.dpost, a.dcomb, a.hc_scale, a.hc_base, brec,
+                 static_cast<const float*>(dpt), a.dpre, dy_fold ? 1 : 0, a.dpost, a.dcomb,
+                 a.hc_scale, a.hc_base, brec,
                  a.T, K, fp);
   if (e != cudaSuccess) return -4;
   // 4. d_scale, d_base.
@@ -793,8 +804,8 @@ int launch_pre_backward(const PreBwdArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return -4;
     note_launches(2);
   }
-  // dpre, coef, param, d_R on CUDA cores (the tensor-core forms count their own launches).
-  note_launches(dr == 0 ? 3 : 4);
+  // [dpre], coef, param, [d_R on CUDA cores] (the tensor-core forms count their own launches).
+  note_launches((dy_fold ? 2 : 3) + (dr == 0 ? 0 : 1));
   return 0;
 }
 

@@ -362,9 +362,7 @@ __global__ void __launch_bounds__(kDrThreads, 1)
     uint32_t gph = 0;
     for (int64_t w = lo; w < hi; ++w) {
       const int64_t tt = w / per_tt;
-      const int64_t rem = w - tt * per_tt;
-      const int64_t hc = rem >> 2;
-      const int64_t i = rem & 3;
+      const int64_t i = (w - tt * per_tt) & 3;
       const int64_t g = w >> 2;
       if (g != cur_g) {
         if (cur_g >= 0) {  // this warp is done with the previous group's d_y buffer

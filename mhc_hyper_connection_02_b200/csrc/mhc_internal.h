@@ -190,6 +190,9 @@ size_t pre_tc_workspace_bytes(int64_t T, int64_t H);
 bool pre_tc_supported(int64_t T, int64_t H);
 int launch_pre_tc(const PreArgs& a, cudaStream_t s);
 // The tensor path's split + projection alone: records [nrec][T][32] after the Bw operand.
-int launch_tc_projection(const PreArgs& a, cudaStream_t s, float** part, int* nrec);
+// With dy (the pre-map backward; H % 64 == 0) the records also carry sum_h dy R_i per stream in
+// floats 28..31.
+int launch_tc_projection(const PreArgs& a, cudaStream_t s, float** part, int* nrec,
+                         const uint16_t* dy = nullptr);
 
 }  // namespace mhc

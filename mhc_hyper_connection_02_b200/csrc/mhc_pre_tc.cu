@@ -49,6 +49,13 @@ constexpr int kTcStageBytes = kTcSub * kTcABytes + kTcBBytes;  // 43008 = 42 x 1
 constexpr int kTcThreads = 192;
 constexpr int kTcTmemCols = 512;                   // 2 buffers x 2 sub-tiles x 128 columns
 constexpr int kTcSmem = 1024 + kTcStages * kTcStageBytes + 256;
+// The backward's projection also carries d_y: it walks a tile's K blocks column-block-major (the
+// four streams of a 64-column block consecutively) and keeps the block's d_y tile [256 x 64] in
+// one of two slots for those four stages; three stages.
+constexpr int kTcDyStages = 3;
+constexpr int kTcDyBytes = kTcSub * kTcABytes;  // 32 KB
+constexpr int kTcDySmem = 1024 + kTcDyStages * kTcStageBytes + 2 * kTcDyBytes + 256;
+static_assert(kTcDySmem <= 227 * 1024, "shared memory");
 constexpr int64_t kTcMaxCtas = 148;                // most CTAs the projection plan uses
 constexpr int64_t kTcMinBlocks = 8;                // K blocks per CTA at least (pipeline fill)
 // The tensor-core accumulator is restarted every kTcSubBlocks K blocks of a piece and the sub-piece
@@ -193,28 +200,41 @@ __global__ void __launch_bounds__(256) pre_tc_split_kernel(const float* __restri
     split_hc_fn_row(W, Bw, K, k);
 }
 
+// kDy (the pre-map backward's recomputation): the stages also hold the d_y columns of each K
+// block, and the sum-of-squares warps form d_pre's term sum_h d_y R_i of each token row per stream
+// i, into record floats 28..31 (requires H % 64 == 0, so that a K block lies in one stream).
+template <bool kDy>
 __global__ void __launch_bounds__(kTcThreads, 1) pre_tc_proj_kernel(
     const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmB,
-    float* __restrict__ part, int64_t T, int64_t W, int KB, int S) {
+    const __grid_constant__ CUtensorMap tmDy, float* __restrict__ part, int64_t T, int64_t W,
+    int KB, int S, int64_t H) {
+  constexpr int ST = kDy ? kTcDyStages : kTcStages;
+  constexpr int SB = kTcStageBytes;
+  constexpr int kDyArea = kDy ? 2 * kTcDyBytes : 0;  // d_y slots after the stages
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTcStages * kTcStageBytes);
-  uint64_t* empty = full + kTcStages;
-  uint64_t* afull = empty + kTcStages;  // [2] accumulator buffer b complete (MMA commit)
+  uint8_t* dyslots = smem + ST * SB;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * SB + kDyArea);
+  uint64_t* empty = full + ST;
+  uint64_t* afull = empty + ST;  // [2] accumulator buffer b complete (MMA commit)
   uint64_t* aempty = afull + 2;         // [2] accumulator buffer b read out (4 warps)
   uint64_t* done = aempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
-  static_assert((2 * kTcStages + 5) * 8 + 4 <= 256, "barrier area");
+  static_assert((2 * ST + 5) * 8 + 4 <= 256, "barrier area");
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int64_t P = gridDim.x;
   const int64_t c = blockIdx.x;
   const int64_t lo = c * W / P, hi = (c + 1) * W / P;
+  // kDy: the kb-th block of a tile is stream kb % 4 of column block kb / 4 (KB = 4 H / 64);
+  // otherwise blocks follow k = i H + h.
+  const int hbk = KB / 4;
+  auto pkb = [&](int kb) -> int { return kDy ? (kb & 3) * hbk + (kb >> 2) : kb; };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kTcStages; ++s) {
+    for (int s = 0; s < ST; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1 + 4);  // MMA commit + one arrival per sum-of-squares warp
     }
@@ -241,33 +261,46 @@ __global__ void __launch_bounds__(kTcThreads, 1) pre_tc_proj_kernel(
 
   if (warp == 0) {
     if (lane == 0) {
-      int64_t n = 0;
+      int64_t n = 0, ng = -1;  // ng: d_y groups loaded (kDy)
       bool ok = true;
       for (int64_t u = lo; u < hi && ok;) {
         const int64_t tile = u / KB;
         const int kbs = static_cast<int>(u - tile * KB);
         const int kbe = static_cast<int>(min(static_cast<int64_t>(KB), kbs + (hi - u)));
         for (int kb = kbs; kb < kbe; ++kb, ++n) {
-          const int s = static_cast<int>(n % kTcStages);
-          const uint32_t ph = static_cast<uint32_t>(n / kTcStages) & 1u;
-          if (n >= kTcStages && !mbar_wait(&empty[s], ph ^ 1u, 10)) {
+          const int s = static_cast<int>(n % ST);
+          const uint32_t ph = static_cast<uint32_t>(n / ST) & 1u;
+          if (n >= ST && !mbar_wait(&empty[s], ph ^ 1u, 10)) {
             ok = false;
             break;
           }
-          uint8_t* st = smem + s * kTcStageBytes;
-          mbar_arrive_expect_tx(&full[s], kTcStageBytes);
+          uint8_t* st = smem + s * SB;
+          // kDy: a block that opens a column block (or a piece) also brings that column block's
+          // d_y tile, into the slot the group after next will reuse (by then the sum-of-squares
+          // warps are past this group: the ring is shorter than a group).
+          const bool newg = kDy && ((kb & 3) == 0 || kb == kbs);
+          if (newg) ++ng;
+          mbar_arrive_expect_tx(&full[s], SB + (newg ? kTcDyBytes : 0));
+          const int x = pkb(kb) * kTcKB;
 #pragma unroll
           for (int v = 0; v < kTcSub; ++v)
-            tma_load_2d(st + v * kTcABytes, &tmR, kb * kTcKB,
+            tma_load_2d(st + v * kTcABytes, &tmR, x,
                         static_cast<int>(tile * kTcTile + v * kTcM), &full[s]);
-          tma_load_2d(st + kTcSub * kTcABytes, &tmB, kb * kTcKB, 0, &full[s]);
+          tma_load_2d(st + kTcSub * kTcABytes, &tmB, x, 0, &full[s]);
+          if (newg) {
+            uint8_t* ds = dyslots + (ng & 1) * kTcDyBytes;
+#pragma unroll
+            for (int v = 0; v < kTcSub; ++v)
+              tma_load_2d(ds + v * kTcABytes, &tmDy, (kb >> 2) * kTcKB,
+                          static_cast<int>(tile * kTcTile + v * kTcM), &full[s]);
+          }
         }
         u += kbe - kbs;
       }
       if (!ok) {  // do not leave while copies into shared memory are in flight
-        for (int64_t i = n - kTcStages; i < n; ++i)
+        for (int64_t i = n - ST; i < n; ++i)
           if (i >= 0)
-            mbar_wait(&full[i % kTcStages], static_cast<uint32_t>(i / kTcStages) & 1u, 15);
+            mbar_wait(&full[i % ST], static_cast<uint32_t>(i / ST) & 1u, 15);
       }
     }
   } else if (warp == 1) {
@@ -291,14 +324,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) pre_tc_proj_kernel(
             tc_fence_after();
             dt = tmem + static_cast<uint32_t>(b * kTcSub * kTcM);
           }
-          const int s = static_cast<int>(n % kTcStages);
-          const uint32_t ph = static_cast<uint32_t>(n / kTcStages) & 1u;
+          const int s = static_cast<int>(n % ST);
+          const uint32_t ph = static_cast<uint32_t>(n / ST) & 1u;
           if (!mbar_wait(&full[s], ph, 11)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a = smem_u32(smem + s * kTcStageBytes);
+          const uint32_t a = smem_u32(smem + s * SB);
           const uint64_t bdesc = sw128_desc(a + kTcSub * kTcABytes);
 #pragma unroll
           for (int v = 0; v < kTcSub; ++v) {
@@ -325,7 +358,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) pre_tc_proj_kernel(
     // accumulator; the same thread sums the squares of those rows (one per sub-tile).
     const int q_lane = warp & 3;
     const int row = q_lane * 32 + lane;
-    int64_t n = 0;
+    int64_t n = 0, ng = -1;  // ng: d_y groups seen (kDy), as the producer counts them
     int64_t sp = 0;     // sub-pieces the MMA warp has been asked to finish
     int64_t pend = -1;  // finished sub-piece whose accumulators are not yet added
     bool ok = true;
@@ -362,38 +395,60 @@ __global__ void __launch_bounds__(kTcThreads, 1) pre_tc_proj_kernel(
       const int kbs = static_cast<int>(u - tile * KB);
       const int kbe = static_cast<int>(min(static_cast<int64_t>(KB), kbs + (hi - u)));
       float ss0[kTcSub], ss1[kTcSub];
+      float dpv[kTcSub][4];  // kDy: sum_h d_y R_i of the row, per stream i
 #pragma unroll
       for (int v = 0; v < kTcSub; ++v) {
         ss0[v] = ss1[v] = 0.f;
 #pragma unroll
         for (int j = 0; j < kMix; ++j) racc[v][j] = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dpv[v][i] = 0.f;
       }
       for (int kb = kbs; kb < kbe; ++kb, ++n) {
-        const int s = static_cast<int>(n % kTcStages);
-        const uint32_t ph = static_cast<uint32_t>(n / kTcStages) & 1u;
+        const int s = static_cast<int>(n % ST);
+        const uint32_t ph = static_cast<uint32_t>(n / ST) & 1u;
         // Every lane waits; the warp continues only if all of them saw the stage (warp-uniform,
         // so the __syncwarp and the .sync.aligned TMEM loads below are never reached divergently).
         if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, 12))) {
           ok = false;
           break;
         }
+        if (kDy && ((kb & 3) == 0 || kb == kbs)) ++ng;  // this block's d_y slot: ng & 1
 #pragma unroll
         for (int v = 0; v < kTcSub; ++v) {
           // Row `row` of the swizzled tile is its own 128 contiguous bytes (chunks permuted within
           // it), and a sum does not depend on element order. Each lane starts at a different
-          // 16-byte chunk, so the 8 lanes of a load phase hit 8 different bank groups.
-          const uint4* rp = reinterpret_cast<const uint4*>(smem + s * kTcStageBytes +
+          // 16-byte chunk, so the 8 lanes of a load phase hit 8 different bank groups. The d_y
+          // tile has the same geometry and swizzle, so chunk c of both rows holds the same columns.
+          const uint4* rp = reinterpret_cast<const uint4*>(smem + s * SB +
                                                            v * kTcABytes + row * 128);
+          float dsum = 0.f;
 #pragma unroll
           for (int cc = 0; cc < 8; ++cc) {
             const uint4 w = rp[cc ^ (lane & 7)];
             const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+            uint32_t g4[4] = {0u, 0u, 0u, 0u};
+            if constexpr (kDy) {
+              const uint4 g = reinterpret_cast<const uint4*>(
+                  dyslots + (ng & 1) * kTcDyBytes + v * kTcABytes + row * 128)[cc ^ (lane & 7)];
+              g4[0] = g.x, g4[1] = g.y, g4[2] = g.z, g4[3] = g.w;
+            }
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float x0 = bf16_lo(w4[e]), x1 = bf16_hi(w4[e]);
               ss0[v] = fmaf(x0, x0, ss0[v]);
               ss1[v] = fmaf(x1, x1, ss1[v]);
+              if constexpr (kDy) {
+                dsum = fmaf(bf16_lo(g4[e]), x0, dsum);
+                dsum = fmaf(bf16_hi(g4[e]), x1, dsum);
+              }
             }
+          }
+          if constexpr (kDy) {
+            const int si = kb & 3;  // the block's stream
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              if (si == i) dpv[v][i] += dsum;
           }
         }
         __syncwarp();
@@ -431,12 +486,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) pre_tc_proj_kernel(
             rec[w] = make_float4(racc[v][4 * w], racc[v][4 * w + 1], racc[v][4 * w + 2],
                                  racc[v][4 * w + 3]);
           rec[6] = make_float4(ss0[v] + ss1[v], 0.f, 0.f, 0.f);
+          if constexpr (kDy) rec[7] = make_float4(dpv[v][0], dpv[v][1], dpv[v][2], dpv[v][3]);
           if (last_piece) {
             const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
             for (int64_t sl = slot + 1; sl < S; ++sl) {
               float4* zr = reinterpret_cast<float4*>(part + (sl * T + t) * 32);
 #pragma unroll
-              for (int w = 0; w < 7; ++w) zr[w] = z;
+              for (int w = 0; w < (kDy ? 8 : 7); ++w) zr[w] = z;
             }
           }
         }
@@ -636,17 +692,22 @@ static bool make_map(CUtensorMap* m, const void* base, int64_t cols, int64_t row
 
 // Split + projection: records [S][T][32] (raw[24], ss) in the workspace after Bw. Returns 0 or a
 // negative MHC_ERR_* code; *part_out / *nrec_out receive the records and their slot count.
-int launch_tc_projection(const PreArgs& a, cudaStream_t s, float** part_out, int* nrec_out) {
+int launch_tc_projection(const PreArgs& a, cudaStream_t s, float** part_out, int* nrec_out,
+                         const uint16_t* dy) {
   const TcPlan plan = tc_plan(a.T, a.H, device_sm_count());
   const int64_t K = 4 * a.H;
   uint8_t* ws = static_cast<uint8_t*>(a.workspace);
   uint16_t* Bw = reinterpret_cast<uint16_t*>(ws);
   float* part = reinterpret_cast<float*>(ws + plan.bw_bytes);
 
-  CUtensorMap mR, mB;
+  CUtensorMap mR, mB, mDy;
   if (!make_map(&mR, a.R, K, a.T, kTcM) || !make_map(&mB, Bw, K, kTcN, kTcN)) return -4;
+  if (dy != nullptr && !make_map(&mDy, dy, a.H, a.T, kTcM)) return -4;
+  if (dy == nullptr) mDy = mR;  // unused by the form without d_y
 
-  if (!ensure_smem_limit(reinterpret_cast<const void*>(pre_tc_proj_kernel), kTcSmem)) return -4;
+  if (!ensure_smem_limit(reinterpret_cast<const void*>(pre_tc_proj_kernel<false>), kTcSmem) ||
+      !ensure_smem_limit(reinterpret_cast<const void*>(pre_tc_proj_kernel<true>), kTcDySmem))
+    return -4;
 
   const int64_t sb = (K + 255) / 256;
   const int split_blocks = static_cast<int>(sb < 4096 ? sb : 4096);
@@ -655,10 +716,15 @@ int launch_tc_projection(const PreArgs& a, cudaStream_t s, float** part_out, int
     return -4;
   note_launches(1);
 
-  if (launch_pdl(pre_tc_proj_kernel, dim3(static_cast<unsigned>(plan.P)), dim3(kTcThreads),
-                 static_cast<size_t>(kTcSmem), s, mR, mB, part, a.T, plan.W,
-                 static_cast<int>(plan.kblocks), static_cast<int>(plan.S)) != cudaSuccess)
-    return -4;
+  const cudaError_t e =
+      dy != nullptr
+          ? launch_pdl(pre_tc_proj_kernel<true>, dim3(static_cast<unsigned>(plan.P)),
+                       dim3(kTcThreads), static_cast<size_t>(kTcDySmem), s, mR, mB, mDy, part,
+                       a.T, plan.W, static_cast<int>(plan.kblocks), static_cast<int>(plan.S), a.H)
+          : launch_pdl(pre_tc_proj_kernel<false>, dim3(static_cast<unsigned>(plan.P)),
+                       dim3(kTcThreads), static_cast<size_t>(kTcSmem), s, mR, mB, mDy, part,
+                       a.T, plan.W, static_cast<int>(plan.kblocks), static_cast<int>(plan.S), a.H);
+  if (e != cudaSuccess) return -4;
   note_launches(1);
   *part_out = part;
   *nrec_out = static_cast<int>(plan.S);

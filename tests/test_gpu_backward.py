@@ -105,15 +105,16 @@ def test_pre_backward(T, H):
     _check_sum(db.cpu().numpy(), rb, np.abs(pt["dl"]).sum(0), 1e-4, "d_base")
 
 
-@pytest.mark.parametrize("T,H,dr_tensor,dw_tensor", [(300, 2048, True, True),
-                                                    (130, 1000, False, False),
-                                                    (200, 1056, False, True)])
-def test_pre_backward_d_R_form(T, H, dr_tensor, dw_tensor):
+@pytest.mark.parametrize("T,H,dr_tensor,dw_tensor,dy_fold", [(300, 2048, True, True, True),
+                                                            (130, 1000, False, False, False),
+                                                            (200, 1056, False, True, False)])
+def test_pre_backward_d_R_form(T, H, dr_tensor, dw_tensor, dy_fold):
     """H % 128 == 0 with d_y given takes the tcgen05 d_R (split operands + the tensor kernel: two
     launches), otherwise the CUDA-core kernel (one); 4H % 128 == 0 takes the tcgen05 d_hc_fn
     (transposed d_raw split, the tensor kernel, the partials' sum: three launches), otherwise
-    CUDA-core partials and their sum (two). Both projections here are the tensor form (split +
-    projection); then d_pre, coefficients and parameters."""
+    CUDA-core partials and their sum (two). The projections here are the tensor form (split +
+    projection); with H % 64 == 0 it also forms d_pre's d_y term, otherwise a d_pre kernel runs;
+    then coefficients and parameters."""
     w, d_y, d_pre, d_post, d_comb = _pre_case(T, H, seed=11)
     n0 = mhc.launch_count()
     mhc.pre_backward(dev_bf16(w.R), dev_f32(w.hc_fn), dev_f32(w.hc_scale), dev_f32(w.hc_base),
@@ -121,7 +122,8 @@ def test_pre_backward_d_R_form(T, H, dr_tensor, dw_tensor):
                      d_comb=dev_f32(d_comb), params=mhc.make_params(iters=w.iters))
     torch.cuda.synchronize()
     assert mhc.device_status() == 0
-    assert mhc.launch_count() - n0 == 2 + 3 + (2 if dr_tensor else 1) + (3 if dw_tensor else 2)
+    assert mhc.launch_count() - n0 == (2 + (2 if dy_fold else 3) + (2 if dr_tensor else 1) +
+                                       (3 if dw_tensor else 2))
 
 
 def test_pre_backward_optional_gradients_and_tensor_path():
