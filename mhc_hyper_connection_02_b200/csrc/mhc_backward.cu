@@ -243,20 +243,25 @@ __device__ __forceinline__ float quad_sum(float v) {
 }
 
 // One Sinkhorn round on the quad's 4x4 (lane r holds row r): row normalisation then column
-// normalisation by plain sums; returns B (after the row step), rs and cs (the normalisers) for the
-// reverse pass.
-__device__ __forceinline__ void sk_round(float (&a)[4], float (&b)[4], float& rs, float (&cs)[4]) {
-  rs = ((a[0] + a[1]) + a[2]) + a[3];
+// normalisation by plain sums, with the forward's arithmetic (sinkhorn_quad: multiplication by
+// recip_nr of the sum, column sums (a0 + a1) + (a2 + a3) across the quad), so the recomputed
+// states are the forward's bit for bit; returns B (after the row step) and the reciprocals of the
+// normalisers for the reverse pass.
+__device__ __forceinline__ void sk_round(float (&a)[4], float (&b)[4], float& rrs,
+                                         float (&rcs)[4]) {
+  rrs = recip_nr(((a[0] + a[1]) + a[2]) + a[3]);
 #pragma unroll
-  for (int n = 0; n < 4; ++n) b[n] = a[n] / rs;
+  for (int n = 0; n < 4; ++n) b[n] = a[n] * rrs;
 #pragma unroll
   for (int n = 0; n < 4; ++n) {
-    cs[n] = quad_sum(b[n]);
-    a[n] = b[n] / cs[n];
+    float c = b[n] + __shfl_xor_sync(0xffffffffu, b[n], 1);
+    c = c + __shfl_xor_sync(0xffffffffu, c, 2);
+    rcs[n] = recip_nr(c);
+    a[n] = b[n] * rcs[n];
   }
 }
 
-constexpr int kSkCk = 16;  // Sinkhorn forward checkpoints kept by the reverse pass
+constexpr int kSkCk = 32;  // Sinkhorn forward checkpoints kept by the reverse pass (every round up to 32)
 
 // Per token, one lane quad (lane r: pre r, post r, comb row r). Writes the backward record
 // brec[t][64]: [0..23] d_raw, [24] d_ss, [25..28] pre gates, [29..31] the token's terms of
@@ -303,43 +308,43 @@ __global__ void __launch_bounds__(256) pre_bwd_coef_kernel(
   // are checkpointed every G rounds (at most kSkCk checkpoints); the state entering round k is
   // recomputed from the checkpoint at or before it, by the same operations as the forward, so it
   // is the forward's state exactly.
-  float p[4], dA[4];
+  float p[4], a0[4], dA[4];
   {
     const float mx = fmaxf(fmaxf(lc[0], lc[1]), fmaxf(lc[2], lc[3]));
+    float e[4];
 #pragma unroll
-    for (int n = 0; n < 4; ++n) p[n] = expf(lc[n] - mx);
-    const float es = ((p[0] + p[1]) + p[2]) + p[3];
+    for (int n = 0; n < 4; ++n) e[n] = expf(lc[n] - mx);
+    const float res = recip_nr(((e[0] + e[1]) + e[2]) + e[3]);
 #pragma unroll
     for (int n = 0; n < 4; ++n) {
-      p[n] = p[n] / es;
+      p[n] = e[n] * res;
+      a0[n] = fmaf(e[n], res, fp.sinkhorn_eps);  // as the forward forms A0
       dA[n] = dcomb ? dcomb[tt * 16 + 4 * r + n] : 0.f;
     }
   }
   const int G = (fp.iters + kSkCk - 1) / kSkCk;
   float ck[kSkCk][4];
   {
-    float a[4] = {p[0] + fp.sinkhorn_eps, p[1] + fp.sinkhorn_eps, p[2] + fp.sinkhorn_eps,
-                  p[3] + fp.sinkhorn_eps},
-          b[4], rs, cs[4];
+    float a[4] = {a0[0], a0[1], a0[2], a0[3]}, b[4], rrs, rcs[4];
     for (int k = 0; k < fp.iters; ++k) {
       if (k % G == 0) {
 #pragma unroll
         for (int n = 0; n < 4; ++n) ck[k / G][n] = a[n];
       }
-      sk_round(a, b, rs, cs);
+      sk_round(a, b, rrs, rcs);
     }
   }
   for (int k = fp.iters - 1; k >= 0; --k) {
     const int c = k / G;
-    float a[4] = {ck[c][0], ck[c][1], ck[c][2], ck[c][3]}, b[4], rs, cs[4];
-    for (int j = c * G; j < k; ++j) sk_round(a, b, rs, cs);
-    sk_round(a, b, rs, cs);  // round k: a is now C
+    float a[4] = {ck[c][0], ck[c][1], ck[c][2], ck[c][3]}, b[4], rrs, rcs[4];
+    for (int j = c * G; j < k; ++j) sk_round(a, b, rrs, rcs);
+    sk_round(a, b, rrs, rcs);  // round k: a is now C
     float dB[4];
 #pragma unroll
-    for (int n = 0; n < 4; ++n) dB[n] = (dA[n] - quad_sum(dA[n] * a[n])) / cs[n];
+    for (int n = 0; n < 4; ++n) dB[n] = (dA[n] - quad_sum(dA[n] * a[n])) * rcs[n];
     const float rdot = ((dB[0] * b[0] + dB[1] * b[1]) + dB[2] * b[2]) + dB[3] * b[3];
 #pragma unroll
-    for (int n = 0; n < 4; ++n) dA[n] = (dB[n] - rdot) / rs;
+    for (int n = 0; n < 4; ++n) dA[n] = (dB[n] - rdot) * rrs;
   }
   // Softmax: d_l = P (dA0 - sum_n dA0 P) along the row.
   float dlc[4];
