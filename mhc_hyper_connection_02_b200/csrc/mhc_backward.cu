@@ -699,7 +699,7 @@ static BwPlan bw_plan(int64_t T, int64_t H) {
   p.tchunk = ((T + nchunk - 1) / nchunk + kDwTok - 1) / kDwTok * kDwTok;
   p.nchunk = static_cast<int>((T + p.tchunk - 1) / p.tchunk);
   p.dwp = up(static_cast<size_t>(p.nchunk) * 4 * H * kMix * 4);
-  p.drtc = up(pre_bwd_dr_tc_workspace_bytes(T, H));  // split operands of the tensor-core d_R
+  p.drtc = up(pre_bwd_dr_tc_workspace_bytes(T, H));  // operands + partials of d_R with d_hc_fn
   p.dwtc = up(pre_bwd_dw_tc_workspace_bytes(T, H));  // B operand and partials of its d_hc_fn
   p.total = p.proj + p.dpt + p.brec + p.dwp + p.drtc + p.dwtc;
   return p;
@@ -760,12 +760,13 @@ int launch_pre_backward(const PreBwdArgs& a, cudaStream_t s) {
   e = launch_pdl(pre_bwd_param_kernel, dim3(3 + kMix), dim3(256), 0, s,
                  static_cast<const float*>(brec), a.dscale, a.dbase, a.T);
   if (e != cudaSuccess) return -4;
-  // 5. d_R: on tensor cores where the shape allows (1: not this shape, nothing launched), else
-  // column slices x token chunks on CUDA cores, one wave of kDxSlotsPerSm CTAs per SM.
+  // 5. d_R: on tensor cores where the shape allows, together with d_hc_fn (1: not this shape,
+  // nothing launched), else column slices x token chunks on CUDA cores, one wave of
+  // kDxSlotsPerSm CTAs per SM.
   int dr = 1;
   if (vec && a.dy != nullptr) {
     dr = launch_pre_bwd_dr_tc(a.R, a.dy, a.hc_fn, static_cast<const float*>(brec), kBrec, a.dR,
-                              drtc_ws, a.T, a.H, s);
+                              a.dW, drtc_ws, a.T, a.H, s);
     if (dr < 0) return dr;
   }
   if (dr == 0) {
@@ -788,11 +789,15 @@ int launch_pre_backward(const PreBwdArgs& a, cudaStream_t s) {
                    a.R, a.dy, a.hc_fn, static_cast<const float*>(brec), a.dR, a.T, a.H);
   }
   if (e != cudaSuccess) return -4;
-  // 6. d_hc_fn: on tensor cores where 4H % 128 == 0 (1: not this shape, nothing launched), else
-  // CUDA-core partials over token chunks; then the partials' in-order sum.
-  int dwr = launch_pre_bwd_dw_tc(a.R, static_cast<const float*>(brec), kBrec, a.dW, dwtc_ws, a.T,
-                                 a.H, s);
-  if (dwr < 0) return dwr;
+  // 6. d_hc_fn (unless step 5 formed it): on tensor cores where 4H % 128 == 0 (1: not this
+  // shape, nothing launched), else CUDA-core partials over token chunks; then the partials'
+  // in-order sum.
+  int dwr = 0;
+  if (dr != 0) {
+    dwr = launch_pre_bwd_dw_tc(a.R, static_cast<const float*>(brec), kBrec, a.dW, dwtc_ws, a.T,
+                               a.H, s);
+    if (dwr < 0) return dwr;
+  }
   if (dwr == 1) {
     const dim3 gw(static_cast<unsigned>((K + kDwCols - 1) / kDwCols),
                   static_cast<unsigned>(plan.nchunk));

@@ -1,29 +1,41 @@
-// Pre-map backward, d_R on tcgen05 tensor cores.
+// Pre-map backward, d_R and d_hc_fn on tcgen05 tensor cores, in one pass over R.
 //
 // d_R[t][k] = sum_j d_raw[t][j] hc_fn[k][j] + 2 R[t][k] d_ss[t] + pre_i[t] d_y[t][h], k = i*H + h
+// d_hc_fn[k][j] = sum_t R[t][k] d_raw[t][j]
 // (the chain rule through raw = R_flat . hc_fn, the sum of squares and y = sum_i pre_i R_i;
-// "FlashInfer mHC module deep dive" §3.4 / §5.2 forward). The contraction has inner dimension 24:
-// on CUDA cores that is 24 FMAs per element of d_R and the kernel is bound by issue; on tensor
-// cores it is bound by its traffic (R and d_y read, d_R written).
+// "FlashInfer mHC module deep dive" §3.4 / §5.2 forward). Both contractions have 24 as one
+// dimension: on CUDA cores they are bound by issue; on tensor cores the kernel is bound by its
+// traffic (R and d_y read once, d_R written).
 //
-// Operands (written by pre_bwd_split_kernel, bf16, 128 columns per row, zero past 72; the MMAs
-// read columns 0..79: four K=16 steps in a 128-byte-swizzled box, one in a 32-byte-swizzled box):
-//   A[t] = [hi(d_raw) | hi(d_raw) | lo(d_raw)],  B[k] = [hi(w) | lo(w) | hi(w)],  w = hc_fn[k][.]
-// so A.B = hi.hi + hi.lo + lo.hi of each product, exact in the fp32 accumulator; the dropped
-// lo.lo term and the split's remainders are below 2^-15 of each product.
+// Operands (written by pre_bwd_split_kernel, bf16, 128 columns per row, zero past 72; the d_R
+// MMAs read columns 0..79: four K=16 steps in a 128-byte-swizzled box, one in a 32-byte-swizzled
+// box):
+//   A[t] = [hi(d_raw) | lo(d_raw) | hi(d_raw)],  B[k] = [hi(w) | hi(w) | lo(w)],  w = hc_fn[k][.]
+// so A.B = hi.hi + lo.hi + hi.lo of each product, exact in the fp32 accumulator; the dropped
+// lo.lo term and the split's remainders are below 2^-15 of each product. The first 48 columns of
+// A, [hi | lo] of d_raw, are also d_hc_fn's B operand (read MN-major: tokens along K), with R's
+// staged tile as its A operand (MN-major: 128 columns k along M), so each d_hc_fn product is
+// R.hi + R.lo, exact in fp32 (R is exact in bf16; hi + lo leaves below 2^-16 of d_raw).
 //
-// pre_bwd_dr_kernel: persistent, one CTA per SM. Work items (token tile tt of 128, column block
-// hc of 128 columns within a stream, stream i), numbered with i fastest, so the four items of a
-// (tt, hc) group share one d_y tile; the list is cut into equal contiguous ranges, one per CTA.
-//   warp 0      TMA: A of the token tile (32 KB, reloaded when the tile changes), the group's d_y
-//               tile (two buffers), and per item the R tile and the B tile (rings of two: an R
-//               slot is free once its d_R has been stored, a B slot once its MMAs have read it);
-//               all [128 x 64] boxes with the 128-byte swizzle.
-//   warp 1      tcgen05.mma M=128 N=128 K=16, five steps (K columns 0..79), into one of two TMEM
-//               accumulators.
+// pre_bwd_drw_kernel: persistent, one CTA per SM. Work items (column block hc of 128 columns
+// within a stream, token tile tt of 128, stream i), numbered with i fastest, so the four items of
+// an (hc, tt) group share one d_y tile and one A tile; the list is cut into equal contiguous
+// ranges, one per CTA. A unit is (hc, chunk of kDrwChunk token tiles); a CTA's items inside one
+// unit form a piece, whose rank among the unit's CTAs is its partial slot.
+//   warp 0      TMA: the group's d_y tile (two buffers), and per item the R tile and the B tile
+//               (rings of three and two: an R slot is free once its d_R has been stored, a B slot
+//               once its MMAs have read it); all [128 x 64] boxes with the 128-byte swizzle.
+//   warp 1      tcgen05.mma: per item, eight M=128 N=64 K=16 steps of d_hc_fn into stream i's
+//               accumulator (restarted at the piece's first item of that stream), then five
+//               M=128 N=128 K=16 steps of d_R into one of two accumulators (TMEM: 2 x 128 + 4 x
+//               64 columns). It also loads the A tile, once the MMAs on the previous one are done.
 //   warps 2-5   epilogue, thread = token row (its TMEM lane): 64 accumulator columns at a time
 //               (tcgen05.ld), R and d_y from the staged tiles, out = bf16_rn(fma(pre_i, d_y,
-//               fma(2 d_ss, R, acc))) written over R in place.
+//               fma(2 d_ss, R, acc))) written over R in place (after the item's MMAs, which read
+//               R, have completed). At a piece's end, thread = column k: the partial
+//               [ck * S + slot][k][24] = lo + hi columns of each stream's accumulator (zero for a
+//               stream the piece did not reach); the CTA holding a unit's last item zero-fills its
+//               unused slots. pre_bwd_dw_sum_kernel adds the slices in order.
 //   warp 6      stores each finished d_R tile with a TMA bulk-tensor store and releases its R slot
 //               once the store has read it (the epilogue warps go on to the next item meanwhile).
 // Every wait is bounded; copies in flight are drained and stores completed before exit.
@@ -55,7 +67,16 @@ constexpr int kDrOffR = kDrOffB + kDrBSlots * kDrOpTile;
 constexpr int kDrOffBars = kDrOffR + kDrRSlots * kDrTile;  // 225280
 constexpr int kDrSmem = 1024 + kDrOffBars + 256;
 constexpr int kDrThreads = 224;
-constexpr int kDrTmemCols = 256;
+constexpr int kDrTmemCols = 512;
+// d_hc_fn: accumulators of the four streams at columns 256 + 64 i (N = 64: split columns
+// [hi | lo | hi(0..15)] of d_raw; the last 16 are not read), restarted every kDrwChunk token tiles.
+constexpr int kDrwN = 64;
+constexpr int kDrwCol0 = 2 * 128;
+constexpr int kDrwChunk = 64;
+// kind::f16, D fp32, A and B bf16, both MN-major (bits 15, 16), N = 64, M = 128.
+constexpr uint32_t kDrwIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
+                               (static_cast<uint32_t>(kDrwN >> 3) << 17) |
+                               (static_cast<uint32_t>(128 >> 4) << 24);
 constexpr uint32_t kDrIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
                               (static_cast<uint32_t>(kDrN >> 3) << 17) |
                               (static_cast<uint32_t>(kDrM >> 4) << 24);
@@ -65,10 +86,34 @@ bool pre_bwd_dr_tc_supported(int64_t T, int64_t H) {
   return T >= 1 && H >= 128 && H % 128 == 0 && (T + kDrM - 1) / kDrM <= (int64_t(1) << 24);
 }
 
+// Work plan: W items over P CTAs; S = most CTAs one unit meets (a unit holds at most
+// min(ntt, kDrwChunk) * 4 consecutive items and a range at least floor(W / P)).
+struct DrPlan {
+  int64_t ntt, nhc, W, nck, P, S;
+};
+
+static DrPlan dr_plan(int64_t T, int64_t H, int64_t sms) {
+  DrPlan p;
+  p.ntt = (T + kDrM - 1) / kDrM;
+  p.nhc = H / kDrN;
+  p.W = p.ntt * p.nhc * 4;
+  p.nck = (p.ntt + kDrwChunk - 1) / kDrwChunk;
+  p.P = sms < 148 ? sms : 148;
+  if (p.P > p.W) p.P = p.W;
+  if (p.P < 1) p.P = 1;
+  const int64_t per_unit = (p.ntt < kDrwChunk ? p.ntt : kDrwChunk) * 4;
+  p.S = per_unit * p.P / p.W + 2;
+  if (p.S > p.P) p.S = p.P;
+  return p;
+}
+
+// A and B operands, then the d_hc_fn partials (a plan over fewer SMs never needs more slots).
 size_t pre_bwd_dr_tc_workspace_bytes(int64_t T, int64_t H) {
   if (!pre_bwd_dr_tc_supported(T, H)) return 0;
   auto up = [](size_t v) { return (v + 1023) / 1024 * 1024; };
-  return up(static_cast<size_t>(T) * kDrKd * 2) + up(static_cast<size_t>(4 * H) * kDrKd * 2);
+  const DrPlan p = dr_plan(T, H, 148);
+  return up(static_cast<size_t>(T) * kDrKd * 2) + up(static_cast<size_t>(4 * H) * kDrKd * 2) +
+         up(static_cast<size_t>(p.nck * p.S) * static_cast<size_t>(4 * H) * kMix * 4);
 }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -110,7 +155,7 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int 
       : "memory");
 }
 
-// A[t] = [hi | hi | lo] of d_raw (backward record floats 0..23), B[k] = [hi | lo | hi] of
+// A[t] = [hi | lo | hi] of d_raw (backward record floats 0..23), B[k] = [hi | hi | lo] of
 // hc_fn[k]; columns 72..127 zero. One thread per row, 16-byte stores.
 __global__ void __launch_bounds__(256) pre_bwd_split_kernel(const float* __restrict__ brec,
                                                             const float* __restrict__ W,
@@ -141,8 +186,8 @@ __global__ void __launch_bounds__(256) pre_bwd_split_kernel(const float* __restr
         const int grp = col / kMix, j = col - grp * kMix;
         e[u] = col >= 3 * kMix ? 0
                : grp == 0       ? hi[j]
-               : grp == 1       ? (is_a ? hi[j] : lo[j])
-                                : (is_a ? lo[j] : hi[j]);
+               : grp == 1       ? (is_a ? lo[j] : hi[j])
+                                : (is_a ? hi[j] : lo[j]);
       }
       row[c] = static_cast<uint32_t>(e[0]) | (static_cast<uint32_t>(e[1]) << 16);
     }
@@ -155,15 +200,55 @@ __global__ void __launch_bounds__(256) pre_bwd_split_kernel(const float* __restr
 
 struct DrArgs {
   const float* brec;
-  int64_t T, H, ntt, nhc, W;
-  int rec_stride;
+  float* dwp;  // d_hc_fn partials [nck * S][4H][24]
+  int64_t T, H, ntt, nhc, W, nck;
+  int rec_stride, S;
 };
 
+// Item w of the flattened list: chunk ck of kDrwChunk token tiles (slowest), column block hc,
+// token tile tt, stream i (fastest). The unit (ck, hc) is the run of items whose d_hc_fn products
+// share a partial slice; u0, u1 are its first and last items.
+struct DrwItem {
+  int64_t hc, tt, i, ck, u0, u1;
+};
+__host__ __device__ __forceinline__ DrwItem drw_item(const DrArgs& a, int64_t w) {
+  DrwItem r;
+  const int64_t per_ck = a.nhc * kDrwChunk * 4;  // items of a full chunk
+  r.ck = w / per_ck;
+  const int64_t t0 = r.ck * kDrwChunk;           // the chunk's first token tile
+  const int64_t ct = a.ntt - t0 < kDrwChunk ? a.ntt - t0 : kDrwChunk;
+  const int64_t rem = w - r.ck * per_ck;
+  r.hc = rem / (ct * 4);
+  const int64_t rem2 = rem - r.hc * ct * 4;
+  r.tt = t0 + (rem2 >> 2);
+  r.i = rem2 & 3;
+  r.u0 = r.ck * per_ck + r.hc * ct * 4;
+  r.u1 = r.u0 + ct * 4 - 1;
+  return r;
+}
+
+// MN-major, 128-byte swizzle: the next 64-element atom along M (or N) one 16 KB box on (leading
+// byte offset), the next 8 tokens 1 KB on (stride byte offset).
+__device__ __forceinline__ uint64_t drw_mn_desc(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) |
+         (static_cast<uint64_t>(kDrAtom >> 4) << 16) | (static_cast<uint64_t>(1024 >> 4) << 32) |
+         (static_cast<uint64_t>(1) << 46) | (static_cast<uint64_t>(2) << 61);
+}
+
+__device__ __forceinline__ void drw_umma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(kDrwIdesc), "r"(accumulate)
+      : "memory");
+}
+
 __global__ void __launch_bounds__(kDrThreads, 1)
-    pre_bwd_dr_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      const __grid_constant__ CUtensorMap tmA16, const __grid_constant__ CUtensorMap tmB16,
-                      const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmDy,
-                      const __grid_constant__ CUtensorMap tmDR, const DrArgs a) {
+    pre_bwd_drw_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                       const __grid_constant__ CUtensorMap tmA16, const __grid_constant__ CUtensorMap tmB16,
+                       const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmDy,
+                       const __grid_constant__ CUtensorMap tmDR, const DrArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
@@ -174,24 +259,24 @@ __global__ void __launch_bounds__(kDrThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kDrOffBars);
   uint64_t* rfull = bars;          // [3] R tile landed
   uint64_t* rempty = bars + 3;     // [3] d_R stored from the slot (the store has read it)
-  uint64_t* afull = bars + 6;      // [2] accumulator ready
-  uint64_t* aempty = bars + 8;     // [2] accumulator read out (4 warps)
+  uint64_t* afull = bars + 6;      // [2] d_R accumulator ready (and the item's d_hc_fn MMAs done)
+  uint64_t* aempty = bars + 8;     // [2] d_R accumulator read out (4 warps)
   uint64_t* dyfull = bars + 10;    // [2] d_y buffer landed
   uint64_t* dyempty = bars + 12;   // [2] d_y buffer's group finished (4 warps)
   uint64_t* abar = bars + 14;      // A landed
-  uint64_t* afree = bars + 15;     // MMAs on the previous A finished
-  uint64_t* adone = bars + 16;     // MMA warp's own commit point
-  uint64_t* done = bars + 17;
-  uint64_t* bfull = bars + 18;     // [2] B landed
-  uint64_t* bempty = bars + 20;    // [2] MMAs on B finished
-  uint64_t* drready = bars + 22;   // [2] d_R tile of an R slot written (4 warps)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
+  uint64_t* adone = bars + 15;     // MMAs on the current A finished
+  uint64_t* done = bars + 16;
+  uint64_t* bfull = bars + 17;     // [2] B landed
+  uint64_t* bempty = bars + 19;    // [2] MMAs on B finished
+  uint64_t* drready = bars + 21;   // [3] d_R tile of an R slot written (4 warps)
+  uint64_t* wfull = bars + 24;     // d_hc_fn accumulators of a piece complete
+  uint64_t* wempty = bars + 25;    // d_hc_fn accumulators read out (4 warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 26);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int64_t P = gridDim.x;
   const int64_t lo = blockIdx.x * a.W / P, hi = (blockIdx.x + 1) * a.W / P;
-  const int64_t per_tt = a.nhc * 4;
 
   if (threadIdx.x == 0) {
     for (int r = 0; r < kDrRSlots; ++r) {
@@ -210,9 +295,10 @@ __global__ void __launch_bounds__(kDrThreads, 1)
       mbar_init(&dyempty[b], 4);
     }
     mbar_init(abar, 1);
-    mbar_init(afree, 1);
     mbar_init(adone, 1);
     mbar_init(done, 1);
+    mbar_init(wfull, 1);
+    mbar_init(wempty, 4);
     fence_mbarrier_init();
   }
   if (warp == 1) {
@@ -229,28 +315,14 @@ __global__ void __launch_bounds__(kDrThreads, 1)
   pdl_wait();  // the records, the split operands and d_R's previous readers are done
 
   if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------------ TMA producer (R, B, d_y)
     if (lane == 0) {
-      int64_t it = 0, nbl = 0, na = 0, ng = 0, cur_tt = -1, cur_g = -1;
+      int64_t it = 0, nbl = 0, ng = 0, cur_g = -1;
       bool ok = true;
       for (int64_t w = lo; w < hi && ok; ++w) {
-        const int64_t tt = w / per_tt;
-        const int64_t rem = w - tt * per_tt;
-        const int64_t hc = rem >> 2;
-        const int64_t i = rem & 3;
+        const DrwItem d = drw_item(a, w);
         const int64_t g = w >> 2;
-        const int y = static_cast<int>(tt * kDrM);
-        if (tt != cur_tt) {
-          if (na > 0 && !mbar_wait(afree, static_cast<uint32_t>(na - 1) & 1u, 90)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(abar, kDrOpTile);
-          tma_load_2d(sA, &tmA, 0, y, abar);
-          tma_load_2d(sA + kDrAtom, &tmA16, 64, y, abar);
-          ++na;
-          cur_tt = tt;
-        }
+        const int y = static_cast<int>(d.tt * kDrM);
         if (g != cur_g) {
           const int gb = static_cast<int>(ng & 1);
           if (ng >= 2 &&
@@ -258,16 +330,16 @@ __global__ void __launch_bounds__(kDrThreads, 1)
             ok = false;
             break;
           }
-          uint8_t* d = sDy + gb * kDrTile;
+          uint8_t* dd = sDy + gb * kDrTile;
           mbar_arrive_expect_tx(&dyfull[gb], kDrTile);
-          tma_load_2d(d, &tmDy, static_cast<int>(hc * kDrN), y, &dyfull[gb]);
-          tma_load_2d(d + kDrAtom, &tmDy, static_cast<int>(hc * kDrN + 64), y, &dyfull[gb]);
+          tma_load_2d(dd, &tmDy, static_cast<int>(d.hc * kDrN), y, &dyfull[gb]);
+          tma_load_2d(dd + kDrAtom, &tmDy, static_cast<int>(d.hc * kDrN + 64), y, &dyfull[gb]);
           ++ng;
           cur_g = g;
         }
-        const int k0 = static_cast<int>(i * a.H + hc * kDrN);
+        const int k0 = static_cast<int>(d.i * a.H + d.hc * kDrN);
         // R first (the HBM stream; the ring slot is free once the item three back is stored),
-        // then B (one buffer: free once the previous item's MMAs have read it).
+        // then B (free once the MMAs two items back have read it).
         const int rs = static_cast<int>(it % kDrRSlots);
         if (it >= kDrRSlots &&
             !mbar_wait(&rempty[rs], static_cast<uint32_t>((it - kDrRSlots) / kDrRSlots) & 1u, 92)) {
@@ -302,34 +374,47 @@ __global__ void __launch_bounds__(kDrThreads, 1)
             mbar_wait(&bfull[k % kDrBSlots], static_cast<uint32_t>(k / kDrBSlots) & 1u, 93);
         if (ng > 0) mbar_wait(&dyfull[(ng - 1) & 1], static_cast<uint32_t>((ng - 1) >> 1) & 1u, 93);
         if (ng > 1) mbar_wait(&dyfull[(ng - 2) & 1], static_cast<uint32_t>((ng - 2) >> 1) & 1u, 93);
-        if (na > 0) mbar_wait(abar, static_cast<uint32_t>(na - 1) & 1u, 93);
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------------ MMA issuer (+ A loads)
     if (lane == 0) {
-      int64_t it = 0, na = 0, cur_tt = -1;
+      int64_t it = 0, na_issued = 0, na = 0, nad = 0, cur_tt = -1, pc = 0, cur_u0 = -1;
+      uint32_t started = 0;  // streams whose d_hc_fn accumulator this piece has begun
       bool ok = true;
+      auto load_a = [&](int64_t tt) {
+        mbar_arrive_expect_tx(abar, kDrOpTile);
+        tma_load_2d(sA, &tmA, 0, static_cast<int>(tt * kDrM), abar);
+        tma_load_2d(sA + kDrAtom, &tmA16, 64, static_cast<int>(tt * kDrM), abar);
+        ++na_issued;
+      };
+      if (lo < hi) load_a(drw_item(a, lo).tt);
       for (int64_t w = lo; w < hi && ok; ++w) {
-        const int64_t tt = w / per_tt;
-        if (tt != cur_tt) {
-          if (na > 0) {  // every MMA on the previous A has finished before the producer reloads it
-            umma_commit(adone);
-            if (!mbar_wait(adone, static_cast<uint32_t>(na - 1) & 1u, 94)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive(afree);
-          }
+        const DrwItem d = drw_item(a, w);
+        if (d.tt != cur_tt) {
           if (!mbar_wait(abar, static_cast<uint32_t>(na) & 1u, 95)) {
             ok = false;
             break;
           }
           ++na;
-          cur_tt = tt;
+          cur_tt = d.tt;
         }
+        if (d.u0 != cur_u0) {  // a new piece: the previous piece's accumulators have been read
+          if (pc > 0 && !mbar_wait(wempty, static_cast<uint32_t>(pc - 1) & 1u, 103)) {
+            ok = false;
+            break;
+          }
+          started = 0;
+          cur_u0 = d.u0;
+          ++pc;
+        }
+        const int rs = static_cast<int>(it % kDrRSlots);
         const int b = static_cast<int>(it & 1);
         const int bs = static_cast<int>(it % kDrBSlots);
+        if (!mbar_wait(&rfull[rs], static_cast<uint32_t>(it / kDrRSlots) & 1u, 104)) {
+          ok = false;
+          break;
+        }
         if (!mbar_wait(&bfull[bs], static_cast<uint32_t>(it / kDrBSlots) & 1u, 96)) {
           ok = false;
           break;
@@ -341,15 +426,42 @@ __global__ void __launch_bounds__(kDrThreads, 1)
         tc_fence_after();
         const uint32_t aaddr = smem_u32(sA);
         const uint32_t baddr = smem_u32(sB + bs * kDrOpTile);
+        const uint32_t raddr = smem_u32(sRr + rs * kDrTile);
+        // d_hc_fn of stream i: D_i[k][n] += sum_t R[t][k] A[t][n] over the tile's 128 tokens
+        // (A = R MN-major, M = 128 columns k; B = the A tile's first 64 split columns, MN-major).
+        const uint32_t dw = tmem + static_cast<uint32_t>(kDrwCol0 + kDrwN * d.i);
+        const uint32_t first = (started >> d.i) & 1u;
+#pragma unroll
+        for (int k = 0; k < kDrM / 16; ++k)  // 16 tokens: +2 KB in both operands
+          drw_umma(dw, drw_mn_desc(raddr) + 128 * k, drw_mn_desc(aaddr) + 128 * k,
+                   (first != 0u || k > 0) ? 1u : 0u);
+        started |= 1u << d.i;
+        // d_R's contraction.
         const uint32_t dt = tmem + static_cast<uint32_t>(b * kDrN);
 #pragma unroll
         for (int k = 0; k < 4; ++k)  // split columns 0..63: +32 bytes along the row per step
           dr_umma(dt, sw128_desc(aaddr) + 2 * k, sw128_desc(baddr) + 2 * k, k > 0 ? 1u : 0u);
         dr_umma(dt, sw32_desc(aaddr + kDrAtom), sw32_desc(baddr + kDrAtom), 1u);  // 64..79
         umma_commit(&bempty[bs]);  // B read: the slot may take a later item's B
-        umma_commit(&afull[b]);
+        umma_commit(&afull[b]);    // also covers the d_hc_fn MMAs that read the R slot
         ++it;
+        if (w == d.u1 || w + 1 == hi) umma_commit(wfull);  // the piece's accumulators
+        // The next item needs another token tile: reload A once these MMAs have read it.
+        if (w + 1 < hi) {
+          const int64_t ntt = drw_item(a, w + 1).tt;
+          if (ntt != d.tt) {
+            umma_commit(adone);
+            if (!mbar_wait(adone, static_cast<uint32_t>(nad) & 1u, 94)) {
+              ok = false;
+              break;
+            }
+            ++nad;
+            load_a(ntt);
+          }
+        }
       }
+      // Do not leave while an A load is in flight.
+      if (!ok && na_issued > na) mbar_wait(abar, static_cast<uint32_t>(na) & 1u, 93);
       umma_commit(done);  // every issued MMA has finished before TMEM is released
       mbar_wait(done, 0, 98);
     }
@@ -357,12 +469,11 @@ __global__ void __launch_bounds__(kDrThreads, 1)
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter
     const int row = q * 32 + lane;
-    int64_t it = 0, ng = 0, cur_g = -1;
+    int64_t it = 0, ng = 0, cur_g = -1, pc = 0;
     int gb = 0;
     uint32_t gph = 0;
     for (int64_t w = lo; w < hi; ++w) {
-      const int64_t tt = w / per_tt;
-      const int64_t i = (w - tt * per_tt) & 3;
+      const DrwItem d = drw_item(a, w);
       const int64_t g = w >> 2;
       if (g != cur_g) {
         if (cur_g >= 0) {  // this warp is done with the previous group's d_y buffer
@@ -385,11 +496,11 @@ __global__ void __launch_bounds__(kDrThreads, 1)
       // The four warps agree on going on (a stop keeps the named-barrier sequence matched).
       if (named_bar_or(1, 128, !ok)) break;
       tc_fence_after();
-      const int64_t tok = tt * kDrM + row;
+      const int64_t tok = d.tt * kDrM + row;
       float dss2 = 0.f, pi = 0.f;
       if (tok < a.T) {
         dss2 = 2.0f * __ldg(a.brec + tok * a.rec_stride + 24);
-        pi = __ldg(a.brec + tok * a.rec_stride + 25 + i);
+        pi = __ldg(a.brec + tok * a.rec_stride + 25 + d.i);
       }
       uint8_t* sR = sRr + rs * kDrTile;
       const uint8_t* sY = sDy + gb * kDrTile;
@@ -436,21 +547,64 @@ __global__ void __launch_bounds__(kDrThreads, 1)
         mbar_arrive(&drready[rs]);
       }
       ++it;
+      if (w != d.u1 && w + 1 != hi) continue;
+      // ---- the piece's end: d_hc_fn partials of its four streams, thread = column k of the
+      // block (TMEM lane), into slot (this CTA's rank among the unit's CTAs) of chunk d.ck.
+      ok = __all_sync(0xffffffffu, mbar_wait(wfull, static_cast<uint32_t>(pc) & 1u, 105));
+      if (named_bar_or(1, 128, !ok)) break;
+      tc_fence_after();
+      const int64_t ps = lo > d.u0 ? lo : d.u0;
+      const int64_t n = w - ps + 1;  // the piece's items ps..w
+      const int64_t slot = static_cast<int64_t>(blockIdx.x) - tc_first_cta(d.u0, P, a.W);
+      const int64_t K = 4 * a.H;
+      for (int s = 0; s < 4; ++s) {
+        // Stream s has an item in the piece iff its first position after ps is within n.
+        const bool present = ((s - static_cast<int>(ps & 3)) & 3) < n;
+        float v[kMix];
+        if (present) {
+          uint32_t dd[3][16];
+          const uint32_t wb = tmem + static_cast<uint32_t>(kDrwCol0 + kDrwN * s) +
+                              (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll
+          for (int cc = 0; cc < 3; ++cc) tmem_ld16(wb + cc * 16, dd[cc]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < kMix; ++j)  // columns j: R.hi(d_raw_j), 24 + j: R.lo(d_raw_j)
+            v[j] = __uint_as_float(dd[(kMix + j) / 16][(kMix + j) % 16]) +
+                   __uint_as_float(dd[j / 16][j % 16]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < kMix; ++j) v[j] = 0.f;
+        }
+        const int64_t k = s * a.H + d.hc * kDrN + row;
+        float4* dst = reinterpret_cast<float4*>(a.dwp + ((d.ck * a.S + slot) * K + k) * kMix);
+#pragma unroll
+        for (int w4 = 0; w4 < kMix / 4; ++w4)
+          dst[w4] = make_float4(v[4 * w4], v[4 * w4 + 1], v[4 * w4 + 2], v[4 * w4 + 3]);
+        if (w == d.u1) {  // the unit's last piece: zero its unused slots
+          for (int64_t sl = slot + 1; sl < a.S; ++sl) {
+            float4* z = reinterpret_cast<float4*>(a.dwp + ((d.ck * a.S + sl) * K + k) * kMix);
+#pragma unroll
+            for (int w4 = 0; w4 < kMix / 4; ++w4) z[w4] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(wempty);
+      ++pc;
     }
   } else if (warp == 6) {
     // ------------------------------------------------------------------ d_R storer
     if (lane == 0) {
       int64_t it = 0;
       for (int64_t w = lo; w < hi; ++w, ++it) {
-        const int64_t tt = w / per_tt;
-        const int64_t rem = w - tt * per_tt;
-        const int64_t hc = rem >> 2;
-        const int64_t i = rem & 3;
+        const DrwItem d = drw_item(a, w);
         const int rs = static_cast<int>(it % kDrRSlots);
         if (!mbar_wait(&drready[rs], static_cast<uint32_t>(it / kDrRSlots) & 1u, 102)) break;
         const uint8_t* sR = sRr + rs * kDrTile;
-        const int x = static_cast<int>(i * a.H + hc * kDrN);
-        const int y = static_cast<int>(tt * kDrM);
+        const int x = static_cast<int>(d.i * a.H + d.hc * kDrN);
+        const int y = static_cast<int>(d.tt * kDrM);
         tma_store_2d(&tmDR, x, y, sR);
         tma_store_2d(&tmDR, x + 64, y, sR + kDrAtom);
         asm volatile("cp.async.bulk.commit_group;" ::: "memory");
@@ -793,19 +947,23 @@ int launch_pre_bwd_dw_tc(const uint16_t* R, const float* brec, int rec_stride, f
   return 0;
 }
 
-// Returns 0, a negative MHC_ERR_* code, or 1 when this form cannot run (nothing launched).
+// d_R and d_hc_fn on tensor cores: the split operands, the fused kernel, the partials' in-order
+// sum. Returns 0, a negative MHC_ERR_* code, or 1 when this form cannot run (nothing launched).
 int launch_pre_bwd_dr_tc(const uint16_t* R, const uint16_t* dy, const float* hc_fn,
-                         const float* brec, int rec_stride, uint16_t* dR, void* ws, int64_t T,
-                         int64_t H, cudaStream_t s) {
+                         const float* brec, int rec_stride, uint16_t* dR, float* dW, void* ws,
+                         int64_t T, int64_t H, cudaStream_t s) {
   if (!pre_bwd_dr_tc_supported(T, H) || dy == nullptr || !aligned16(R) || !aligned16(dy) ||
       !aligned16(dR) || !aligned16(ws))
     return 1;
-  if (!ensure_smem_limit(reinterpret_cast<const void*>(pre_bwd_dr_kernel), kDrSmem)) return 1;
+  if (!ensure_smem_limit(reinterpret_cast<const void*>(pre_bwd_drw_kernel), kDrSmem)) return 1;
   const int64_t K = 4 * H;
+  const DrPlan plan = dr_plan(T, H, device_sm_count());
+  auto up = [](size_t v) { return (v + 1023) / 1024 * 1024; };
   uint8_t* w8 = static_cast<uint8_t*>(ws);
   uint16_t* A = reinterpret_cast<uint16_t*>(w8);
-  uint16_t* B = reinterpret_cast<uint16_t*>(
-      w8 + (static_cast<size_t>(T) * kDrKd * 2 + 1023) / 1024 * 1024);
+  uint16_t* B = reinterpret_cast<uint16_t*>(w8 + up(static_cast<size_t>(T) * kDrKd * 2));
+  float* dwp = reinterpret_cast<float*>(w8 + up(static_cast<size_t>(T) * kDrKd * 2) +
+                                        up(static_cast<size_t>(K) * kDrKd * 2));
   CUtensorMap mA, mB, mA16, mB16, mR, mDy, mDR;
   // [rows x 16] boxes of columns 64..79, 32-byte swizzle.
   auto narrow_map = [](CUtensorMap* m, const void* base, int64_t rows) {
@@ -831,20 +989,26 @@ int launch_pre_bwd_dr_tc(const uint16_t* R, const uint16_t* dy, const float* hc_
     return -4;
   DrArgs da;
   da.brec = brec;
+  da.dwp = dwp;
   da.T = T;
   da.H = H;
-  da.ntt = (T + kDrM - 1) / kDrM;
-  da.nhc = H / kDrN;
-  da.W = da.ntt * da.nhc * 4;
+  da.ntt = plan.ntt;
+  da.nhc = plan.nhc;
+  da.W = plan.W;
+  da.nck = plan.nck;
   da.rec_stride = rec_stride;
-  int P = device_sm_count();
-  if (P > 148) P = 148;
-  if (static_cast<int64_t>(P) > da.W) P = static_cast<int>(da.W);
-  if (launch_pdl(pre_bwd_dr_kernel, dim3(static_cast<unsigned>(P)), dim3(kDrThreads),
+  da.S = static_cast<int>(plan.S);
+  if (launch_pdl(pre_bwd_drw_kernel, dim3(static_cast<unsigned>(plan.P)), dim3(kDrThreads),
                  static_cast<size_t>(kDrSmem), s, mA, mB, mA16, mB16, mR, mDy, mDR, da) !=
       cudaSuccess)
     return -4;
-  note_launches(2);
+  int64_t sb = (K * kMix + 255) / 256;
+  if (sb > 148 * 8) sb = 148 * 8;
+  if (launch_pdl(pre_bwd_dw_sum_kernel, dim3(static_cast<unsigned>(sb)), dim3(256), 0, s,
+                 static_cast<const float*>(dwp), dW, K * kMix,
+                 static_cast<int>(plan.nck * plan.S)) != cudaSuccess)
+    return -4;
+  note_launches(3);
   return 0;
 }
 

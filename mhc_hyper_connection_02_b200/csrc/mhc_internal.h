@@ -165,14 +165,14 @@ struct PreBwdArgs {
   float post_mult;
 };
 size_t pre_backward_workspace_bytes(int64_t T, int64_t H);
-// d_R of the pre-map backward on tensor cores (mhc_backward_tc.cu): 0, a negative MHC_ERR_* code,
-// or 1 when this form cannot run the shape (nothing launched).
+// d_R and d_hc_fn of the pre-map backward on tensor cores in one pass over R (mhc_backward_tc.cu):
+// 0, a negative MHC_ERR_* code, or 1 when this form cannot run the shape (nothing launched).
 bool pre_bwd_dr_tc_supported(int64_t T, int64_t H);
 size_t pre_bwd_dr_tc_workspace_bytes(int64_t T, int64_t H);
 int launch_pre_bwd_dr_tc(const uint16_t* R, const uint16_t* dy, const float* hc_fn,
-                         const float* brec, int rec_stride, uint16_t* dR, void* ws, int64_t T,
-                         int64_t H, cudaStream_t s);
-// d_hc_fn of the pre-map backward on tensor cores: same return convention.
+                         const float* brec, int rec_stride, uint16_t* dR, float* dW, void* ws,
+                         int64_t T, int64_t H, cudaStream_t s);
+// d_hc_fn alone on tensor cores (where the fused form cannot run): same return convention.
 bool pre_bwd_dw_tc_supported(int64_t T, int64_t H);
 size_t pre_bwd_dw_tc_workspace_bytes(int64_t T, int64_t H);
 int launch_pre_bwd_dw_tc(const uint16_t* R, const float* brec, int rec_stride, float* dW,

@@ -42,7 +42,7 @@ CASES = {
     "head_mean_scalar_H1001": ("mhc_head_mean T=8192 H=1001", "head_mean_scalar_kernel"),
     "pre_backward_H1001": ("mhc_pre_backward T=4096 H=1001", "pre_bwd_* (dx scalar form)"),
     "pre_backward_large": ("mhc_pre_backward T=8192 H=7168",
-                           "pre_bwd_* (d_R on tensor cores: pre_bwd_split_kernel, pre_bwd_dr_kernel)"),
+                           "pre_bwd_* (d_R with d_hc_fn on tensor cores: pre_bwd_split_kernel, pre_bwd_drw_kernel)"),
 }
 
 

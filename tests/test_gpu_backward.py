@@ -76,7 +76,7 @@ def _pre_case(T, H, seed, with_dy=True, with_comb=True):
 
 @pytest.mark.parametrize("T,H", [(1, 8), (5, 127), (64, 512), (130, 1000), (300, 2048),
                                  (20, 7168), (3, 1001), (1000, 1024), (513, 4096), (777, 256),
-                                 (200, 1056), (3000, 64)])
+                                 (200, 1056), (3000, 64), (9000, 128)])
 def test_pre_backward(T, H):
     w, d_y, d_pre, d_post, d_comb = _pre_case(T, H, seed=7 * T + H)
     prm = mhc.make_params(iters=w.iters, eps=w.eps, rms_eps=w.rms_eps, pre_eps=w.pre_eps,
@@ -109,9 +109,10 @@ def test_pre_backward(T, H):
                                                             (130, 1000, False, False, False),
                                                             (200, 1056, False, True, False)])
 def test_pre_backward_d_R_form(T, H, dr_tensor, dw_tensor, dy_fold):
-    """H % 128 == 0 with d_y given takes the tcgen05 d_R (split operands + the tensor kernel: two
-    launches), otherwise the CUDA-core kernel (one); 4H % 128 == 0 takes the tcgen05 d_hc_fn
-    (transposed d_raw split, the tensor kernel, the partials' sum: three launches), otherwise
+    """H % 128 == 0 with d_y given takes the tcgen05 kernel that forms d_R and d_hc_fn in one
+    pass over R (split operands, the tensor kernel, the d_hc_fn partials' sum: three launches);
+    otherwise d_R runs on CUDA cores (one) and d_hc_fn on its own: where 4H % 128 == 0 the tcgen05
+    d_hc_fn (transposed d_raw split, the tensor kernel, the partials' sum: three launches), else
     CUDA-core partials and their sum (two). The projections here are the tensor form (split +
     projection); with H % 64 == 0 it also forms d_pre's d_y term, otherwise a d_pre kernel runs;
     then coefficients and parameters."""
@@ -122,8 +123,8 @@ def test_pre_backward_d_R_form(T, H, dr_tensor, dw_tensor, dy_fold):
                      d_comb=dev_f32(d_comb), params=mhc.make_params(iters=w.iters))
     torch.cuda.synchronize()
     assert mhc.device_status() == 0
-    assert mhc.launch_count() - n0 == (2 + (2 if dy_fold else 3) + (2 if dr_tensor else 1) +
-                                       (3 if dw_tensor else 2))
+    grads = 3 if dr_tensor else 1 + (3 if dw_tensor else 2)
+    assert mhc.launch_count() - n0 == 2 + (2 if dy_fold else 3) + grads
 
 
 def test_pre_backward_optional_gradients_and_tensor_path():
