@@ -40,6 +40,7 @@ CASES = {
                             "pre_bigfuse_coef_kernel, pre_bigfuse_loop_kernel"),
     "expand_scalar_H1001": ("mhc_expand T=8192 H=1001", "expand_scalar_kernel"),
     "head_mean_scalar_H1001": ("mhc_head_mean T=8192 H=1001", "head_mean_scalar_kernel"),
+    "post_backward_large": ("mhc_post_backward T=8192 H=7168", "post_bwd_persistent_kernel"),
     "pre_backward_H1001": ("mhc_pre_backward T=4096 H=1001", "pre_bwd_* (dx scalar form)"),
     "pre_backward_large": ("mhc_pre_backward T=8192 H=7168",
                            "pre_bwd_* (d_R with d_hc_fn on tensor cores: pre_bwd_split_kernel, pre_bwd_drw_kernel)"),
@@ -70,7 +71,8 @@ def make_call(case):
     import torch
     from . import (PRE_PATH_TENSOR_FUSED, PRE_PATH_TENSOR_SPLIT, PRE_PATH_TENSOR_WAVE,
                    POST_PATH_SCALAR, expand,
-                   head_mean, post, pre, pre_backward, pre_big_fuse, sinkhorn, workspace_bytes)
+                   head_mean, post, post_backward, pre, pre_backward, pre_big_fuse, sinkhorn,
+                   workspace_bytes)
 
     def pre_call(T, H, path=0):
         _, R, _, W, S, B = _inputs(T, H)
@@ -126,6 +128,12 @@ def make_call(case):
         _, R, _, _, _, _ = _inputs(8192, 1001)
         y = torch.empty((8192, 1001), dtype=torch.bfloat16, device="cuda")
         return lambda: head_mean(R, y=y)
+    if case == "post_backward_large":
+        T, H = 8192, 7168
+        g, R, x, _, _, _ = _inputs(T, H)
+        pc, cc = _coefficients(g, T)
+        dout = torch.randn((T, 4, H), device="cuda", generator=g).to(torch.bfloat16)
+        return lambda: post_backward(dout, x, R, pc, cc)
     if case in ("pre_backward_H1001", "pre_backward_large"):
         T, H = (4096, 1001) if case == "pre_backward_H1001" else (8192, 7168)
         g, R, x, W, S, B = _inputs(T, H)

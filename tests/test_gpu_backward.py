@@ -39,7 +39,7 @@ def _check_sum(gpu, ref, terms_abs, rel, name):
 
 
 @pytest.mark.parametrize("T,H", [(1, 8), (5, 127), (64, 512), (33, 1000), (16, 7168),
-                                 (3, 16392)])
+                                 (3, 16392), (1000, 1032), (500, 3000)])
 def test_post_backward(T, H):
     w = inputs.custom(T, H, seed=11 * T + H)
     post, comb = post_coefficients(w)
