@@ -17,8 +17,8 @@
 //      and the reverse pass -> d_raw, d_ss, the gates, and the per-token terms of d_scale, d_base;
 //   4. d_scale, d_base: fixed-order sums over tokens;
 //   5. d_R = d_raw . hc_fn^T + 2 R d_ss + pre_i d_y: on tcgen05 tensor cores where H % 128 == 0
-//      and d_y is given (mhc_backward_tc.cu), else column slice x token chunk per CTA, a thread's
-//      hc_fn weights in registers, fp32 on CUDA cores;
+//      (mhc_backward_tc.cu, with d_hc_fn in the same pass over R), else column slice x token
+//      chunk per CTA, a thread's hc_fn weights in registers, fp32 on CUDA cores;
 //   6. d_hc_fn = R_flat^T d_raw: on tcgen05 where 4H % 128 == 0 (mhc_backward_tc.cu: R read
 //      MN-major as the A operand), else column slice x token chunk per CTA on CUDA cores; the
 //      partials are summed in order.
@@ -981,7 +981,7 @@ int launch_pre_backward(const PreBwdArgs& a, cudaStream_t s) {
   // nothing launched), else column slices x token chunks on CUDA cores, one wave of
   // kDxSlotsPerSm CTAs per SM.
   int dr = 1;
-  if (vec && a.dy != nullptr) {
+  if (vec) {
     dr = launch_pre_bwd_dr_tc(a.R, a.dy, a.hc_fn, static_cast<const float*>(brec), kBrec, a.dR,
                               a.dW, drtc_ws, a.T, a.H, s);
     if (dr < 0) return dr;

@@ -39,7 +39,8 @@
 //   warp 6      stores each finished d_R tile with a TMA bulk-tensor store and releases its R slot
 //               once the store has read it (the epilogue warps go on to the next item meanwhile).
 // Every wait is bounded; copies in flight are drained and stores completed before exit.
-// Requires H % 128 == 0, d_y present, 16-byte aligned R, d_y, d_R and workspace.
+// Requires H % 128 == 0, 16-byte aligned R, d_y (when given; absent, its term is zero and no d_y
+// tile is loaded), d_R and workspace.
 // The TMA, descriptor, MMA and TMEM helpers and the tensor-map encoder are mhc_pre_tc.cu's (same
 // translation unit).
 #include <cuda.h>
@@ -203,6 +204,7 @@ struct DrArgs {
   float* dwp;  // d_hc_fn partials [nck * S][4H][24]
   int64_t T, H, ntt, nhc, W, nck;
   int rec_stride, S;
+  int has_dy;  // 0: d_y absent (zero), no d_y tiles are loaded
 };
 
 // Item w of the flattened list: chunk ck of kDrwChunk token tiles (slowest), column block hc,
@@ -323,7 +325,7 @@ __global__ void __launch_bounds__(kDrThreads, 1)
         const DrwItem d = drw_item(a, w);
         const int64_t g = w >> 2;
         const int y = static_cast<int>(d.tt * kDrM);
-        if (g != cur_g) {
+        if (a.has_dy && g != cur_g) {
           const int gb = static_cast<int>(ng & 1);
           if (ng >= 2 &&
               !mbar_wait(&dyempty[gb], static_cast<uint32_t>((ng - 2) >> 1) & 1u, 91)) {
@@ -490,7 +492,7 @@ __global__ void __launch_bounds__(kDrThreads, 1)
       bool ok = __all_sync(
           0xffffffffu,
           mbar_wait(&rfull[rs], static_cast<uint32_t>(it / kDrRSlots) & 1u, 99));
-      ok = ok && __all_sync(0xffffffffu, mbar_wait(&dyfull[gb], gph, 100));
+      ok = ok && (!a.has_dy || __all_sync(0xffffffffu, mbar_wait(&dyfull[gb], gph, 100)));
       ok = ok && __all_sync(0xffffffffu,
                             mbar_wait(&afull[b], static_cast<uint32_t>(it >> 1) & 1u, 101));
       // The four warps agree on going on (a stop keeps the named-barrier sequence matched).
@@ -522,7 +524,8 @@ __global__ void __launch_bounds__(kDrThreads, 1)
             const int c = (cq & 1) * 4 + u;
             const int off = atom * kDrAtom + row * 128 + ((c ^ (row & 7)) << 4);
             const uint4 rv = *reinterpret_cast<const uint4*>(sR + off);
-            const uint4 yv = *reinterpret_cast<const uint4*>(sY + off);
+            const uint4 yv =
+                a.has_dy ? *reinterpret_cast<const uint4*>(sY + off) : make_uint4(0u, 0u, 0u, 0u);
             const uint32_t r4[4] = {rv.x, rv.y, rv.z, rv.w};
             const uint32_t y4[4] = {yv.x, yv.y, yv.z, yv.w};
             uint32_t o[4];
@@ -952,7 +955,7 @@ int launch_pre_bwd_dw_tc(const uint16_t* R, const float* brec, int rec_stride, f
 int launch_pre_bwd_dr_tc(const uint16_t* R, const uint16_t* dy, const float* hc_fn,
                          const float* brec, int rec_stride, uint16_t* dR, float* dW, void* ws,
                          int64_t T, int64_t H, cudaStream_t s) {
-  if (!pre_bwd_dr_tc_supported(T, H) || dy == nullptr || !aligned16(R) || !aligned16(dy) ||
+  if (!pre_bwd_dr_tc_supported(T, H) || !aligned16(R) || (dy != nullptr && !aligned16(dy)) ||
       !aligned16(dR) || !aligned16(ws))
     return 1;
   if (!ensure_smem_limit(reinterpret_cast<const void*>(pre_bwd_drw_kernel), kDrSmem)) return 1;
@@ -979,8 +982,11 @@ int launch_pre_bwd_dr_tc(const uint16_t* R, const uint16_t* dy, const float* hc_
   };
   if (!make_map(&mA, A, kDrKd, T, kDrM) || !make_map(&mB, B, kDrKd, K, kDrN) ||
       !narrow_map(&mA16, A, T) || !narrow_map(&mB16, B, K) ||
-      !make_map(&mR, R, K, T, kDrM) || !make_map(&mDy, dy, H, T, kDrM) ||
-      !make_map(&mDR, dR, K, T, kDrM))
+      !make_map(&mR, R, K, T, kDrM) || !make_map(&mDR, dR, K, T, kDrM))
+    return -4;
+  if (dy == nullptr)
+    mDy = mR;  // not read: no d_y tile is loaded
+  else if (!make_map(&mDy, dy, H, T, kDrM))
     return -4;
   int64_t nb = (T + K + 255) / 256;
   if (nb > 148 * 8) nb = 148 * 8;
@@ -998,6 +1004,7 @@ int launch_pre_bwd_dr_tc(const uint16_t* R, const uint16_t* dy, const float* hc_
   da.nck = plan.nck;
   da.rec_stride = rec_stride;
   da.S = static_cast<int>(plan.S);
+  da.has_dy = dy != nullptr ? 1 : 0;
   if (launch_pdl(pre_bwd_drw_kernel, dim3(static_cast<unsigned>(plan.P)), dim3(kDrThreads),
                  static_cast<size_t>(kDrSmem), s, mA, mB, mA16, mB16, mR, mDy, mDR, da) !=
       cudaSuccess)

@@ -128,13 +128,18 @@ def test_pre_backward_d_R_form(T, H, dr_tensor, dw_tensor, dy_fold):
 
 
 def test_pre_backward_optional_gradients_and_tensor_path():
-    """T = 256 takes the tensor-core projection; d_y and d_comb absent (zero)."""
+    """T = 256 takes the tensor-core projection; d_y and d_comb absent (zero). Without d_y the
+    projection does not form d_pre's term (a d_pre kernel runs), and d_R with d_hc_fn still takes
+    the tensor kernel (no d_y tiles): 2 + 3 + 3 launches."""
     w, _, d_pre, d_post, _ = _pre_case(256, 512, seed=3, with_dy=False, with_comb=False)
+    n0 = mhc.launch_count()
     dR, dW, ds, db = mhc.pre_backward(dev_bf16(w.R), dev_f32(w.hc_fn), dev_f32(w.hc_scale),
                                       dev_f32(w.hc_base), d_pre=dev_f32(d_pre),
                                       d_post=dev_f32(d_post),
                                       params=mhc.make_params(iters=w.iters))
     torch.cuda.synchronize()
+    assert mhc.device_status() == 0
+    assert mhc.launch_count() - n0 == 8
     rR, rW, rs, rb, pt = backward.pre_backward(None, d_pre, d_post, None, w.R, w.hc_fn, w.hc_scale,
                                                w.hc_base, iters=w.iters, parts=True)
     Wa = np.abs(w.hc_fn.astype(np.float64))
