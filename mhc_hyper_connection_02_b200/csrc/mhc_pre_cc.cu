@@ -231,6 +231,17 @@ __global__ void __launch_bounds__(256) pre_cc_partial_staged_kernel(const uint16
   const int64_t kb = s * KS;
   const int64_t ke = min(K, kb + KS);
   const int nw = static_cast<int>((ke - kb) * kMix);
+  const int64_t KW = KS / kCcWarps;  // multiple of 8
+  const int64_t k0 = kb + warp * KW;
+  const int64_t k1 = min(ke, k0 + KW);
+  const int64_t t = lane;
+  // The lane's row values are loaded before the W slice is staged, so both round trips overlap.
+  constexpr int kStVec = kStMaxKS / kCcWarps / 8;  // 16-byte chunks per lane at most
+  uint4 rq[kStVec];
+#pragma unroll
+  for (int q = 0; q < kStVec; ++q)
+    rq[q] = (kVecR && t < T && k0 + 8 * q + 8 <= k1) ? ld_stream_ro(R + t * K + k0 + 8 * q)
+                                                      : make_uint4(0u, 0u, 0u, 0u);
   if (kAlignedW) {
     const float4* src = reinterpret_cast<const float4*>(W + kb * kMix);
     for (int i = threadIdx.x; i < nw / 4; i += blockDim.x)
@@ -239,10 +250,6 @@ __global__ void __launch_bounds__(256) pre_cc_partial_staged_kernel(const uint16
     for (int i = threadIdx.x; i < nw; i += blockDim.x) sm[i] = __ldg(W + kb * kMix + i);
   }
   __syncthreads();
-  const int64_t KW = KS / kCcWarps;  // multiple of 8
-  const int64_t k0 = kb + warp * KW;
-  const int64_t k1 = min(ke, k0 + KW);
-  const int64_t t = lane;
   float acc[kMix];
 #pragma unroll
   for (int j = 0; j < kMix; ++j) acc[j] = 0.f;
@@ -263,14 +270,16 @@ __global__ void __launch_bounds__(256) pre_cc_partial_staged_kernel(const uint16
     const uint16_t* row = R + t * K;
     int64_t k = k0;
     if (kVecR) {
-      for (; k + 8 <= k1; k += 8) {
-        const uint4 v = ld_stream_ro(row + k);
-        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < kStVec; ++q) {
+        if (k + 8 > k1) break;
+        const uint32_t u[4] = {rq[q].x, rq[q].y, rq[q].z, rq[q].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           add_row(bf16_lo(u[e]), k + 2 * e);
           add_row(bf16_hi(u[e]), k + 2 * e + 1);
         }
+        k += 8;
       }
     }
     for (; k < k1; ++k) add_row(bf16_to_f32(row[k]), k);
@@ -335,6 +344,28 @@ __device__ __forceinline__ void finish_coefficients(float tot, int64_t t, int64_
   }
 }
 
+// Eight columns of y = bf16_rn(sum_i pre_i R_i) from the four streams' 16-byte chunks.
+__device__ __forceinline__ uint4 agg8(const uint4 (&r)[4], const float (&p)[4]) {
+  uint32_t o[4];
+  const uint32_t* r0 = &r[0].x;
+  const uint32_t* r1 = &r[1].x;
+  const uint32_t* r2 = &r[2].x;
+  const uint32_t* r3 = &r[3].x;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    float lo = p[0] * bf16_lo(r0[e]);
+    lo = fmaf(p[1], bf16_lo(r1[e]), lo);
+    lo = fmaf(p[2], bf16_lo(r2[e]), lo);
+    lo = fmaf(p[3], bf16_lo(r3[e]), lo);
+    float hi = p[0] * bf16_hi(r0[e]);
+    hi = fmaf(p[1], bf16_hi(r1[e]), hi);
+    hi = fmaf(p[2], bf16_hi(r2[e]), hi);
+    hi = fmaf(p[3], bf16_hi(r3[e]), hi);
+    o[e] = pack_bf16x2(lo, hi);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 // y[t][h0..h0+8) = bf16_rn(sum_i pre_i * R[t][i][..]) for the columns this thread owns.
 template <bool kVec>
 __device__ __forceinline__ void aggregate_cols(const uint16_t* __restrict__ R,
@@ -347,24 +378,7 @@ __device__ __forceinline__ void aggregate_cols(const uint16_t* __restrict__ R,
       uint4 r[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) r[i] = ld_stream_ro(rr + i * H + h);
-      uint32_t o[4];
-      const uint32_t* r0 = &r[0].x;
-      const uint32_t* r1 = &r[1].x;
-      const uint32_t* r2 = &r[2].x;
-      const uint32_t* r3 = &r[3].x;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float lo = p[0] * bf16_lo(r0[e]);
-        lo = fmaf(p[1], bf16_lo(r1[e]), lo);
-        lo = fmaf(p[2], bf16_lo(r2[e]), lo);
-        lo = fmaf(p[3], bf16_lo(r3[e]), lo);
-        float hi = p[0] * bf16_hi(r0[e]);
-        hi = fmaf(p[1], bf16_hi(r1[e]), hi);
-        hi = fmaf(p[2], bf16_hi(r2[e]), hi);
-        hi = fmaf(p[3], bf16_hi(r3[e]), hi);
-        o[e] = pack_bf16x2(lo, hi);
-      }
-      st_plain(yy + h, make_uint4(o[0], o[1], o[2], o[3]));
+      st_plain(yy + h, agg8(r, p));
     }
   } else {
     for (int64_t h = c0 + threadIdx.x; h < c1; h += blockDim.x) {
@@ -390,6 +404,17 @@ __global__ void __launch_bounds__(256) pre_cc_finish_kernel(
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int64_t t = blockIdx.x;
+  // An aggregate block's thread owns one 8-column chunk (kAggCols = 256 x 8): with 16-byte access
+  // its four R chunks are loaded first, so their round trip overlaps the records'.
+  static_assert(kAggCols == 256 * 8, "one chunk per thread");
+  const int64_t c0 = blockIdx.y > 0 ? static_cast<int64_t>(blockIdx.y - 1) * kAggCols : 0;
+  const int64_t c1 = min(H, c0 + kAggCols);
+  const int64_t hh = c0 + threadIdx.x * 8;
+  const bool own = kVec && blockIdx.y > 0 && hh + 8 <= c1;
+  uint4 rq[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    rq[i] = own ? ld_stream_ro(R + t * 4 * H + i * H + hh) : make_uint4(0u, 0u, 0u, 0u);
   float v = 0.f;
   if (lane < 25) {
     // Warp w adds the records of splits w, w + 8, w + 16, ... in that order. A batch of up to
@@ -419,9 +444,11 @@ __global__ void __launch_bounds__(256) pre_cc_finish_kernel(
   __syncthreads();
   if (blockIdx.y == 0) return;
   const float p[4] = {pre_s[0], pre_s[1], pre_s[2], pre_s[3]};
-  const int64_t c0 = static_cast<int64_t>(blockIdx.y - 1) * kAggCols;
-  const int64_t c1 = min(H, c0 + kAggCols);
-  aggregate_cols<kVec>(R, y, t, H, c0, c1, p);
+  if (kVec) {
+    if (own) st_plain(y + t * H + hh, agg8(rq, p));
+  } else {
+    aggregate_cols<false>(R, y, t, H, c0, c1, p);
+  }
 }
 
 // Split-K projection partials: records [nsplit][T][32] (raw[24], ss) at the workspace start.
