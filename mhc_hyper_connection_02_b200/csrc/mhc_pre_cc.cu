@@ -404,17 +404,6 @@ __global__ void __launch_bounds__(256) pre_cc_finish_kernel(
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int64_t t = blockIdx.x;
-  // An aggregate block's thread owns one 8-column chunk (kAggCols = 256 x 8): with 16-byte access
-  // its four R chunks are loaded first, so their round trip overlaps the records'.
-  static_assert(kAggCols == 256 * 8, "one chunk per thread");
-  const int64_t c0 = blockIdx.y > 0 ? static_cast<int64_t>(blockIdx.y - 1) * kAggCols : 0;
-  const int64_t c1 = min(H, c0 + kAggCols);
-  const int64_t hh = c0 + threadIdx.x * 8;
-  const bool own = kVec && blockIdx.y > 0 && hh + 8 <= c1;
-  uint4 rq[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    rq[i] = own ? ld_stream_ro(R + t * 4 * H + i * H + hh) : make_uint4(0u, 0u, 0u, 0u);
   float v = 0.f;
   if (lane < 25) {
     // Warp w adds the records of splits w, w + 8, w + 16, ... in that order. A batch of up to
@@ -444,11 +433,9 @@ __global__ void __launch_bounds__(256) pre_cc_finish_kernel(
   __syncthreads();
   if (blockIdx.y == 0) return;
   const float p[4] = {pre_s[0], pre_s[1], pre_s[2], pre_s[3]};
-  if (kVec) {
-    if (own) st_plain(y + t * H + hh, agg8(rq, p));
-  } else {
-    aggregate_cols<false>(R, y, t, H, c0, c1, p);
-  }
+  const int64_t c0 = static_cast<int64_t>(blockIdx.y - 1) * kAggCols;
+  const int64_t c1 = min(H, c0 + kAggCols);
+  aggregate_cols<kVec>(R, y, t, H, c0, c1, p);
 }
 
 // Split-K projection partials: records [nsplit][T][32] (raw[24], ss) at the workspace start.
