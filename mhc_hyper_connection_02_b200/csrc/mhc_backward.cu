@@ -19,9 +19,9 @@
 //   5. d_R = d_raw . hc_fn^T + 2 R d_ss + pre_i d_y: on tcgen05 tensor cores where H % 128 == 0
 //      (mhc_backward_tc.cu, with d_hc_fn in the same pass over R), else column slice x token
 //      chunk per CTA, a thread's hc_fn weights in registers, fp32 on CUDA cores;
-//   6. d_hc_fn = R_flat^T d_raw: on tcgen05 where 4H % 128 == 0 (mhc_backward_tc.cu: R read
-//      MN-major as the A operand), else column slice x token chunk per CTA on CUDA cores; the
-//      partials are summed in order.
+//   6. d_hc_fn = R_flat^T d_raw, where step 5 did not form it: on tcgen05 where 4H % 128 == 0
+//      (mhc_backward_tc.cu: R read MN-major as the A operand), else column slice x token chunk
+//      per CTA on CUDA cores; the partials are summed in order.
 #include "mhc_device.cuh"
 #include "mhc_internal.h"
 
